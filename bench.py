@@ -1,0 +1,357 @@
+"""Benchmark of the MoE split-LoRA expert block, forward + backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config gpt-oss-20b]
+
+One step = route -> permute -> gate_up + SwiGLU -> down -> weighted combine ->
+weighted dY gather -> down / gate_up backward -> LoRA gradients -> dX combine,
+all through the C ABI on one stream.  Inputs are seeded synthetic tensors of
+the gpt-oss-20b-shaped layer (T = 8192 tokens, H = I = 2880, 32 experts,
+top-4, LoRA r = 16, s = 2) resident in HBM before the timed region.
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs an
+independent replica (the block has no exchange step on one layer): weak
+scaling, time = max over ranks.  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_expert_grouped_softmax_b200 import synthetic as S  # noqa: E402
+from moe_expert_grouped_softmax_b200 import workload as WL  # noqa: E402
+
+METRIC = "MoE-LoRA block fwd+bwd tokens/s and TFLOP/s (% BF16 tensor peak) on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args, cfg):
+    import torch.distributed as dist
+    from moe_expert_grouped_softmax_b200 import ops
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=300))
+
+    T, H, I, E, k, r, s = (cfg[x] for x in ("T", "H", "I", "E", "k", "r", "s"))
+    R = T * k
+    inp = S.make_inputs(cfg)
+    W = [inp[n].to(dev) for n in ("W1", "A1", "B1", "W2", "A2", "B2")]
+    X, logits, dY = (inp[n].to(dev) for n in ("X", "logits", "dY"))
+    blk = ops.MoeBlock(T, H, I, E, k, r, s, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        blk.step(X, logits, dY, W)
+    torch.cuda.synchronize()
+    st = ops.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ops.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        for i in range(K):
+            flush.zero_()                      # L2 flush, outside the timed span
+            ev0[i].record(stream)
+            blk.step(X, logits, dY, W)
+            ev1[i].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ops.profile_enable(False)
+    ms_steps = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    ms_total = float(sum(ms_steps))
+    kern = {}
+    for kind in ops.PROF_KINDS:
+        d = ops.profile_collect(kind)
+        if d:
+            kern[kind] = {"launches": len(d), "avg_ms": float(np.mean(d)),
+                          "total_ms": float(np.sum(d))}
+    st = ops.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timed steps")
+    if ws > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hX = X.cpu().pin_memory()
+        hL = logits.cpu().pin_memory()
+        hdY = dY.cpu().pin_memory()
+        outs = [blk.Y, blk.dX, blk.dA1, blk.dB1, blk.dA2, blk.dB2]
+        hout = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        dX_, dL_, ddY_ = torch.empty_like(X), torch.empty_like(logits), torch.empty_like(dY)
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+        def e2e_step(i=None):
+            if i is not None:
+                e0[i].record(stream)
+            dX_.copy_(hX, non_blocking=True)
+            dL_.copy_(hL, non_blocking=True)
+            ddY_.copy_(hdY, non_blocking=True)
+            blk.step(dX_, dL_, ddY_, W)
+            for o, h in zip(outs, hout):
+                h.copy_(o, non_blocking=True)
+            if i is not None:
+                e1[i].record(stream)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        for i in range(K):
+            flush.zero_()
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = float(sum(a.elapsed_time(b) for a, b in zip(e0, e1)))
+        if ws > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = hX.numel() * 2 + hL.numel() * 4 + hdY.numel() * 2
+        d2h = sum(h.numel() * h.element_size() for h in hout)
+        e2e = {"value": T * K * ws / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    counts = blk.counts.cpu().numpy()
+    if ws > 1:
+        dist.destroy_process_group()
+    return dict(ms_total=ms_total, ms_steps=ms_steps, kern=kern, e2e=e2e,
+                clocks=clk.summary(), counts=counts, ws=ws, rank=rank,
+                launches=ops.MoeBlock.KERNELS_PER_STEP * K)
+
+
+_CPU_INPUTS = {}
+
+
+def cpu_oracle_sample(cfg, n_tok):
+    """Times the fp64 oracle (as it stands) on the first n_tok tokens of the
+    workload (same weights, same routing rule).  Returns (seconds, threads)."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        threads = os.cpu_count() or 1
+    key = (cfg["name"], n_tok)
+    if key not in _CPU_INPUTS:
+        inp = S.make_inputs(cfg)
+        _CPU_INPUTS[key] = (
+            inp["X"][:n_tok].float().numpy(), inp["logits"][:n_tok].numpy(),
+            inp["dY"][:n_tok].float().numpy(),
+            [inp[n].float().numpy() for n in ("W1", "A1", "B1", "W2", "A2", "B2")])
+    X, L, dY, Wt = _CPU_INPUTS[key]
+    t0 = time.perf_counter()
+    Y, ctx = O.block_forward(X, L, cfg["k"], *Wt, cfg["s"])
+    O.block_backward(dY, ctx)
+    return time.perf_counter() - t0, threads
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="gpt-oss-20b", choices=list(S.CONFIGS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=128)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = S.make_config(args.config)
+    T, H, I, E, k, r = (cfg[x] for x in ("T", "H", "I", "E", "k", "r"))
+    R = T * k
+    flops = WL.block_flops(T, H, I, E, k, r)["total"]
+    pk = peaks()
+    workload = {"gpt-oss-20b": "gpt-oss-20b-shaped MoE layer fwd+bwd",
+                "qwen3-30b-a3b": "Qwen3-30B-A3B-shaped MoE layer fwd+bwd",
+                "gpt-oss-20b-long": "long-context gpt-oss-20b-shaped MoE layer fwd+bwd",
+                "deepseek-v3": "DeepSeek-V3-shaped MoE layer fwd+bwd",
+                "tiny": "tiny MoE block fwd+bwd"}[args.config]
+    config = {"workload": workload, "T": T, "H": H, "I": I, "E": E, "top_k": k,
+              "lora_r": r, "lora_s": cfg["s"], "logits": cfg["logits"],
+              "parallelism": "replicas", "l2": "256 MiB memset before each step, "
+              "outside the timed span"}
+    ws, rank, _ = dist_env()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        n_tok = max(8, min(T, args.cpu_sample_tokens // 2))
+        secs = []
+        threads = 1
+        for i in range(args.warmup + args.steps):
+            dt, threads = cpu_oracle_sample(cfg, n_tok)
+            if i >= args.warmup:
+                secs.append(dt)
+        tot = float(sum(secs))
+        val = n_tok * len(secs) / tot
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * tot / len(secs), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads,
+                                 "kind": "oracle",
+                                 "sample": f"first {n_tok} tokens of the layer per step "
+                                           f"(all {E} experts' weights), fwd+bwd"},
+                "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    res = run_ours(args, cfg)
+    if res["rank"] != 0:
+        return
+    K = args.steps
+    ms_per_step = res["ms_total"] / K
+    tokens_s = T * K * res["ws"] / (res["ms_total"] / 1e3)
+    tflops = flops / (ms_per_step / 1e3) / 1e12
+    # dominant kernel by measured share
+    kern = res["kern"]
+    gemm_flops = WL.gemm_flops(R, H, I, r)
+    dom = max((kk for kk in kern if kk in gemm_flops),
+              key=lambda kk: kern[kk]["total_ms"], default=None)
+    roof = None
+    if dom is not None:
+        ach = gemm_flops[dom] / (kern[dom]["avg_ms"] / 1e3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / pk["bf16_tflops"], "traffic": None,
+                "peak_source": pk["source"] + " (burst bf16)",
+                "flops_per_launch": gemm_flops[dom]}
+    hb = WL.hbm_bytes(T, H, E, k)
+    mem = {}
+    for kk, nbytes in (("permute", hb["permute"]), ("unpermute", hb["unpermute"])):
+        if kk in kern:
+            gbs = nbytes / (kern[kk]["avg_ms"] / 1e3) / 1e9
+            mem[kk] = {"GB_s": gbs, "frac_of_measured_hbm": gbs / pk["hbm_gbs"],
+                       "frac_of_8TBs": gbs / 8000.0}
+    cpu = None
+    if not args.no_cpu_baseline:
+        n_tok = args.cpu_sample_tokens
+        dt, threads = cpu_oracle_sample(cfg, n_tok)
+        cpu = {"value": n_tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {n_tok} tokens of the layer (all {E} experts' weights), "
+                         f"fwd+bwd, {dt:.1f} s"}
+    st = S.routing_stats(res["counts"])
+    line = {"metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": res["ws"],
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": config,
+            "tflops": tflops, "frac_of_bf16_peak": tflops / pk["bf16_tflops"],
+            "flops_per_step": flops, "roofline": roof, "hbm_kernels": mem,
+            "kernels": kern, "cpu_baseline": cpu, "e2e": res["e2e"],
+            "gpu_launches": res["launches"], "clocks": res["clocks"],
+            "routing": st}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

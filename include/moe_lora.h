@@ -1,0 +1,189 @@
+/*
+ * moe_lora.h -- C ABI of the B200 (sm_100a) MoE split-LoRA expert block.
+ *
+ * The block (forward and backward) is the Mixture-of-Experts expert MLP used
+ * in LoRA fine-tuning, as described on the Unsloth page "Fine-tune MoE LLMs
+ * 12x faster with Unsloth":
+ *   route (top-k over router logits) -> permute tokens into expert order ->
+ *   grouped GEMM over gate_up_proj [E, 2I, H] with SwiGLU -> grouped GEMM over
+ *   down_proj [E, H, I] -> routing-weighted unpermute (combine).
+ * Every projection carries split LoRA (section "Faster LoRA MoE training"):
+ *   y = x W^T + s (x A^T) B^T,   A [E, r, in], B [E, out, r],
+ * so W + s B A is never formed.  The backward computes dX and the LoRA
+ * gradients dA, dB with the base weights frozen.
+ *
+ * Conventions (all entry points):
+ *  - Every pointer except the status helpers is a DEVICE pointer; every
+ *    tensor is dense row-major.  "bf16" means IEEE bfloat16 (16-bit, stored
+ *    as uint16).  The caller owns and allocates every buffer, including the
+ *    workspace and the saved-activation buffer; the library never allocates,
+ *    frees or synchronises (except moe_get_device_status).
+ *  - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) on the current device.
+ *  - Argument errors are detected on the host and returned before anything is
+ *    launched.  Errors that only the device can see (a bounded wait that ran
+ *    out, an index out of range) are recorded in a per-device status word that
+ *    moe_get_device_status() returns and clears; the kernel that saw the error
+ *    skips the offending access and returns.
+ *  - Shape limits: 1 <= k <= E <= 512; H and I multiples of 16 and >= 64;
+ *    r in {16, 32, 64}; T * k < 2^31.  Router logits must be finite.
+ *  - R = T * k is the number of routed (token, slot) rows.
+ */
+#ifndef MOE_LORA_H_
+#define MOE_LORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int moe_status_t;
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG 1     /* null pointer, bad size, too-small buffer */
+#define MOE_ERR_UNSUPPORTED 2     /* shape outside the limits above */
+#define MOE_ERR_CUDA 3            /* a CUDA runtime / driver call failed */
+#define MOE_ERR_DEVICE_TIMEOUT 4  /* a kernel's bounded wait ran out */
+#define MOE_ERR_DEVICE_BOUNDS 5   /* a kernel found an index out of range */
+
+typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* ---------------------------------------------------------------- a1: route
+ * Top-k routing (page section "What is torch._grouped_mm?": each token is sent
+ * to the experts its router picks; section "Implementation details": the
+ * router is frozen, so logits are an input).
+ *   logits        fp32 [T, E]   router logits (finite).
+ *   topk_idx      int32 [T, k]  experts by (logit desc, expert index asc).
+ *   topk_w        fp32 [T, k]   w_j = exp(l_j - l_max) / sum_sel exp(l - l_max)
+ *                               (softmax over E renormalised over the kept k).
+ *   expert_counts int32 [E]     rows routed to each expert.
+ *   expert_offsets int32 [E+1]  exclusive prefix sum of counts; [E] = T*k.
+ *   dest          int32 [T, k]  permuted row of (t, j): offsets[e] + the
+ *                               number of earlier flat indices t'*k+j' routed
+ *                               to the same expert (stable counting sort).
+ *   ws            device scratch of moe_route_workspace_bytes(T, E, k) bytes.
+ * Deterministic: the same inputs give the same bytes. */
+MOE_API size_t moe_route_workspace_bytes(int T, int E, int k);
+MOE_API moe_status_t moe_route_topk(const float* logits, int T, int E, int k,
+                            int32_t* topk_idx, float* topk_w,
+                            int32_t* expert_counts, int32_t* expert_offsets,
+                            int32_t* dest, void* ws, size_t ws_bytes,
+                            moe_stream_t stream);
+
+/* ------------------------------------------------------- a2 / a6: permute
+ * Gather into expert order: Xp[dest[t, j]] = scale[t, j] * X[t] (scale NULL
+ * means 1; with scale the product is formed in fp32 and rounded to bf16).
+ *   X [T, H] bf16 -> Xp [T*k, H] bf16.
+ * Optional, for the routing-weight gradient (backward of the combine):
+ *   if dw != NULL, dw[t, j] = <X[t], Zp[dest[t, j]]> (fp32 accumulation) with
+ *   Zp [T*k, H] bf16 (pass the forward's Z2 and X = dY). */
+MOE_API moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
+                         int T, int H, int k, void* Xp, const void* Zp,
+                         float* dw, moe_stream_t stream);
+
+/* ----------------------------------------------------- a5 / a10: unpermute
+ * Weighted combine: Y[t] = sum_j w[t, j] * Yp[dest[t, j]], accumulated in fp32
+ * in j order, rounded once to bf16 (w NULL means 1: used for dX).
+ *   Yp [T*k, H] bf16 -> Y [T, H] bf16.  No atomics; deterministic. */
+MOE_API moe_status_t moe_unpermute(const void* Yp, const int32_t* dest, const float* w,
+                           int T, int H, int k, void* Y, moe_stream_t stream);
+
+/* ---------------------------------------------- saved activations / scratch
+ * The forward writes what the backward needs into `saved`
+ * (moe_saved_bytes(R, H, I, r) bytes, 256-byte aligned parts):
+ *   part 0: Z1  bf16 [R, 2I]  gate_up output (gate = cols [0, I), up = [I, 2I))
+ *   part 1: h   bf16 [R, I]   silu(gate) * up
+ *   part 2: XA1 bf16 [r, R]   s * (Xp A1^T), transposed, row pitch
+ *                             round_up(R, 64) elements (padding zeroed)
+ *   part 3: HA2 bf16 [r, R]   s * (h A2^T), transposed, same pitch
+ * moe_saved_part_offset(R, H, I, r, part) gives each part's byte offset. */
+MOE_API size_t moe_saved_bytes(int R, int H, int I, int r);
+MOE_API size_t moe_saved_part_offset(int R, int H, int I, int r, int part);
+/* Scratch needed by moe_lora_mlp_fwd / moe_lora_mlp_bwd (device bytes). */
+MOE_API size_t moe_workspace_bytes(int R, int E, int H, int I, int r);
+
+/* ------------------------------------------------- a3 + a4: expert forward
+ * Per expert e, on its rows Xp[offsets[e] : offsets[e+1]] (page section "What
+ * is torch._grouped_mm?": gate, up = chunk(2) of linear(x, gate_up_proj[e])):
+ *   Z1 = Xp W1[e]^T + s (Xp A1[e]^T) B1[e]^T             [M_e, 2I]
+ *   h  = silu(Z1[:, :I]) * Z1[:, I:]                     [M_e, I]
+ *   Z2 = h W2[e]^T + s (h A2[e]^T) B2[e]^T               [M_e, H]
+ * Weights: W1 [E, 2I, H], A1 [E, r, H], B1 [E, 2I, r], W2 [E, H, I],
+ * A2 [E, r, I], B2 [E, H, r]; all bf16.  Xp [R, H], Z2 [R, H] bf16.
+ * expert_offsets is the device array from moe_route_topk (read on the device;
+ * no host synchronisation).  Products accumulate in fp32 on the tensor cores;
+ * the rank-r intermediates are rounded to bf16 before the second product. */
+MOE_API moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets,
+                              int E, int H, int I, int r, float s,
+                              const void* W1, const void* A1, const void* B1,
+                              const void* W2, const void* A2, const void* B2,
+                              int R, void* Z2, void* saved, size_t saved_bytes,
+                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------- a7 + a8 + a9: expert backward
+ * Input dZ2 [R, H] bf16 is the gradient at Z2 already multiplied by the
+ * routing weight (moe_permute of dY with scale = topk_w).  With the base
+ * weights frozen:
+ *   dh   = dZ2 W2[e] + s (dZ2 B2[e]) A2[e]                 [M_e, I]
+ *   dZ1  = [dh * up * silu'(gate), dh * silu(gate)]        [M_e, 2I]
+ *   dXp  = dZ1 W1[e] + s (dZ1 B1[e]) A1[e]                 [M_e, H]
+ *   dA2[e] = s (dZ2 B2)^T h,   dB2[e] = s dZ2^T (h A2^T)
+ *   dA1[e] = s (dZ1 B1)^T Xp,  dB1[e] = s dZ1^T (Xp A1^T)
+ * with silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g))).  Outputs dXp [R, H],
+ * dA1 [E, r, H], dB1 [E, 2I, r], dA2 [E, r, I], dB2 [E, H, r], all bf16
+ * (fp32 accumulation, fixed order: deterministic).  Experts with no rows get
+ * exact zeros.  `saved` must hold the forward's saved activations. */
+MOE_API moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
+                              const int32_t* expert_offsets,
+                              int E, int H, int I, int r, float s,
+                              const void* W1, const void* A1, const void* B1,
+                              const void* W2, const void* A2, const void* B2,
+                              const void* saved, size_t saved_bytes, int R,
+                              void* dXp, void* dA1, void* dB1, void* dA2,
+                              void* dB2, void* ws, size_t ws_bytes,
+                              moe_stream_t stream);
+
+/* ---------------------------------------------------------------- status
+ * moe_get_device_status synchronises `stream`, returns the first device-side
+ * error recorded since the last call (MOE_OK if none) and clears it.
+ * moe_status_string never returns NULL. */
+MOE_API moe_status_t moe_get_device_status(moe_stream_t stream);
+MOE_API const char* moe_status_string(moe_status_t status);
+
+/* Testing hook: caps every bounded device wait at `ns` nanoseconds (0 restores
+ * the default of one second).  A cap of 1 makes the first wait that does not
+ * succeed immediately give up, which exercises the timeout path. */
+MOE_API void moe_set_wait_limit_ns(uint64_t ns);
+
+/* Benchmark hook (not thread-safe; for measurement only).
+ * moe_profile_enable(1) starts recording, for every kernel kind below, a pair
+ * of CUDA events around each of its launches on the launching stream (up to
+ * 512 launches per kind; the counts restart at each enable call);
+ * moe_profile_enable(0) stops recording.  moe_profile_collect synchronises on
+ * the recorded events and writes the durations (ms) of up to max_n launches
+ * of `kind` into ms[], returning how many (or -1 on a CUDA error).  Route
+ * covers its three kernels together. */
+#define MOE_PROF_ROUTE 0
+#define MOE_PROF_PERMUTE 1
+#define MOE_PROF_GATE_UP_FWD 2
+#define MOE_PROF_DOWN_FWD 3
+#define MOE_PROF_UNPERMUTE 4
+#define MOE_PROF_DOWN_BWD 5
+#define MOE_PROF_GATE_UP_BWD 6
+#define MOE_PROF_LORA_GRAD 7
+#define MOE_PROF_TRANSPOSE 8
+#define MOE_PROF_KINDS 9
+MOE_API moe_status_t moe_profile_enable(int on);
+MOE_API int moe_profile_collect(int kind, float* ms, int max_n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_LORA_H_ */

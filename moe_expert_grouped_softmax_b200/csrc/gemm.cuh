@@ -1,0 +1,511 @@
+// a3 / a4 / a7 / a8: persistent grouped GEMM over ragged experts on the
+// 5th-generation tensor cores, with the split-LoRA product fused in.
+//
+// Per output tile (128 rows of one expert x BN columns):
+//   mainloop  : acc  += A_k * B_k^T          (base weight, fp32 in TMEM)
+//               lora += A_k * LA_k^T         (rank-r down-projection, same A
+//                                             tile from shared memory)
+//   then      : xa    = bf16(s * lora)        (TMEM -> registers -> smem)
+//               acc  += xa * LB^T             (rank-r up-projection, second
+//                                             accumulate into the same tile)
+//   epilogue  : mode-specific (SwiGLU, plain store, SwiGLU backward).
+// This is the "split LoRA" order of the Unsloth page "Fine-tune MoE LLMs 12x
+// faster with Unsloth" (section "Faster LoRA MoE training"): x W^T +
+// s (x A^T) B^T, so W + s B A is never formed.
+//
+// Roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
+// owner), warps 2..5 = epilogue (TMEM lane quarter = warp % 4).  TMEM holds
+// two accumulator sets (256 columns each: BN base + r LoRA) so the epilogue
+// of one tile overlaps the mainloop of the next.  Tiles are enumerated on the
+// device from expert_offsets (no host synchronisation): m-tiles of all
+// experts in expert order, n fastest.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace moe {
+
+enum GemmMode : int {
+  kGateUpFwd = 0,  // Z1 = Xp W1^T + s (Xp A1^T) B1^T -> SwiGLU -> h (+ Z1, XA1)
+  kDownFwd = 1,    // Z2 = h W2^T + s (h A2^T) B2^T (+ hA2)
+  kDownBwd = 2,    // dh = dZ2 W2 + s (dZ2 B2) A2 -> SwiGLU backward -> dZ1
+  kGateUpBwd = 3,  // dXp = dZ1 W1 + s (dZ1 B1) A1
+};
+
+struct GemmArgs {
+  const int32_t* offsets;  // [E+1] expert row offsets (device)
+  int E, R, K;
+  int N;                   // output columns (I for gate_up fwd / down bwd)
+  int n_tiles;             // tiles along N
+  int I;                   // gate/up split
+  int b_rows;              // rows per expert in B's 2-D view
+  int lb_rows;             // rows per expert in LB's 2-D view
+  float s;
+  __nv_bfloat16* out;
+  int ld_out;
+  __nv_bfloat16* out2;     // saved Z1 (gate_up fwd)
+  int ld_out2;
+  const __nv_bfloat16* aux;  // saved Z1 (down bwd)
+  int ld_aux;
+  __nv_bfloat16* lora_t;   // [r, ld_lora] s-scaled rank-r product, transposed
+  int ld_lora;
+  uint64_t wait_ns;
+};
+
+constexpr int kSmemOptin = 232448;  // max dynamic shared memory per block
+
+template <int BN, int RK>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int LA_BYTES = RK * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + LA_BYTES;
+  static constexpr int LB_BYTES = BN * RK * 2;
+  static constexpr int XA_BYTES = BM * RK * 2;
+  static constexpr int MISC_BYTES = 256 + 8 * 520;  // barriers, flags, tables
+  static constexpr int FIXED = 2 * LB_BYTES + 2 * XA_BYTES + MISC_BYTES;
+  static constexpr int NS_FIT = (kSmemOptin - 1024 - FIXED) / STAGE_BYTES;
+  static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
+  static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + FIXED;
+  static constexpr int LSPAN = RK * 2;  // bytes of one LoRA row = swizzle span
+  static constexpr uint32_t LLAYOUT =
+      RK == 16 ? kLayoutSW32 : (RK == 32 ? kLayoutSW64 : kLayoutSW128);
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int ACC_STRIDE = 256;
+  static_assert(NS >= 2, "not enough shared memory for two stages");
+  static_assert(SMEM_BYTES <= kSmemOptin, "shared memory over the opt-in limit");
+  static_assert(BN + RK <= ACC_STRIDE, "TMEM: BN + r must fit 256 columns");
+  static_assert(BN % 64 == 0, "BN must be a multiple of 64");
+  static_assert(RK == 16 || RK == 32 || RK == 64, "rank must be 16, 32 or 64");
+};
+
+__device__ __forceinline__ void decode_tile(int tile, int n_tiles,
+                                            const int* s_mstart, int E, int& e,
+                                            int& mt, int& nt) {
+  const int gm = tile / n_tiles;
+  nt = tile - gm * n_tiles;
+  int lo = 0, hi = E;  // s_mstart[lo] <= gm < s_mstart[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_mstart[mid] <= gm) lo = mid; else hi = mid;
+  }
+  e = lo;
+  mt = gm - s_mstart[lo];
+}
+
+// Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait that ignores the abort flag (used to drain work in flight).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity,
+                                           uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      set_status(4);
+      return;
+    }
+  }
+}
+
+// Builds the m-tile table in shared memory (one warp): s_off = offsets,
+// s_mstart[e] = first global m-tile of expert e, s_mstart[E] = total.
+// Offsets that are not a valid partition of [0, R) give zero tiles.
+__device__ __forceinline__ void build_tile_table(const int32_t* offsets, int E,
+                                                 int R, int* s_off,
+                                                 int* s_mstart, int lane) {
+  const int per = (E + 31) / 32;
+  const int lo = min(E, lane * per), hi = min(E, lo + per);
+  bool bad = false;
+  int local = 0;
+  for (int e = lo; e < hi; ++e) {
+    const int a = offsets[e], b = offsets[e + 1];
+    if (b < a) bad = true;
+    local += (b - a + 127) >> 7;
+  }
+  if (lane == 0 && offsets[0] != 0) bad = true;
+  if (lane == 0 && offsets[E] != R) bad = true;
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  int run = incl - local;
+  for (int e = lo; e < hi; ++e) {
+    const int a = offsets[e], b = offsets[e + 1];
+    s_off[e] = a;
+    s_mstart[e] = run;
+    run += (b - a + 127) >> 7;
+  }
+  const bool any_bad = __any_sync(0xffffffffu, bad);
+  if (lane == 31) {
+    s_mstart[E] = any_bad ? 0 : incl;
+    s_off[E] = R;
+  }
+  if (any_bad && lane == 0) set_status(5);
+}
+
+template <int MODE, int BN, int RK>
+__global__ void __launch_bounds__(192, 1)
+    grouped_lora_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmLA,
+                             const __grid_constant__ CUtensorMap tmLB,
+                             const GemmArgs args) {
+  using C = GemmCfg<BN, RK>;
+  constexpr bool kSwiGLU = (MODE == kGateUpFwd);
+  constexpr bool kBMN = (MODE == kDownBwd || MODE == kGateUpBwd);
+  constexpr int HALF = BN / 2;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sStage = smem;
+  uint8_t* sLB = sStage + C::NS * C::STAGE_BYTES;
+  uint8_t* sXA = sLB + 2 * C::LB_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sXA + 2 * C::XA_BYTES);
+  uint64_t* empty = full + C::NS;
+  uint64_t* lb_full = empty + C::NS;
+  uint64_t* lb_empty = lb_full + 2;
+  uint64_t* lora_full = lb_empty + 2;
+  uint64_t* xa_ready = lora_full + 2;
+  uint64_t* acc_full = xa_ready + 2;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain_bar = acc_empty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_off = reinterpret_cast<int*>(s_tmem + 4);
+  int* s_mstart = s_off + 520;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = args.E;
+  const uint64_t wait_ns = args.wait_ns;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&lb_full[i], 1);
+      mbar_init(&lb_empty[i], 1);
+      mbar_init(&lora_full[i], 1);
+      mbar_init(&xa_ready[i], 4);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(drain_bar, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmLA);
+    prefetch_tmap(&tmLB);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 2) build_tile_table(args.offsets, E, args.R, s_off, s_mstart, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = *s_tmem;
+  const int total_tiles = s_mstart[E] * args.n_tiles;
+  const int k_iters = (args.K + C::BK - 1) / C::BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed_stages = 0;      // stages armed at least once
+      uint32_t lb_armed = 0;     // LB buffers armed at least once
+      uint32_t lb_par[2] = {0, 0};
+      bool ok = true;
+      int local = 0;
+      for (int tile = blockIdx.x; tile < total_tiles && ok;
+           tile += gridDim.x, ++local) {
+        int e, mt, nt;
+        decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+        const int row0 = s_off[e] + mt * C::BM;
+        const int b = local & 1;
+        const uint32_t use = (local >> 1) & 1;
+        if (!mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
+        mbar_arrive_expect_tx(&lb_full[b], C::LB_BYTES);
+        lb_armed |= 1u << b;
+        lb_par[b] = use;
+        uint8_t* lb = sLB + b * C::LB_BYTES;
+        if (kSwiGLU) {
+          tma_load_2d(lb, &tmLB, &lb_full[b], 0, e * args.lb_rows + nt * HALF);
+          tma_load_2d(lb + HALF * C::LSPAN, &tmLB, &lb_full[b], 0,
+                      e * args.lb_rows + args.I + nt * HALF);
+        } else {
+          tma_load_2d(lb, &tmLB, &lb_full[b], 0, e * args.lb_rows + nt * BN);
+        }
+        for (int kt = 0; kt < k_iters; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, wait_ns)) { ok = false; break; }
+          uint8_t* st = sStage + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(st, &tmA, &full[stage], kt * C::BK, row0);
+          uint8_t* sb = st + C::A_BYTES;
+          if (kBMN) {
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i)
+              tma_load_2d(sb + i * 8192, &tmB, &full[stage], nt * BN + 64 * i,
+                          e * args.b_rows + kt * C::BK);
+          } else if (kSwiGLU) {
+            tma_load_2d(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * HALF);
+            tma_load_2d(sb + HALF * 128, &tmB, &full[stage], kt * C::BK,
+                        e * args.b_rows + args.I + nt * HALF);
+          } else {
+            tma_load_2d(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * BN);
+          }
+          tma_load_2d(sb + C::B_BYTES, &tmLA, &full[stage], kt * C::BK, e * RK);
+          if (armed_stages < C::NS) ++armed_stages;
+          if (++stage == C::NS) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Wait until every load issued has landed before the CTA may exit.
+      for (int i = 0; i < armed_stages; ++i) {
+        // the last arming of stage s had parity (phase of that arming)
+        int s = stage - 1 - i;
+        uint32_t ph = phase;
+        if (s < 0) {
+          s += C::NS;
+          ph ^= 1;
+        }
+        drain_wait(&full[s], ph, wait_ns);
+      }
+      for (int bb = 0; bb < 2; ++bb)
+        if (lb_armed & (1u << bb)) drain_wait(&lb_full[bb], lb_par[bb], wait_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescMain = idesc_bf16_f32(128, BN, false, kBMN);
+      constexpr uint32_t kIdescLora = idesc_bf16_f32(128, RK, false, false);
+      constexpr uint32_t kIdescUp = idesc_bf16_f32(128, BN, false, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++local) {
+        const int b = local & 1;
+        const uint32_t use = (local >> 1) & 1;
+        const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
+        const uint32_t t_lora = t_acc + BN;
+        if (!mbar_wait(&acc_empty[b], use ^ 1, s_abort, wait_ns)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = 0; kt < k_iters; ++kt) {
+          if (!mbar_wait(&full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sStage + stage * C::STAGE_BYTES);
+          const uint32_t b0 = a0 + C::A_BYTES;
+          const uint32_t la0 = b0 + C::B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
+            const uint64_t da = smem_desc(a0 + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t db = kBMN ? smem_desc(b0 + kk * 2048, 8192, 1024, kLayoutSW128)
+                                     : smem_desc(b0 + kk * 32, 16, 1024, kLayoutSW128);
+            const uint64_t dla = smem_desc(la0 + kk * 32, 16, 1024, kLayoutSW128);
+            const uint32_t accum = (kt | kk) ? 1u : 0u;
+            umma_bf16(t_acc, da, db, kIdescMain, accum);
+            umma_bf16(t_lora, da, dla, kIdescLora, accum);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::NS) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&lora_full[b]);
+        if (!mbar_wait(&xa_ready[b], use, s_abort, wait_ns)) break;
+        if (!mbar_wait(&lb_full[b], use, s_abort, wait_ns)) break;
+        tc_fence_after();
+        const uint32_t xa0 = smem_u32(sXA + b * C::XA_BYTES);
+        const uint32_t lb0 = smem_u32(sLB + b * C::LB_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < RK / 16; ++kk) {
+          umma_bf16(t_acc, smem_desc(xa0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
+                    smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), kIdescUp, 1u);
+        }
+        umma_commit(&lb_empty[b]);
+        umma_commit(&acc_full[b]);
+      }
+      // every MMA issued by this thread must be complete before TMEM is freed
+      umma_commit(drain_bar);
+      drain_wait(drain_bar, 0, wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp & 3;
+    const int row_in_tile = ew * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(ew * 32) << 16;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++local) {
+      int e, mt, nt;
+      decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+      const int b = local & 1;
+      const uint32_t use = (local >> 1) & 1;
+      const int grow = s_off[e] + mt * C::BM + row_in_tile;
+      const bool rvalid = grow < s_off[e + 1];
+      const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
+      const uint32_t t_lora = t_acc + BN;
+
+      // rank-r product: TMEM -> bf16 A operand of the up-projection
+      if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
+      tc_fence_after();
+      {
+        float xa[RK];
+#pragma unroll
+        for (int c = 0; c < RK; c += 16) tmem_ld16(t_lora + c, xa + c);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < RK; ++i) xa[i] *= args.s;
+        uint8_t* xt = sXA + b * C::XA_BYTES;
+#pragma unroll
+        for (int ch = 0; ch < RK / 8; ++ch) {
+          uint4 v;
+          v.x = pack_bf16x2(xa[8 * ch + 0], xa[8 * ch + 1]);
+          v.y = pack_bf16x2(xa[8 * ch + 2], xa[8 * ch + 3]);
+          v.z = pack_bf16x2(xa[8 * ch + 4], xa[8 * ch + 5]);
+          v.w = pack_bf16x2(xa[8 * ch + 6], xa[8 * ch + 7]);
+          *reinterpret_cast<uint4*>(xt + swz_offset(row_in_tile, ch, C::LSPAN)) = v;
+        }
+        if (nt == 0 && rvalid && args.lora_t != nullptr) {
+#pragma unroll
+          for (int q = 0; q < RK; ++q)
+            args.lora_t[static_cast<size_t>(q) * args.ld_lora + grow] =
+                __float2bfloat16_rn(xa[q]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xa_ready[b]);
+
+      if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
+      tc_fence_after();
+      if (kSwiGLU) {
+#pragma unroll 1
+        for (int c = 0; c < HALF; c += 32) {
+          float g[32], u[32];
+          tmem_ld32(t_acc + c, g);
+          tmem_ld32(t_acc + HALF + c, u);
+          tmem_ld_wait();
+          const int col = nt * HALF + c;
+          if (rvalid) {
+            __nv_bfloat16* hp = args.out + static_cast<size_t>(grow) * args.ld_out + col;
+            __nv_bfloat16* gp = args.out2 + static_cast<size_t>(grow) * args.ld_out2 + col;
+            __nv_bfloat16* up = gp + args.I;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (col + 8 * q < args.N) {
+                uint32_t hv[4], gv[4], uv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float g0 = g[8 * q + 2 * i], g1 = g[8 * q + 2 * i + 1];
+                  const float u0 = u[8 * q + 2 * i], u1 = u[8 * q + 2 * i + 1];
+                  hv[i] = pack_bf16x2(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
+                  gv[i] = pack_bf16x2(g0, g1);
+                  uv[i] = pack_bf16x2(u0, u1);
+                }
+                *reinterpret_cast<uint4*>(hp + 8 * q) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                *reinterpret_cast<uint4*>(gp + 8 * q) = make_uint4(gv[0], gv[1], gv[2], gv[3]);
+                *reinterpret_cast<uint4*>(up + 8 * q) = make_uint4(uv[0], uv[1], uv[2], uv[3]);
+              }
+            }
+          }
+        }
+      } else if (MODE == kDownBwd) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float dh[32];
+          tmem_ld32(t_acc + c, dh);
+          tmem_ld_wait();
+          const int col = nt * BN + c;
+          if (rvalid) {
+            const __nv_bfloat16* gp = args.aux + static_cast<size_t>(grow) * args.ld_aux + col;
+            const __nv_bfloat16* up = gp + args.I;
+            __nv_bfloat16* dgp = args.out + static_cast<size_t>(grow) * args.ld_out + col;
+            __nv_bfloat16* dup = dgp + args.I;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (col + 8 * q < args.N) {
+                const uint4 gq = *reinterpret_cast<const uint4*>(gp + 8 * q);
+                const uint4 uq = *reinterpret_cast<const uint4*>(up + 8 * q);
+                const uint32_t ga[4] = {gq.x, gq.y, gq.z, gq.w};
+                const uint32_t ua[4] = {uq.x, uq.y, uq.z, uq.w};
+                uint32_t dg[4], du[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  float gg[2] = {bf16_lo(ga[i]), bf16_hi(ga[i])};
+                  float uu[2] = {bf16_lo(ua[i]), bf16_hi(ua[i])};
+                  float o_g[2], o_u[2];
+#pragma unroll
+                  for (int h2 = 0; h2 < 2; ++h2) {
+                    const float d = dh[8 * q + 2 * i + h2];
+                    const float sg = sigmoidf_(gg[h2]);
+                    o_g[h2] = d * uu[h2] * sg * (1.f + gg[h2] * (1.f - sg));
+                    o_u[h2] = d * gg[h2] * sg;
+                  }
+                  dg[i] = pack_bf16x2(o_g[0], o_g[1]);
+                  du[i] = pack_bf16x2(o_u[0], o_u[1]);
+                }
+                *reinterpret_cast<uint4*>(dgp + 8 * q) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+                *reinterpret_cast<uint4*>(dup + 8 * q) = make_uint4(du[0], du[1], du[2], du[3]);
+              }
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          tmem_ld32(t_acc + c, v);
+          tmem_ld_wait();
+          const int col = nt * BN + c;
+          if (rvalid) {
+            __nv_bfloat16* op = args.out + static_cast<size_t>(grow) * args.ld_out + col;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (col + 8 * q < args.N) {
+                *reinterpret_cast<uint4*>(op + 8 * q) = make_uint4(
+                    pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                    pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace moe

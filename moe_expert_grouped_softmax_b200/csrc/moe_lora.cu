@@ -1,0 +1,582 @@
+// Host side of the C ABI declared in include/moe_lora.h: argument checks,
+// tensor-map encoding, tile-shape choice and kernel launches.  Every kernel
+// of the block is compiled into this one translation unit (so they share the
+// device status word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "moe_lora.h"
+#include "ptx.cuh"
+#include "route.cuh"
+#include "permute.cuh"
+#include "gemm.cuh"
+#include "lora_grad.cuh"
+
+using namespace moe;
+
+namespace {
+
+uint64_t g_wait_limit_ns = 1000000000ull;  // one second per bounded wait
+
+// ------------------------------------------------ optional per-kernel timing
+// When enabled, each launch site of a kernel kind records a CUDA event before
+// and after its launch on the caller's stream (up to kProfCap pairs per kind).
+constexpr int kProfCap = 512;
+bool g_prof_on = false;
+cudaEvent_t g_prof_ev[MOE_PROF_KINDS][kProfCap][2];
+int g_prof_n[MOE_PROF_KINDS];
+bool g_prof_created = false;
+
+void prof_record(int kind, int which, cudaStream_t st) {
+  if (!g_prof_on || kind < 0 || kind >= MOE_PROF_KINDS) return;
+  const int n = g_prof_n[kind];
+  if (n >= kProfCap) return;
+  cudaEventRecord(g_prof_ev[kind][n][which], st);
+  if (which == 1) g_prof_n[kind] = n + 1;
+}
+
+struct ProfScope {
+  int kind;
+  cudaStream_t st;
+  ProfScope(int k, cudaStream_t s) : kind(k), st(s) { prof_record(kind, 0, st); }
+  ~ProfScope() { prof_record(kind, 1, st); }
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                  void*, const cuuint64_t*, const cuuint64_t*,
+                                  const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows,
+// row pitch `pitch_bytes`; box of box_inner x box_outer elements.
+bool tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+             uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+             CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) || (pitch_bytes & 15u)) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+CUtensorMapSwizzle lora_swizzle(int r) {
+  return r == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                 : (r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline int ld_rank(int R) { return (R + 63) & ~63; }  // row pitch of [r, R] parts
+
+moe_status_t launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool shape_ok(int E, int H, int I, int r) {
+  if (E < 1 || E > 512) return false;
+  if (H < 64 || I < 64 || (H % 16) || (I % 16)) return false;
+  if (!(r == 16 || r == 32 || r == 64)) return false;
+  return true;
+}
+
+// Tile width along N: 192 unless it pads noticeably more than 128 does.
+int pick_bn(int n_cols, bool swiglu, int r) {
+  if (r == 64) return 128;
+  auto waste = [&](int bn) {
+    const int w = swiglu ? bn / 2 : bn;
+    const int tiles = (n_cols + w - 1) / w;
+    return static_cast<double>(tiles * w - n_cols) / n_cols;
+  };
+  return waste(192) <= waste(128) + 0.02 ? 192 : 128;
+}
+
+template <int MODE, int BN, int RK>
+moe_status_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b,
+                           const CUtensorMap& la, const CUtensorMap& lb,
+                           const GemmArgs& args, cudaStream_t st) {
+  using C = GemmCfg<BN, RK>;
+  auto kern = grouped_lora_gemm_kernel<MODE, BN, RK>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_BYTES) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const long long max_tiles =
+      (static_cast<long long>(args.R) / 128 + args.E) * args.n_tiles;
+  const int grid = static_cast<int>(std::min<long long>(num_sms(), max_tiles));
+  if (grid <= 0) return MOE_ERR_CUDA;
+  ProfScope prof(MODE == kGateUpFwd ? MOE_PROF_GATE_UP_FWD
+                 : MODE == kDownFwd ? MOE_PROF_DOWN_FWD
+                 : MODE == kDownBwd ? MOE_PROF_DOWN_BWD : MOE_PROF_GATE_UP_BWD, st);
+  kern<<<grid, 192, C::SMEM_BYTES, st>>>(a, b, la, lb, args);
+  return launch_status();
+}
+
+template <int MODE>
+moe_status_t launch_gemm(int bn, int r, const CUtensorMap& a, const CUtensorMap& b,
+                         const CUtensorMap& la, const CUtensorMap& lb,
+                         const GemmArgs& args, cudaStream_t st) {
+  if (r == 16 && bn == 192) return launch_gemm_t<MODE, 192, 16>(a, b, la, lb, args, st);
+  if (r == 16 && bn == 128) return launch_gemm_t<MODE, 128, 16>(a, b, la, lb, args, st);
+  if (r == 32 && bn == 192) return launch_gemm_t<MODE, 192, 32>(a, b, la, lb, args, st);
+  if (r == 32 && bn == 128) return launch_gemm_t<MODE, 128, 32>(a, b, la, lb, args, st);
+  if (r == 64 && bn == 128) return launch_gemm_t<MODE, 128, 64>(a, b, la, lb, args, st);
+  return MOE_ERR_UNSUPPORTED;
+}
+
+template <int RK>
+moe_status_t launch_grad_t(const CUtensorMap* u, const CUtensorMap* v,
+                           const GradArgs& args, cudaStream_t st) {
+  using C = GradCfg<RK>;
+  auto kern = lora_grad_kernel<RK>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_BYTES) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int grid = std::min(num_sms(), args.total_tiles);
+  if (grid <= 0) return MOE_OK;
+  ProfScope prof(MOE_PROF_LORA_GRAD, st);
+  kern<<<grid, 192, C::SMEM_BYTES, st>>>(u[0], u[1], u[2], u[3], v[0], v[1], v[2],
+                                         v[3], args);
+  return launch_status();
+}
+
+// Saved-activation parts (bytes from the start of `saved`).
+void saved_layout(int R, int H, int I, int r, size_t off[5]) {
+  (void)H;
+  const size_t z1 = static_cast<size_t>(R) * 2 * I * 2;
+  const size_t h = static_cast<size_t>(R) * I * 2;
+  const size_t xa = static_cast<size_t>(r) * ld_rank(R) * 2;
+  off[0] = 0;
+  off[1] = off[0] + align256(z1);
+  off[2] = off[1] + align256(h);
+  off[3] = off[2] + align256(xa);
+  off[4] = off[3] + align256(xa);
+}
+
+// Backward scratch parts.
+void bwd_layout(int R, int E, int H, int I, int r, size_t off[8]) {
+  const size_t dz1 = static_cast<size_t>(R) * 2 * I * 2;
+  const size_t vt = static_cast<size_t>(r) * ld_rank(R) * 2;
+  off[0] = 0;                                                  // dZ1 [R, 2I]
+  off[1] = off[0] + align256(dz1);                             // dZB2t [r, ldR]
+  off[2] = off[1] + align256(vt);                              // dZB1t [r, ldR]
+  off[3] = off[2] + align256(vt);                              // B2t [E, r, H]
+  off[4] = off[3] + align256(static_cast<size_t>(E) * r * H * 2);   // A2t [E, I, r]
+  off[5] = off[4] + align256(static_cast<size_t>(E) * I * r * 2);   // B1t [E, r, 2I]
+  off[6] = off[5] + align256(static_cast<size_t>(E) * r * 2 * I * 2);  // A1t [E, H, r]
+  off[7] = off[6] + align256(static_cast<size_t>(E) * H * r * 2);
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+template <typename T>
+const T* at(const void* base, size_t off) {
+  return reinterpret_cast<const T*>(static_cast<const char*>(base) + off);
+}
+
+// zero the padding columns [R, ldR) of an [r, ldR] bf16 part
+moe_status_t zero_rank_padding(void* p, int R, int r, cudaStream_t st) {
+  const int ld = ld_rank(R);
+  if (ld == R) return MOE_OK;
+  const cudaError_t e = cudaMemset2DAsync(static_cast<char*>(p) + static_cast<size_t>(R) * 2,
+                                          static_cast<size_t>(ld) * 2, 0,
+                                          static_cast<size_t>(ld - R) * 2, r, st);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t transpose(const void* in, void* out, int nb, int P, int Q, cudaStream_t st) {
+  dim3 grid((Q + 31) / 32, (P + 31) / 32, nb);
+  ProfScope prof(MOE_PROF_TRANSPOSE, st);
+  transpose_kernel<<<grid, dim3(32, 8), 0, st>>>(static_cast<const __nv_bfloat16*>(in),
+                                                 static_cast<__nv_bfloat16*>(out), P, Q);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_BOUNDS: return "device index out of range";
+    default: return "unknown status";
+  }
+}
+
+void moe_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns = ns ? ns : 1000000000ull;
+}
+
+moe_status_t moe_profile_enable(int on) {
+  if (on && !g_prof_created) {
+    for (int k = 0; k < MOE_PROF_KINDS; ++k)
+      for (int i = 0; i < kProfCap; ++i)
+        for (int w = 0; w < 2; ++w)
+          if (cudaEventCreate(&g_prof_ev[k][i][w]) != cudaSuccess) return MOE_ERR_CUDA;
+    g_prof_created = true;
+  }
+  for (int k = 0; k < MOE_PROF_KINDS; ++k) g_prof_n[k] = 0;
+  g_prof_on = on != 0;
+  return MOE_OK;
+}
+
+int moe_profile_collect(int kind, float* ms, int max_n) {
+  if (!g_prof_created || kind < 0 || kind >= MOE_PROF_KINDS) return 0;
+  const int n = std::min(g_prof_n[kind], max_n);
+  for (int i = 0; i < n; ++i) {
+    if (cudaEventSynchronize(g_prof_ev[kind][i][1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms[i], g_prof_ev[kind][i][0], g_prof_ev[kind][i][1]) !=
+            cudaSuccess)
+      return -1;
+  }
+  return n;
+}
+
+moe_status_t moe_get_device_status(moe_stream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return v;
+}
+
+// ------------------------------------------------------------------ route
+size_t moe_route_workspace_bytes(int T, int E, int k) {
+  if (T <= 0 || E <= 0 || k <= 0) return 256;
+  const int tpb = route_tokens_per_warp(k) * kRouteWarps;
+  const size_t nblk = (static_cast<size_t>(T) + tpb - 1) / tpb;
+  return align256(nblk * E * 4) + align256(static_cast<size_t>(T) * k * 4);
+}
+
+moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                            float* topk_w, int32_t* expert_counts,
+                            int32_t* expert_offsets, int32_t* dest, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  if (T < 0 || E < 1 || E > 512 || k < 1 || k > E) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (!expert_counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = stream;
+  if (T == 0) {
+    if (cudaMemsetAsync(expert_counts, 0, E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(expert_offsets, 0, (E + 1) * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (!logits || !topk_idx || !topk_w || !dest || !ws) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_route_workspace_bytes(T, E, k)) return MOE_ERR_INVALID_ARG;
+  ProfScope prof(MOE_PROF_ROUTE, st);
+  const int tpb = route_tokens_per_warp(k) * kRouteWarps;
+  const int nblk = (T + tpb - 1) / tpb;
+  int32_t* blk_hist = static_cast<int32_t*>(ws);
+  int32_t* local_rank = at<int32_t>(ws, align256(static_cast<size_t>(nblk) * E * 4));
+  const size_t smem = (2 * static_cast<size_t>(tpb) * k + kRouteWarps * E) * 4 +
+                      static_cast<size_t>(kRouteWarps) * k * 4;
+  const int epl = (E + 31) / 32;
+  auto launch = [&](auto kern) -> moe_status_t {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    kern<<<nblk, kRouteWarps * 32, smem, st>>>(logits, T, E, k, topk_idx, topk_w,
+                                               blk_hist, local_rank);
+    return launch_status();
+  };
+  moe_status_t s;
+  if (epl <= 1) s = launch(route_topk_kernel<1>);
+  else if (epl <= 2) s = launch(route_topk_kernel<2>);
+  else if (epl <= 4) s = launch(route_topk_kernel<4>);
+  else if (epl <= 8) s = launch(route_topk_kernel<8>);
+  else s = launch(route_topk_kernel<16>);
+  if (s != MOE_OK) return s;
+  const int P = std::max(1, 1024 / E);
+  const size_t smem2 = (static_cast<size_t>(P) * E + E + 1) * 4;
+  route_scan_kernel<<<1, 1024, smem2, st>>>(blk_hist, nblk, E, T * k, expert_counts,
+                                            expert_offsets);
+  if ((s = launch_status()) != MOE_OK) return s;
+  const int R = T * k;
+  const int grid = std::min((R + 255) / 256, std::max(1, num_sms()) * 8);
+  route_dest_kernel<<<grid, 256, 0, st>>>(topk_idx, blk_hist, local_rank, R, E, k, tpb,
+                                          dest);
+  return launch_status();
+}
+
+// ---------------------------------------------------------- permute / combine
+moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale, int T,
+                         int H, int k, void* Xp, const void* Zp, float* dw,
+                         moe_stream_t stream) {
+  if (T < 0 || H <= 0 || k < 1 || (H % 8)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!X || !dest || !Xp) return MOE_ERR_INVALID_ARG;
+  if ((dw == nullptr) != (Zp == nullptr)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Xp) |
+       reinterpret_cast<uintptr_t>(Zp)) & 15u)
+    return MOE_ERR_INVALID_ARG;
+  const int warps = 8;
+  const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
+  ProfScope prof(MOE_PROF_PERMUTE, stream);
+  permute_kernel<<<grid, warps * 32, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
+      static_cast<__nv_bfloat16*>(Xp), static_cast<const __nv_bfloat16*>(Zp), dw);
+  return launch_status();
+}
+
+moe_status_t moe_unpermute(const void* Yp, const int32_t* dest, const float* w, int T,
+                           int H, int k, void* Y, moe_stream_t stream) {
+  if (T < 0 || H <= 0 || k < 1 || (H % 8)) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!Yp || !dest || !Y) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(Yp) | reinterpret_cast<uintptr_t>(Y)) & 15u)
+    return MOE_ERR_INVALID_ARG;
+  const int warps = 8;
+  const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
+  ProfScope prof(MOE_PROF_UNPERMUTE, stream);
+  unpermute_kernel<<<grid, warps * 32, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(Yp), dest, w, T, H, k,
+      static_cast<__nv_bfloat16*>(Y));
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ sizes
+size_t moe_saved_bytes(int R, int H, int I, int r) {
+  if (R < 0 || H <= 0 || I <= 0 || r <= 0) return 0;
+  size_t off[5];
+  saved_layout(R, H, I, r, off);
+  return off[4];
+}
+
+size_t moe_saved_part_offset(int R, int H, int I, int r, int part) {
+  if (part < 0 || part > 4 || R < 0) return 0;
+  size_t off[5];
+  saved_layout(R, H, I, r, off);
+  return off[part];
+}
+
+size_t moe_workspace_bytes(int R, int E, int H, int I, int r) {
+  if (R < 0 || E <= 0 || H <= 0 || I <= 0 || r <= 0) return 0;
+  size_t off[8];
+  bwd_layout(R, E, H, I, r, off);
+  return off[7];
+}
+
+// ------------------------------------------------------------------ forward
+moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int E,
+                              int H, int I, int r, float s, const void* W1,
+                              const void* A1, const void* B1, const void* W2,
+                              const void* A2, const void* B2, int R, void* Z2,
+                              void* saved, size_t saved_bytes, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!shape_ok(E, H, I, r) || R < 0) return MOE_ERR_UNSUPPORTED;
+  if (R == 0) return MOE_OK;
+  if (!Xp || !expert_offsets || !W1 || !A1 || !B1 || !W2 || !A2 || !B2 || !Z2 || !saved)
+    return MOE_ERR_INVALID_ARG;
+  if (saved_bytes < moe_saved_bytes(R, H, I, r)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = stream;
+  size_t off[5];
+  saved_layout(R, H, I, r, off);
+  __nv_bfloat16* Z1 = at<__nv_bfloat16>(saved, off[0]);
+  __nv_bfloat16* h = at<__nv_bfloat16>(saved, off[1]);
+  __nv_bfloat16* xa1 = at<__nv_bfloat16>(saved, off[2]);
+  __nv_bfloat16* ha2 = at<__nv_bfloat16>(saved, off[3]);
+  moe_status_t stt;
+  if ((stt = zero_rank_padding(xa1, R, r, st)) != MOE_OK) return stt;
+  if ((stt = zero_rank_padding(ha2, R, r, st)) != MOE_OK) return stt;
+  const CUtensorMapSwizzle lsw = lora_swizzle(r);
+  const uint64_t EU = static_cast<uint64_t>(E);
+
+  // gate_up + SwiGLU
+  {
+    const int bn = pick_bn(I, true, r), half = bn / 2;
+    CUtensorMap ta, tb, tla, tlb;
+    bool ok = tmap_2d(&ta, Xp, H, R, H * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, half, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, A1, H, EU * r, H * 2ull, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tlb, B1, r, EU * 2 * I, r * 2ull, r, half, lsw);
+    if (!ok) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + half - 1) / half; g.I = I;
+    g.b_rows = 2 * I; g.lb_rows = 2 * I; g.s = s;
+    g.out = h; g.ld_out = I; g.out2 = Z1; g.ld_out2 = 2 * I;
+    g.lora_t = xa1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    if ((stt = launch_gemm<kGateUpFwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
+  }
+  // down
+  {
+    const int bn = pick_bn(H, false, r);
+    CUtensorMap ta, tb, tla, tlb;
+    bool ok = tmap_2d(&ta, h, I, R, I * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tb, W2, I, EU * H, I * 2ull, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, A2, I, EU * r, I * 2ull, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tlb, B2, r, EU * H, r * 2ull, r, bn, lsw);
+    if (!ok) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
+    g.b_rows = H; g.lb_rows = H; g.s = s;
+    g.out = static_cast<__nv_bfloat16*>(Z2); g.ld_out = H;
+    g.lora_t = ha2; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    if ((stt = launch_gemm<kDownFwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
+  }
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ backward
+moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
+                              const int32_t* expert_offsets, int E, int H, int I, int r,
+                              float s, const void* W1, const void* A1, const void* B1,
+                              const void* W2, const void* A2, const void* B2,
+                              const void* saved, size_t saved_bytes, int R, void* dXp,
+                              void* dA1, void* dB1, void* dA2, void* dB2, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+  if (!shape_ok(E, H, I, r) || R < 0) return MOE_ERR_UNSUPPORTED;
+  if (!dA1 || !dB1 || !dA2 || !dB2) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = stream;
+  if (R == 0) {
+    const size_t n = static_cast<size_t>(E) * r * 2;
+    if (cudaMemsetAsync(dA1, 0, n * H, st) != cudaSuccess ||
+        cudaMemsetAsync(dB1, 0, n * 2 * I, st) != cudaSuccess ||
+        cudaMemsetAsync(dA2, 0, n * I, st) != cudaSuccess ||
+        cudaMemsetAsync(dB2, 0, n * H, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (!dZ2 || !Xp || !expert_offsets || !W1 || !A1 || !B1 || !W2 || !A2 || !B2 ||
+      !saved || !dXp || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (saved_bytes < moe_saved_bytes(R, H, I, r)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_workspace_bytes(R, E, H, I, r)) return MOE_ERR_INVALID_ARG;
+  size_t so[5], wo[8];
+  saved_layout(R, H, I, r, so);
+  bwd_layout(R, E, H, I, r, wo);
+  const __nv_bfloat16* Z1 = at<__nv_bfloat16>(saved, so[0]);
+  const __nv_bfloat16* h = at<__nv_bfloat16>(saved, so[1]);
+  const __nv_bfloat16* xa1 = at<__nv_bfloat16>(saved, so[2]);
+  const __nv_bfloat16* ha2 = at<__nv_bfloat16>(saved, so[3]);
+  __nv_bfloat16* dZ1 = at<__nv_bfloat16>(ws, wo[0]);
+  __nv_bfloat16* dzb2 = at<__nv_bfloat16>(ws, wo[1]);
+  __nv_bfloat16* dzb1 = at<__nv_bfloat16>(ws, wo[2]);
+  __nv_bfloat16* B2t = at<__nv_bfloat16>(ws, wo[3]);
+  __nv_bfloat16* A2t = at<__nv_bfloat16>(ws, wo[4]);
+  __nv_bfloat16* B1t = at<__nv_bfloat16>(ws, wo[5]);
+  __nv_bfloat16* A1t = at<__nv_bfloat16>(ws, wo[6]);
+  moe_status_t stt;
+  if ((stt = zero_rank_padding(dzb2, R, r, st)) != MOE_OK) return stt;
+  if ((stt = zero_rank_padding(dzb1, R, r, st)) != MOE_OK) return stt;
+  // K-major copies of the LoRA factors used as MMA operands
+  if ((stt = transpose(B2, B2t, E, H, r, st)) != MOE_OK) return stt;
+  if ((stt = transpose(A2, A2t, E, r, I, st)) != MOE_OK) return stt;
+  if ((stt = transpose(B1, B1t, E, 2 * I, r, st)) != MOE_OK) return stt;
+  if ((stt = transpose(A1, A1t, E, r, H, st)) != MOE_OK) return stt;
+  const CUtensorMapSwizzle lsw = lora_swizzle(r);
+  const uint64_t EU = static_cast<uint64_t>(E);
+
+  // down backward: dh = dZ2 W2 + s (dZ2 B2) A2, SwiGLU backward -> dZ1
+  {
+    const int bn = pick_bn(I, false, r);
+    CUtensorMap ta, tb, tla, tlb;
+    bool ok = tmap_2d(&ta, dZ2, H, R, H * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tb, W2, I, EU * H, I * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, B2t, H, EU * r, H * 2ull, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tlb, A2t, r, EU * I, r * 2ull, r, bn, lsw);
+    if (!ok) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + bn - 1) / bn; g.I = I;
+    g.b_rows = H; g.lb_rows = I; g.s = s;
+    g.out = dZ1; g.ld_out = 2 * I; g.aux = Z1; g.ld_aux = 2 * I;
+    g.lora_t = dzb2; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    if ((stt = launch_gemm<kDownBwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
+  }
+  // gate_up backward: dXp = dZ1 W1 + s (dZ1 B1) A1
+  {
+    const int bn = pick_bn(H, false, r);
+    CUtensorMap ta, tb, tla, tlb;
+    bool ok = tmap_2d(&ta, dZ1, 2 * I, R, 4ull * I, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, B1t, 2 * I, EU * r, 4ull * I, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tlb, A1t, r, EU * H, r * 2ull, r, bn, lsw);
+    if (!ok) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
+    g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
+    g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
+    g.lora_t = dzb1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    if ((stt = launch_gemm<kGateUpBwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
+  }
+  // LoRA gradients
+  {
+    const int ldr = ld_rank(R);
+    const void* U[4] = {Xp, dZ1, h, dZ2};
+    const void* V[4] = {dzb1, xa1, dzb2, ha2};
+    const int P[4] = {H, 2 * I, I, H};
+    void* out[4] = {dA1, dB1, dA2, dB2};
+    const int tr[4] = {1, 0, 1, 0};
+    CUtensorMap tu[4], tv[4];
+    GradArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.wait_ns = g_wait_limit_ns;
+    int begin = 0;
+    for (int i = 0; i < 4; ++i) {
+      bool ok = tmap_2d(&tu[i], U[i], P[i], R, P[i] * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+      ok = ok && tmap_2d(&tv[i], V[i], ldr, r, ldr * 2ull, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+      if (!ok) return MOE_ERR_CUDA;
+      g.prob[i].P = P[i];
+      g.prob[i].p_tiles = (P[i] + 127) / 128;
+      g.prob[i].tile_begin = begin;
+      g.prob[i].transpose_out = tr[i];
+      g.prob[i].out = static_cast<__nv_bfloat16*>(out[i]);
+      begin += E * g.prob[i].p_tiles;
+    }
+    g.total_tiles = begin;
+    if (r == 16) stt = launch_grad_t<16>(tu, tv, g, st);
+    else if (r == 32) stt = launch_grad_t<32>(tu, tv, g, st);
+    else stt = launch_grad_t<64>(tu, tv, g, st);
+    if (stt != MOE_OK) return stt;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,194 @@
+// a2 / a6: gather tokens into expert order (optionally scaled by the routing
+// weight, optionally with the routing-weight gradient), and a5 / a10: the
+// weighted combine back to token order.  Both are HBM-bound copies: one warp
+// per token, 16-byte vector accesses, several loads in flight per lane.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t scale2(uint32_t v, float c) {
+  return pack_bf16x2(bf16_lo(v) * c, bf16_hi(v) * c);
+}
+
+__device__ __forceinline__ float dot8(uint4 a, uint4 b) {
+  float s = bf16_lo(a.x) * bf16_lo(b.x);
+  s = fmaf(bf16_hi(a.x), bf16_hi(b.x), s);
+  s = fmaf(bf16_lo(a.y), bf16_lo(b.y), s);
+  s = fmaf(bf16_hi(a.y), bf16_hi(b.y), s);
+  s = fmaf(bf16_lo(a.z), bf16_lo(b.z), s);
+  s = fmaf(bf16_hi(a.z), bf16_hi(b.z), s);
+  s = fmaf(bf16_lo(a.w), bf16_lo(b.w), s);
+  s = fmaf(bf16_hi(a.w), bf16_hi(b.w), s);
+  return s;
+}
+
+constexpr int kCopyUnroll = 4;
+
+// Xp[dest[t,j]] = (scale ? scale[t,j] : 1) * X[t]; optional dw[t,j] =
+// <X[t], Zp[dest[t,j]]>.  One warp per token, grid-stride over tokens.
+__global__ void __launch_bounds__(256)
+    permute_kernel(const __nv_bfloat16* __restrict__ X,
+                   const int32_t* __restrict__ dest,
+                   const float* __restrict__ scale, int T, int H, int k,
+                   __nv_bfloat16* __restrict__ Xp,
+                   const __nv_bfloat16* __restrict__ Zp,
+                   float* __restrict__ dw) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int nvec = H >> 3;
+  const int R = T * k;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+    const char* xrow = reinterpret_cast<const char*>(X + static_cast<size_t>(t) * H);
+    for (int j = 0; j < k; ++j) {
+      const int d = dest[static_cast<size_t>(t) * k + j];
+      if (d < 0 || d >= R) {
+        if (lane == 0) set_status(5);
+        continue;
+      }
+      const float c = scale ? scale[static_cast<size_t>(t) * k + j] : 1.f;
+      char* orow = reinterpret_cast<char*>(Xp + static_cast<size_t>(d) * H);
+      const char* zrow =
+          Zp ? reinterpret_cast<const char*>(Zp + static_cast<size_t>(d) * H)
+             : nullptr;
+      float acc = 0.f;
+      for (int v0 = lane; v0 < nvec; v0 += 32 * kCopyUnroll) {
+        uint4 x[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nvec) x[u] = ld_v4(xrow + 16 * static_cast<size_t>(v));
+        }
+        if (dw) {
+#pragma unroll
+          for (int u = 0; u < kCopyUnroll; ++u) {
+            const int v = v0 + 32 * u;
+            if (v < nvec) acc += dot8(x[u], ld_nc_v4(zrow + 16 * static_cast<size_t>(v)));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nvec) {
+            uint4 y = x[u];
+            if (scale) {
+              y.x = scale2(y.x, c);
+              y.y = scale2(y.y, c);
+              y.z = scale2(y.z, c);
+              y.w = scale2(y.w, c);
+            }
+            st_v4(orow + 16 * static_cast<size_t>(v), y);
+          }
+        }
+      }
+      if (dw) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) dw[static_cast<size_t>(t) * k + j] = acc;
+      }
+    }
+  }
+}
+
+// Y[t] = sum_j (w ? w[t,j] : 1) * Yp[dest[t,j]], fp32 in j order -> bf16.
+__global__ void __launch_bounds__(256)
+    unpermute_kernel(const __nv_bfloat16* __restrict__ Yp,
+                     const int32_t* __restrict__ dest,
+                     const float* __restrict__ w, int T, int H, int k,
+                     __nv_bfloat16* __restrict__ Y) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int nvec = H >> 3;
+  const int R = T * k;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+    char* yrow = reinterpret_cast<char*>(Y + static_cast<size_t>(t) * H);
+    for (int v0 = lane; v0 < nvec; v0 += 64) {
+      float acc[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+      for (int j = 0; j < k; ++j) {
+        int d = dest[static_cast<size_t>(t) * k + j];
+        if (d < 0 || d >= R) {
+          if (lane == 0) set_status(5);
+          continue;
+        }
+        const float c = w ? w[static_cast<size_t>(t) * k + j] : 1.f;
+        const char* zrow = reinterpret_cast<const char*>(Yp + static_cast<size_t>(d) * H);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nvec) {
+            const uint4 z = ld_nc_v4(zrow + 16 * static_cast<size_t>(v));
+            acc[u][0] = fmaf(c, bf16_lo(z.x), acc[u][0]);
+            acc[u][1] = fmaf(c, bf16_hi(z.x), acc[u][1]);
+            acc[u][2] = fmaf(c, bf16_lo(z.y), acc[u][2]);
+            acc[u][3] = fmaf(c, bf16_hi(z.y), acc[u][3]);
+            acc[u][4] = fmaf(c, bf16_lo(z.z), acc[u][4]);
+            acc[u][5] = fmaf(c, bf16_hi(z.z), acc[u][5]);
+            acc[u][6] = fmaf(c, bf16_lo(z.w), acc[u][6]);
+            acc[u][7] = fmaf(c, bf16_hi(z.w), acc[u][7]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < nvec) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+          o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+          o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+          o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+          st_v4(yrow + 16 * static_cast<size_t>(v), o);
+        }
+      }
+    }
+  }
+}
+
+// out[b][q][p] = in[b][p][q] for bf16 matrices [nb][P][Q] (LoRA factors only).
+__global__ void transpose_kernel(const __nv_bfloat16* __restrict__ in,
+                                 __nv_bfloat16* __restrict__ out, int P, int Q) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const size_t b = blockIdx.z;
+  const __nv_bfloat16* src = in + b * static_cast<size_t>(P) * Q;
+  __nv_bfloat16* dst = out + b * static_cast<size_t>(P) * Q;
+  const int q0 = blockIdx.x * 32, p0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int p = p0 + i, q = q0 + threadIdx.x;
+    if (p < P && q < Q) tile[i][threadIdx.x] = src[static_cast<size_t>(p) * Q + q];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int q = q0 + i, p = p0 + threadIdx.x;
+    if (p < P && q < Q) dst[static_cast<size_t>(q) * P + p] = tile[threadIdx.x][i];
+  }
+}
+
+}  // namespace moe
