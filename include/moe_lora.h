@@ -77,6 +77,35 @@ MOE_API moe_status_t moe_route_topk(const float* logits, int T, int E, int k,
                             int32_t* dest, void* ws, size_t ws_bytes,
                             moe_stream_t stream);
 
+/* Allocation-free variant of moe_route_topk (the pages have no counterpart:
+ * this is an interface convenience, not part of the method).
+ * Some callers cannot allocate device memory at the time they route: for
+ * example a plugin whose enqueue hook runs inside a host engine that owns all
+ * device memory and forbids cudaMalloc there, or code running under a fixed
+ * memory budget decided at start-up.  This entry point needs no workspace:
+ * its scratch is a 4 MiB array inside the library's own device memory (every
+ * GPU that loads the library holds it until the process exits).  It computes
+ * exactly what moe_route_topk computes; the caller still passes the logits
+ * and all outputs.  It calls no cudaMalloc / cudaFree and no allocating
+ * library routine.
+ *  - Limit: moe_route_workspace_bytes(T, E, k) must not exceed
+ *    moe_route_noalloc_max_workspace_bytes() (4 MiB; e.g. T <= 65536 tokens
+ *    with k <= 8 and E <= 512); larger sizes return MOE_ERR_UNSUPPORTED
+ *    before anything is launched.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps the last call's contents.
+ *    Nothing in it needs to start at zero (each call writes every scratch
+ *    byte it reads before reading it), but calls whose work overlaps on the
+ *    GPU (other streams, other threads) race on it: serialise them. */
+MOE_API moe_status_t moe_route_topk_noalloc(const float* logits, int T, int E, int k,
+                                            int32_t* topk_idx, float* topk_w,
+                                            int32_t* expert_counts,
+                                            int32_t* expert_offsets, int32_t* dest,
+                                            moe_stream_t stream);
+MOE_API size_t moe_route_noalloc_max_workspace_bytes(void);
+
 /* ------------------------------------------------------- a2 / a6: permute
  * Gather into expert order: Xp[dest[t, j]] = scale[t, j] * X[t] (scale NULL
  * means 1; with scale the product is formed in fp32 and rounded to bf16).

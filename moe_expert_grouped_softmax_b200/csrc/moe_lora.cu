@@ -19,7 +19,38 @@
 
 using namespace moe;
 
+// Scratch of moe_route_topk_noalloc: a fixed array in the library's own device
+// memory, so that entry point never needs a caller-provided workspace and never
+// allocates.  Every GPU that loads the library holds these bytes until the
+// process exits.  In host code `g_route_scratch` is only a host-side stand-in
+// for the symbol, never a device address: its device address is obtained with
+// cudaGetSymbolAddress on each device (see route_scratch_on_current_device).
+constexpr size_t kRouteScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
+
 namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_route_scratch_mu;
+void* g_route_scratch_dev[kMaxDevices] = {};
+
+// Device address of g_route_scratch on the current device, looked up once per
+// device (the first call on a device does the lookup, with that device
+// current) and cached.
+moe_status_t route_scratch_on_current_device(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_route_scratch_mu);
+  if (g_route_scratch_dev[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
+      return MOE_ERR_CUDA;
+    g_route_scratch_dev[dev] = p;
+  }
+  *out = g_route_scratch_dev[dev];
+  return MOE_OK;
+}
 
 uint64_t g_wait_limit_ns = 1000000000ull;  // one second per bounded wait
 
@@ -337,6 +368,24 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
                                           dest);
   return launch_status();
 }
+
+// Same routing as moe_route_topk, with the scratch in g_route_scratch instead
+// of a caller-provided workspace; allocates nothing.
+moe_status_t moe_route_topk_noalloc(const float* logits, int T, int E, int k,
+                                    int32_t* topk_idx, float* topk_w,
+                                    int32_t* expert_counts, int32_t* expert_offsets,
+                                    int32_t* dest, moe_stream_t stream) {
+  if (T < 0 || E < 1 || E > 512 || k < 1 || k > E) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (moe_route_workspace_bytes(T, E, k) > kRouteScratchBytes) return MOE_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const moe_status_t st = route_scratch_on_current_device(&scratch);
+  if (st != MOE_OK) return st;
+  return moe_route_topk(logits, T, E, k, topk_idx, topk_w, expert_counts, expert_offsets,
+                        dest, scratch, kRouteScratchBytes, stream);
+}
+
+size_t moe_route_noalloc_max_workspace_bytes(void) { return kRouteScratchBytes; }
 
 // ---------------------------------------------------------- permute / combine
 moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale, int T,
