@@ -59,56 +59,76 @@ def dist_env():
 
 
 class Clocks:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons with nvidia-smi (every 50 ms,
+    into a file) and keeps the samples taken inside [t_begin, t_end]."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.path = None
+        self.t_begin = self.t_end = None
 
-    def __enter__(self):
-        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        return self
+        time.sleep(1.0)  # let the sampler come up before the timed span
 
-    def __exit__(self, *a):
-        self.lines = []
+    def stop(self):
         if self.proc is not None:
+            time.sleep(0.1)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        import datetime as dt
+        sm, mx, pw, reasons = [], None, [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        lines = open(self.path).read().splitlines() if self.path else []
+        for l in lines:
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 8:
+            if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[0]))
-                mx = float(f[1])
+                ts = dt.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, mxx = float(f[1]), float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[4:8]):
+            if self.t_begin is not None and not (self.t_begin - 0.06 <= ts <= self.t_end + 0.06):
+                continue
+            sm.append(clk)
+            mx = mxx
+            try:
+                pw.append(float(f[3]))
+            except ValueError:
+                pass
+            for n, v in zip(names, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.path:
+            os.unlink(self.path)
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+               "reasons": sorted(reasons), "samples": len(sm)}
+        if pw:
+            out["power_w_max"] = max(pw)
+        return out
 
 
 # ---------------------------------------------------------------------------
@@ -146,26 +166,30 @@ def run_ours(args, cfg):
     K = args.steps
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clk = Clocks(local)
+    clk.start()
     ops.profile_enable(True)
     barrier()
     torch.cuda.synchronize()
-    with Clocks(local) as clk:
-        for i in range(K):
-            flush.zero_()                      # L2 flush, outside the timed span
-            ev0[i].record(stream)
-            blk.step(X, logits, dY, W)
-            ev1[i].record(stream)
-        torch.cuda.synchronize()
+    clk.t_begin = time.time()
+    for i in range(K):
+        flush.zero_()                      # L2 flush, outside the timed span
+        ev0[i].record(stream)
+        blk.step(X, logits, dY, W)
+        ev1[i].record(stream)
+    torch.cuda.synchronize()
+    clk.t_end = time.time()
     barrier()
-    ops.profile_enable(False)
+    clk.stop()
     ms_steps = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     ms_total = float(sum(ms_steps))
     kern = {}
-    for kind in ops.PROF_KINDS:
+    for kind in ops.PROF_KINDS:   # collect before the hook is switched off
         d = ops.profile_collect(kind)
         if d:
             kern[kind] = {"launches": len(d), "avg_ms": float(np.mean(d)),
                           "total_ms": float(np.sum(d))}
+    ops.profile_enable(False)
     st = ops.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after timed steps")
@@ -254,17 +278,21 @@ def cpu_oracle_sample(cfg, n_tok):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="gpt-oss-20b", choices=list(S.CONFIGS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=128)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (small cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     cfg = S.make_config(args.config)
+    if args.tokens:
+        cfg["T"] = args.tokens
     T, H, I, E, k, r = (cfg[x] for x in ("T", "H", "I", "E", "k", "r"))
     R = T * k
     flops = WL.block_flops(T, H, I, E, k, r)["total"]
