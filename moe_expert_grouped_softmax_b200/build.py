@@ -24,7 +24,7 @@ DEPS = ["ptx.cuh", "route.cuh", "permute.cuh", "gemm.cuh", "lora_grad.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
-    "-O3", "-lineinfo", "-std=c++17",
+    "-O3", "-lineinfo", "-std=c++20",
     "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "--expt-relaxed-constexpr",
     "-cudart", "static",

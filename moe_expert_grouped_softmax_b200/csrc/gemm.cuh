@@ -1,24 +1,26 @@
 // a3 / a4 / a7 / a8: persistent grouped GEMM over ragged experts on the
 // 5th-generation tensor cores, with the split-LoRA product fused in.
 //
-// Per output tile (128 rows of one expert x BN columns):
-//   mainloop  : acc  += A_k * B_k^T          (base weight, fp32 in TMEM)
-//               lora += A_k * LA_k^T         (rank-r down-projection, same A
-//                                             tile from shared memory)
-//   then      : xa    = bf16(s * lora)        (TMEM -> registers -> smem)
-//               acc  += xa * LB^T             (rank-r up-projection, second
-//                                             accumulate into the same tile)
-//   epilogue  : mode-specific (SwiGLU, plain store, SwiGLU backward).
+// Per output tile (128 rows of one expert x BN columns), with the TMEM
+// accumulator D = [acc (BN columns) | lora (r columns)]:
+//   mainloop : D += A_k * [B_k ; LA_k]^T   one MMA of N = BN + r per K-slice:
+//              the rank-r down-projection factor LA rides in the B operand,
+//              so A is read from shared memory once for both products;
+//   handoff  : xa = bf16(s * lora)          TMEM -> registers -> shared memory
+//   up       : acc += xa * LB^T             the rank-r up-projection, a second
+//              accumulate (K = r) into the same TMEM tile, issued while the
+//              next tile's mainloop is already running;
+//   epilogue : mode-specific (SwiGLU, plain store, SwiGLU backward).
 // This is the "split LoRA" order of the Unsloth page "Fine-tune MoE LLMs 12x
 // faster with Unsloth" (section "Faster LoRA MoE training"): x W^T +
 // s (x A^T) B^T, so W + s B A is never formed.
 //
 // Roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
 // owner), warps 2..5 = epilogue (TMEM lane quarter = warp % 4).  TMEM holds
-// two accumulator sets (256 columns each: BN base + r LoRA) so the epilogue
-// of one tile overlaps the mainloop of the next.  Tiles are enumerated on the
-// device from expert_offsets (no host synchronisation): m-tiles of all
-// experts in expert order, n fastest.
+// two accumulators of 256 columns, so the epilogue of one tile overlaps the
+// mainloop of the next.  Tiles are enumerated on the device from
+// expert_offsets (no host synchronisation): m-tiles of all experts in expert
+// order, n fastest.
 #pragma once
 
 #include "ptx.cuh"
@@ -54,19 +56,22 @@ struct GemmArgs {
 
 constexpr int kSmemOptin = 232448;  // max dynamic shared memory per block
 
-template <int BN, int RK>
+template <int MODE, int BN, int RK>
 struct GemmCfg {
+  static constexpr bool kBMN = (MODE == kDownBwd || MODE == kGateUpBwd);
   static constexpr int BM = 128, BK = 64;
+  static constexpr int NMMA = BN + RK;  // N of the fused mainloop MMA
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int LA_BYTES = RK * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + LA_BYTES;
+  // K-major: BN weight rows then r factor rows, 128 B each.  MN-major: BN/64
+  // weight atoms then one 64-column atom holding the (zero-padded) factor.
+  static constexpr int B_BYTES = kBMN ? (BN / 64 + 1) * 8192 : NMMA * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int LB_BYTES = BN * RK * 2;
   static constexpr int XA_BYTES = BM * RK * 2;
   static constexpr int MISC_BYTES = 256 + 8 * 520;  // barriers, flags, tables
   static constexpr int FIXED = 2 * LB_BYTES + 2 * XA_BYTES + MISC_BYTES;
   static constexpr int NS_FIT = (kSmemOptin - 1024 - FIXED) / STAGE_BYTES;
-  static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + FIXED;
   static constexpr int LSPAN = RK * 2;  // bytes of one LoRA row = swizzle span
   static constexpr uint32_t LLAYOUT =
@@ -75,8 +80,9 @@ struct GemmCfg {
   static constexpr int ACC_STRIDE = 256;
   static_assert(NS >= 2, "not enough shared memory for two stages");
   static_assert(SMEM_BYTES <= kSmemOptin, "shared memory over the opt-in limit");
-  static_assert(BN + RK <= ACC_STRIDE, "TMEM: BN + r must fit 256 columns");
-  static_assert(BN % 64 == 0, "BN must be a multiple of 64");
+  static_assert(NMMA <= ACC_STRIDE && NMMA % 16 == 0, "MMA N = BN + r");
+  static_assert(BN % 16 == 0, "BN must be a multiple of 16");
+  static_assert(!kBMN || BN % 64 == 0, "MN-major B needs 64-column atoms");
   static_assert(RK == 16 || RK == 32 || RK == 64, "rank must be 16, 32 or 64");
 };
 
@@ -152,6 +158,11 @@ __device__ __forceinline__ void build_tile_table(const int32_t* offsets, int E,
   if (any_bad && lane == 0) set_status(5);
 }
 
+__device__ __forceinline__ uint4 pack8(const float* v) {
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                    pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
 template <int MODE, int BN, int RK>
 __global__ void __launch_bounds__(192, 1)
     grouped_lora_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -159,9 +170,9 @@ __global__ void __launch_bounds__(192, 1)
                              const __grid_constant__ CUtensorMap tmLA,
                              const __grid_constant__ CUtensorMap tmLB,
                              const GemmArgs args) {
-  using C = GemmCfg<BN, RK>;
+  using C = GemmCfg<MODE, BN, RK>;
   constexpr bool kSwiGLU = (MODE == kGateUpFwd);
-  constexpr bool kBMN = (MODE == kDownBwd || MODE == kGateUpBwd);
+  constexpr bool kBMN = C::kBMN;
   constexpr int HALF = BN / 2;
 
   extern __shared__ uint8_t smem_raw[];
@@ -264,14 +275,20 @@ __global__ void __launch_bounds__(192, 1)
             for (int i = 0; i < BN / 64; ++i)
               tma_load_2d(sb + i * 8192, &tmB, &full[stage], nt * BN + 64 * i,
                           e * args.b_rows + kt * C::BK);
-          } else if (kSwiGLU) {
-            tma_load_2d(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * HALF);
-            tma_load_2d(sb + HALF * 128, &tmB, &full[stage], kt * C::BK,
-                        e * args.b_rows + args.I + nt * HALF);
+            // factor atom: [K rows, 64 columns] zero-padded past r
+            tma_load_2d(sb + (BN / 64) * 8192, &tmLA, &full[stage], 0,
+                        e * args.b_rows + kt * C::BK);
           } else {
-            tma_load_2d(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * BN);
+            if (kSwiGLU) {
+              tma_load_2d(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * HALF);
+              tma_load_2d(sb + HALF * 128, &tmB, &full[stage], kt * C::BK,
+                          e * args.b_rows + args.I + nt * HALF);
+            } else {
+              tma_load_2d(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * BN);
+            }
+            // factor rows right after the weight rows: one operand of N = BN + r
+            tma_load_2d(sb + BN * 128, &tmLA, &full[stage], kt * C::BK, e * RK);
           }
-          tma_load_2d(sb + C::B_BYTES, &tmLA, &full[stage], kt * C::BK, e * RK);
           if (armed_stages < C::NS) ++armed_stages;
           if (++stage == C::NS) {
             stage = 0;
@@ -281,8 +298,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       // Wait until every load issued has landed before the CTA may exit.
       for (int i = 0; i < armed_stages; ++i) {
-        // the last arming of stage s had parity (phase of that arming)
-        int s = stage - 1 - i;
+        int s = stage - 1 - i;  // the most recent arming of stage s
         uint32_t ph = phase;
         if (s < 0) {
           s += C::NS;
@@ -296,56 +312,78 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescMain = idesc_bf16_f32(128, BN, false, kBMN);
-      constexpr uint32_t kIdescLora = idesc_bf16_f32(128, RK, false, false);
+      constexpr uint32_t kIdesc = idesc_bf16_f32(128, C::NMMA, false, kBMN);
       constexpr uint32_t kIdescUp = idesc_bf16_f32(128, BN, false, false);
+      // acc[b] += xa[b] * LB[b]^T, then release LB[b] and publish acc[b]
+      auto issue_up = [&](int b) {
+        const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
+        const uint32_t xa0 = smem_u32(sXA + b * C::XA_BYTES);
+        const uint32_t lb0 = smem_u32(sLB + b * C::LB_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < RK / 16; ++kk)
+          umma_bf16(t_acc, smem_desc(xa0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
+                    smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), kIdescUp, 1u);
+        umma_commit(&lb_empty[b]);
+        umma_commit(&acc_full[b]);
+      };
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
+      int pending = -1;  // local index of the tile whose up-projection is due
+      bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++local) {
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
-        const uint32_t t_lora = t_acc + BN;
-        if (!mbar_wait(&acc_empty[b], use ^ 1, s_abort, wait_ns)) break;
+        if (!mbar_wait(&acc_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
         tc_fence_after();
-        bool ok = true;
         for (int kt = 0; kt < k_iters; ++kt) {
           if (!mbar_wait(&full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sStage + stage * C::STAGE_BYTES);
           const uint32_t b0 = a0 + C::A_BYTES;
-          const uint32_t la0 = b0 + C::B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
             const uint64_t da = smem_desc(a0 + kk * 32, 16, 1024, kLayoutSW128);
             const uint64_t db = kBMN ? smem_desc(b0 + kk * 2048, 8192, 1024, kLayoutSW128)
                                      : smem_desc(b0 + kk * 32, 16, 1024, kLayoutSW128);
-            const uint64_t dla = smem_desc(la0 + kk * 32, 16, 1024, kLayoutSW128);
-            const uint32_t accum = (kt | kk) ? 1u : 0u;
-            umma_bf16(t_acc, da, db, kIdescMain, accum);
-            umma_bf16(t_lora, da, dla, kIdescLora, accum);
+            umma_bf16(t_acc, da, db, kIdesc, (kt | kk) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == C::NS) {
             stage = 0;
             phase ^= 1;
           }
+          if (pending >= 0) {  // previous tile's up-projection, once it is ready
+            const int pb = pending & 1;
+            const uint32_t pu = (pending >> 1) & 1;
+            if (mbar_test_wait(&xa_ready[pb], pu) && mbar_test_wait(&lb_full[pb], pu)) {
+              tc_fence_after();
+              issue_up(pb);
+              pending = -1;
+            }
+          }
         }
         if (!ok) break;
         umma_commit(&lora_full[b]);
-        if (!mbar_wait(&xa_ready[b], use, s_abort, wait_ns)) break;
-        if (!mbar_wait(&lb_full[b], use, s_abort, wait_ns)) break;
-        tc_fence_after();
-        const uint32_t xa0 = smem_u32(sXA + b * C::XA_BYTES);
-        const uint32_t lb0 = smem_u32(sLB + b * C::LB_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < RK / 16; ++kk) {
-          umma_bf16(t_acc, smem_desc(xa0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
-                    smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), kIdescUp, 1u);
+        if (pending >= 0) {
+          const int pb = pending & 1;
+          const uint32_t pu = (pending >> 1) & 1;
+          if (!mbar_wait(&xa_ready[pb], pu, s_abort, wait_ns) ||
+              !mbar_wait(&lb_full[pb], pu, s_abort, wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          issue_up(pb);
         }
-        umma_commit(&lb_empty[b]);
-        umma_commit(&acc_full[b]);
+        pending = local;
+      }
+      if (ok && pending >= 0) {
+        const int pb = pending & 1;
+        const uint32_t pu = (pending >> 1) & 1;
+        if (mbar_wait(&xa_ready[pb], pu, s_abort, wait_ns) &&
+            mbar_wait(&lb_full[pb], pu, s_abort, wait_ns)) {
+          tc_fence_after();
+          issue_up(pb);
+        }
       }
       // every MMA issued by this thread must be complete before TMEM is freed
       umma_commit(drain_bar);
@@ -379,14 +417,9 @@ __global__ void __launch_bounds__(192, 1)
         for (int i = 0; i < RK; ++i) xa[i] *= args.s;
         uint8_t* xt = sXA + b * C::XA_BYTES;
 #pragma unroll
-        for (int ch = 0; ch < RK / 8; ++ch) {
-          uint4 v;
-          v.x = pack_bf16x2(xa[8 * ch + 0], xa[8 * ch + 1]);
-          v.y = pack_bf16x2(xa[8 * ch + 2], xa[8 * ch + 3]);
-          v.z = pack_bf16x2(xa[8 * ch + 4], xa[8 * ch + 5]);
-          v.w = pack_bf16x2(xa[8 * ch + 6], xa[8 * ch + 7]);
-          *reinterpret_cast<uint4*>(xt + swz_offset(row_in_tile, ch, C::LSPAN)) = v;
-        }
+        for (int ch = 0; ch < RK / 8; ++ch)
+          *reinterpret_cast<uint4*>(xt + swz_offset(row_in_tile, ch, C::LSPAN)) =
+              pack8(xa + 8 * ch);
         if (nt == 0 && rvalid && args.lora_t != nullptr) {
 #pragma unroll
           for (int q = 0; q < RK; ++q)
@@ -398,100 +431,109 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&xa_ready[b]);
+      if constexpr (MODE == kDownBwd) {
+        // pull this row's saved gate / up segments into L2 while the
+        // up-projection and the next tile's mainloop run
+        if (rvalid) {
+          const int col0 = nt * BN;
+          const int ncol = min(BN, args.N - col0);
+          const __nv_bfloat16* gp = args.aux + static_cast<size_t>(grow) * args.ld_aux + col0;
+          prefetch_l2_bulk(gp, static_cast<uint32_t>(ncol) * 2u);
+          prefetch_l2_bulk(gp + args.I, static_cast<uint32_t>(ncol) * 2u);
+        }
+      }
 
       if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
       tc_fence_after();
-      if (kSwiGLU) {
-#pragma unroll 1
-        for (int c = 0; c < HALF; c += 32) {
-          float g[32], u[32];
-          tmem_ld32(t_acc + c, g);
-          tmem_ld32(t_acc + HALF + c, u);
+      if constexpr (kSwiGLU) {
+        // gate columns [0, HALF), up columns [HALF, BN) of the tile
+        const int col0 = nt * HALF;
+        __nv_bfloat16* hrow = args.out + static_cast<size_t>(grow) * args.ld_out;
+        __nv_bfloat16* zrow = args.out2 + static_cast<size_t>(grow) * args.ld_out2;
+        for_chunks<HALF>([&](int c, auto w) {
+          constexpr int W = decltype(w)::value;
+          float g[W], u[W];
+          tmem_ld<W>(t_acc + c, g);
+          tmem_ld<W>(t_acc + HALF + c, u);
           tmem_ld_wait();
-          const int col = nt * HALF + c;
           if (rvalid) {
-            __nv_bfloat16* hp = args.out + static_cast<size_t>(grow) * args.ld_out + col;
-            __nv_bfloat16* gp = args.out2 + static_cast<size_t>(grow) * args.ld_out2 + col;
-            __nv_bfloat16* up = gp + args.I;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (col + 8 * q < args.N) {
-                uint32_t hv[4], gv[4], uv[4];
+            for (int q = 0; q < W / 8; ++q) {
+              const int col = col0 + c + 8 * q;
+              if (col < args.N) {
+                float h[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float g0 = g[8 * q + 2 * i], g1 = g[8 * q + 2 * i + 1];
-                  const float u0 = u[8 * q + 2 * i], u1 = u[8 * q + 2 * i + 1];
-                  hv[i] = pack_bf16x2(g0 * sigmoidf_(g0) * u0, g1 * sigmoidf_(g1) * u1);
-                  gv[i] = pack_bf16x2(g0, g1);
-                  uv[i] = pack_bf16x2(u0, u1);
+                for (int i = 0; i < 8; ++i) {
+                  const float gg = g[8 * q + i];
+                  h[i] = gg * sigmoidf_(gg) * u[8 * q + i];
                 }
-                *reinterpret_cast<uint4*>(hp + 8 * q) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                *reinterpret_cast<uint4*>(gp + 8 * q) = make_uint4(gv[0], gv[1], gv[2], gv[3]);
-                *reinterpret_cast<uint4*>(up + 8 * q) = make_uint4(uv[0], uv[1], uv[2], uv[3]);
+                *reinterpret_cast<uint4*>(hrow + col) = pack8(h);
+                *reinterpret_cast<uint4*>(zrow + col) = pack8(g + 8 * q);
+                *reinterpret_cast<uint4*>(zrow + args.I + col) = pack8(u + 8 * q);
               }
             }
           }
-        }
-      } else if (MODE == kDownBwd) {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float dh[32];
-          tmem_ld32(t_acc + c, dh);
-          tmem_ld_wait();
-          const int col = nt * BN + c;
-          if (rvalid) {
-            const __nv_bfloat16* gp = args.aux + static_cast<size_t>(grow) * args.ld_aux + col;
-            const __nv_bfloat16* up = gp + args.I;
-            __nv_bfloat16* dgp = args.out + static_cast<size_t>(grow) * args.ld_out + col;
-            __nv_bfloat16* dup = dgp + args.I;
+        });
+      } else if constexpr (MODE == kDownBwd) {
+        const int col0 = nt * BN;
+        const __nv_bfloat16* grow_p = args.aux + static_cast<size_t>(grow) * args.ld_aux;
+        __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
+        for_chunks<BN>([&](int c, auto w) {
+          constexpr int W = decltype(w)::value;
+          uint4 gv[W / 8], uv[W / 8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (col + 8 * q < args.N) {
-                const uint4 gq = *reinterpret_cast<const uint4*>(gp + 8 * q);
-                const uint4 uq = *reinterpret_cast<const uint4*>(up + 8 * q);
-                const uint32_t ga[4] = {gq.x, gq.y, gq.z, gq.w};
-                const uint32_t ua[4] = {uq.x, uq.y, uq.z, uq.w};
-                uint32_t dg[4], du[4];
+          for (int q = 0; q < W / 8; ++q) {  // loads first: in flight during the TMEM read
+            const int col = col0 + c + 8 * q;
+            if (rvalid && col < args.N) {
+              gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
+              uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
+            }
+          }
+          float dh[W];
+          tmem_ld<W>(t_acc + c, dh);
+          tmem_ld_wait();
+          if (rvalid) {
+#pragma unroll
+            for (int q = 0; q < W / 8; ++q) {
+              const int col = col0 + c + 8 * q;
+              if (col < args.N) {
+                const uint32_t ga[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+                const uint32_t ua[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
+                float dg[8], du[8];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                  float gg[2] = {bf16_lo(ga[i]), bf16_hi(ga[i])};
-                  float uu[2] = {bf16_lo(ua[i]), bf16_hi(ua[i])};
-                  float o_g[2], o_u[2];
 #pragma unroll
                   for (int h2 = 0; h2 < 2; ++h2) {
+                    const float gg = h2 ? bf16_hi(ga[i]) : bf16_lo(ga[i]);
+                    const float uu = h2 ? bf16_hi(ua[i]) : bf16_lo(ua[i]);
                     const float d = dh[8 * q + 2 * i + h2];
-                    const float sg = sigmoidf_(gg[h2]);
-                    o_g[h2] = d * uu[h2] * sg * (1.f + gg[h2] * (1.f - sg));
-                    o_u[h2] = d * gg[h2] * sg;
+                    const float sg = sigmoidf_(gg);
+                    dg[2 * i + h2] = d * uu * sg * (1.f + gg * (1.f - sg));
+                    du[2 * i + h2] = d * gg * sg;
                   }
-                  dg[i] = pack_bf16x2(o_g[0], o_g[1]);
-                  du[i] = pack_bf16x2(o_u[0], o_u[1]);
                 }
-                *reinterpret_cast<uint4*>(dgp + 8 * q) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-                *reinterpret_cast<uint4*>(dup + 8 * q) = make_uint4(du[0], du[1], du[2], du[3]);
+                *reinterpret_cast<uint4*>(orow + col) = pack8(dg);
+                *reinterpret_cast<uint4*>(orow + args.I + col) = pack8(du);
               }
             }
           }
-        }
+        });
       } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float v[32];
-          tmem_ld32(t_acc + c, v);
+        const int col0 = nt * BN;
+        __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
+        for_chunks<BN>([&](int c, auto w) {
+          constexpr int W = decltype(w)::value;
+          float v[W];
+          tmem_ld<W>(t_acc + c, v);
           tmem_ld_wait();
-          const int col = nt * BN + c;
           if (rvalid) {
-            __nv_bfloat16* op = args.out + static_cast<size_t>(grow) * args.ld_out + col;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (col + 8 * q < args.N) {
-                *reinterpret_cast<uint4*>(op + 8 * q) = make_uint4(
-                    pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                    pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-              }
+            for (int q = 0; q < W / 8; ++q) {
+              const int col = col0 + c + 8 * q;
+              if (col < args.N) *reinterpret_cast<uint4*>(orow + col) = pack8(v + 8 * q);
             }
           }
-        }
+        });
       }
       tc_fence_before();
       __syncwarp();

@@ -145,22 +145,35 @@ bool shape_ok(int E, int H, int I, int r) {
   return true;
 }
 
-// Tile width along N: 192 unless it pads noticeably more than 128 does.
-int pick_bn(int n_cols, bool swiglu, int r) {
-  if (r == 64) return 128;
-  auto waste = [&](int bn) {
+// Tile width along N.  Forward (K-major B): 256 - r, 192 or 128; backward
+// (MN-major B, 64-column atoms): 192 or 128.  Picks the smallest estimated
+// cost tiles * (BN + r + 48), where 48 stands for the per-tile fixed work.
+int pick_bn(int n_cols, bool swiglu, int r, bool backward) {
+  const int fwd_c[3] = {256 - r, 192, 128};
+  const int bwd_c[2] = {192, 128};
+  const int* c = backward ? bwd_c : fwd_c;
+  const int nc = backward ? 2 : 3;
+  int best = 128;
+  double best_cost = 1e300;
+  for (int i = 0; i < nc; ++i) {
+    const int bn = c[i];
+    if (bn + r > 256) continue;
     const int w = swiglu ? bn / 2 : bn;
-    const int tiles = (n_cols + w - 1) / w;
-    return static_cast<double>(tiles * w - n_cols) / n_cols;
-  };
-  return waste(192) <= waste(128) + 0.02 ? 192 : 128;
+    const double tiles = (n_cols + w - 1) / w;
+    const double cost = tiles * (bn + r + 48);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
 }
 
 template <int MODE, int BN, int RK>
 moe_status_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b,
                            const CUtensorMap& la, const CUtensorMap& lb,
                            const GemmArgs& args, cudaStream_t st) {
-  using C = GemmCfg<BN, RK>;
+  using C = GemmCfg<MODE, BN, RK>;
   auto kern = grouped_lora_gemm_kernel<MODE, BN, RK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM_BYTES) != cudaSuccess)
@@ -180,10 +193,16 @@ template <int MODE>
 moe_status_t launch_gemm(int bn, int r, const CUtensorMap& a, const CUtensorMap& b,
                          const CUtensorMap& la, const CUtensorMap& lb,
                          const GemmArgs& args, cudaStream_t st) {
+  constexpr bool kFwd = (MODE == kGateUpFwd || MODE == kDownFwd);
+  if constexpr (kFwd) {
+    if (r == 16 && bn == 240) return launch_gemm_t<MODE, 240, 16>(a, b, la, lb, args, st);
+    if (r == 32 && bn == 224) return launch_gemm_t<MODE, 224, 32>(a, b, la, lb, args, st);
+  }
   if (r == 16 && bn == 192) return launch_gemm_t<MODE, 192, 16>(a, b, la, lb, args, st);
   if (r == 16 && bn == 128) return launch_gemm_t<MODE, 128, 16>(a, b, la, lb, args, st);
   if (r == 32 && bn == 192) return launch_gemm_t<MODE, 192, 32>(a, b, la, lb, args, st);
   if (r == 32 && bn == 128) return launch_gemm_t<MODE, 128, 32>(a, b, la, lb, args, st);
+  if (r == 64 && bn == 192) return launch_gemm_t<MODE, 192, 64>(a, b, la, lb, args, st);
   if (r == 64 && bn == 128) return launch_gemm_t<MODE, 128, 64>(a, b, la, lb, args, st);
   return MOE_ERR_UNSUPPORTED;
 }
@@ -224,10 +243,10 @@ void bwd_layout(int R, int E, int H, int I, int r, size_t off[8]) {
   off[0] = 0;                                                  // dZ1 [R, 2I]
   off[1] = off[0] + align256(dz1);                             // dZB2t [r, ldR]
   off[2] = off[1] + align256(vt);                              // dZB1t [r, ldR]
-  off[3] = off[2] + align256(vt);                              // B2t [E, r, H]
-  off[4] = off[3] + align256(static_cast<size_t>(E) * r * H * 2);   // A2t [E, I, r]
-  off[5] = off[4] + align256(static_cast<size_t>(E) * I * r * 2);   // B1t [E, r, 2I]
-  off[6] = off[5] + align256(static_cast<size_t>(E) * r * 2 * I * 2);  // A1t [E, H, r]
+  off[3] = off[2] + align256(vt);                              // B2p [E*H, 64]
+  off[4] = off[3] + align256(static_cast<size_t>(E) * H * 64 * 2);     // A2t [E, I, r]
+  off[5] = off[4] + align256(static_cast<size_t>(E) * I * r * 2);      // B1p [E*2I, 64]
+  off[6] = off[5] + align256(static_cast<size_t>(E) * 2 * I * 64 * 2);  // A1t [E, H, r]
   off[7] = off[6] + align256(static_cast<size_t>(E) * H * r * 2);
 }
 
@@ -248,6 +267,17 @@ moe_status_t zero_rank_padding(void* p, int R, int r, cudaStream_t st) {
                                           static_cast<size_t>(ld) * 2, 0,
                                           static_cast<size_t>(ld - R) * 2, r, st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// out [rows, 64] = in [rows, r] followed by zero columns (one MN-major
+// 64-column atom per K-slice for the backward's fused rank-r operand).
+moe_status_t pad_cols64(const void* in, void* out, long long rows, int r, cudaStream_t st) {
+  const long long n = rows * 8;  // 16-byte chunks of the output
+  const int grid = static_cast<int>(std::min<long long>((n + 255) / 256, 148ll * 16));
+  ProfScope prof(MOE_PROF_TRANSPOSE, st);
+  pad_cols64_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in),
+                                          static_cast<__nv_bfloat16*>(out), rows, r);
+  return launch_status();
 }
 
 moe_status_t transpose(const void* in, void* out, int nb, int P, int Q, cudaStream_t st) {
@@ -476,7 +506,7 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
 
   // gate_up + SwiGLU
   {
-    const int bn = pick_bn(I, true, r), half = bn / 2;
+    const int bn = pick_bn(I, true, r, false), half = bn / 2;
     CUtensorMap ta, tb, tla, tlb;
     bool ok = tmap_2d(&ta, Xp, H, R, H * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, half, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -493,7 +523,7 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
   }
   // down
   {
-    const int bn = pick_bn(H, false, r);
+    const int bn = pick_bn(H, false, r, false);
     CUtensorMap ta, tb, tla, tlb;
     bool ok = tmap_2d(&ta, h, I, R, I * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && tmap_2d(&tb, W2, I, EU * H, I * 2ull, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -546,28 +576,34 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
   __nv_bfloat16* dZ1 = at<__nv_bfloat16>(ws, wo[0]);
   __nv_bfloat16* dzb2 = at<__nv_bfloat16>(ws, wo[1]);
   __nv_bfloat16* dzb1 = at<__nv_bfloat16>(ws, wo[2]);
-  __nv_bfloat16* B2t = at<__nv_bfloat16>(ws, wo[3]);
+  const void* B2p = B2;  // [E*H, 64]: B2 itself when r = 64, else a padded copy
+  const void* B1p = B1;  // [E*2I, 64]
   __nv_bfloat16* A2t = at<__nv_bfloat16>(ws, wo[4]);
-  __nv_bfloat16* B1t = at<__nv_bfloat16>(ws, wo[5]);
   __nv_bfloat16* A1t = at<__nv_bfloat16>(ws, wo[6]);
   moe_status_t stt;
   if ((stt = zero_rank_padding(dzb2, R, r, st)) != MOE_OK) return stt;
   if ((stt = zero_rank_padding(dzb1, R, r, st)) != MOE_OK) return stt;
-  // K-major copies of the LoRA factors used as MMA operands
-  if ((stt = transpose(B2, B2t, E, H, r, st)) != MOE_OK) return stt;
+  // Operand copies of the LoRA factors: the down-projection factors B2, B1 as
+  // 64-column MN-major atoms (fused into the base MMA), the up-projection
+  // factors A2, A1 transposed to K-major.
+  if (r < 64) {
+    B2p = at<__nv_bfloat16>(ws, wo[3]);
+    B1p = at<__nv_bfloat16>(ws, wo[5]);
+    if ((stt = pad_cols64(B2, const_cast<void*>(B2p), 1ll * E * H, r, st)) != MOE_OK) return stt;
+    if ((stt = pad_cols64(B1, const_cast<void*>(B1p), 2ll * E * I, r, st)) != MOE_OK) return stt;
+  }
   if ((stt = transpose(A2, A2t, E, r, I, st)) != MOE_OK) return stt;
-  if ((stt = transpose(B1, B1t, E, 2 * I, r, st)) != MOE_OK) return stt;
   if ((stt = transpose(A1, A1t, E, r, H, st)) != MOE_OK) return stt;
   const CUtensorMapSwizzle lsw = lora_swizzle(r);
   const uint64_t EU = static_cast<uint64_t>(E);
 
   // down backward: dh = dZ2 W2 + s (dZ2 B2) A2, SwiGLU backward -> dZ1
   {
-    const int bn = pick_bn(I, false, r);
+    const int bn = pick_bn(I, false, r, true);
     CUtensorMap ta, tb, tla, tlb;
     bool ok = tmap_2d(&ta, dZ2, H, R, H * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && tmap_2d(&tb, W2, I, EU * H, I * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, B2t, H, EU * r, H * 2ull, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, B2p, 64, EU * H, 128, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && tmap_2d(&tlb, A2t, r, EU * I, r * 2ull, r, bn, lsw);
     if (!ok) return MOE_ERR_CUDA;
     GemmArgs g{};
@@ -580,11 +616,11 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
   }
   // gate_up backward: dXp = dZ1 W1 + s (dZ1 B1) A1
   {
-    const int bn = pick_bn(H, false, r);
+    const int bn = pick_bn(H, false, r, true);
     CUtensorMap ta, tb, tla, tlb;
     bool ok = tmap_2d(&ta, dZ1, 2 * I, R, 4ull * I, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, B1t, 2 * I, EU * r, 4ull * I, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, B1p, 64, EU * 2 * I, 128, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && tmap_2d(&tlb, A1t, r, EU * H, r * 2ull, r, bn, lsw);
     if (!ok) return MOE_ERR_CUDA;
     GemmArgs g{};

@@ -64,6 +64,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe: has the phase with this parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of `bar` with the given parity to complete.
 // Gives up when another role of the CTA has aborted (*abort != 0) or when
 // `limit_ns` has passed; in the latter case it records
@@ -100,6 +113,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m,
       "tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// Asynchronous prefetch of [p, p + bytes) into L2 (16-byte aligned, size a
+// multiple of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -161,6 +183,18 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 lanes x 32 bit, 8 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+        "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // 32 lanes x 32 bit, 16 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
@@ -194,6 +228,32 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
       : "r"(taddr));
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int W>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float* v) {
+  static_assert(W == 8 || W == 16 || W == 32, "TMEM load width");
+  if constexpr (W == 8) tmem_ld8(taddr, v);
+  else if constexpr (W == 16) tmem_ld16(taddr, v);
+  else tmem_ld32(taddr, v);
+}
+
+template <int N>
+struct Int {
+  static constexpr int value = N;
+};
+
+// Calls f(c, Int<W>) for consecutive column chunks [c, c + W) covering
+// [0, NC): chunks of 32, then at most one of 16 and one of 8 (NC % 8 == 0).
+template <int NC, typename F>
+__device__ __forceinline__ void for_chunks(F&& f) {
+  static_assert(NC % 8 == 0, "column count must be a multiple of 8");
+#pragma unroll 1
+  for (int c = 0; c + 32 <= NC; c += 32) f(c, Int<32>{});
+  constexpr int b16 = (NC / 32) * 32;
+  if constexpr (NC - b16 >= 16) f(b16, Int<16>{});
+  constexpr int b8 = b16 + ((NC - b16 >= 16) ? 16 : 0);
+  if constexpr (NC - b8 >= 8) f(b8, Int<8>{});
 }
 
 // ------------------------------------------------ UMMA operand descriptors
