@@ -191,6 +191,13 @@ MOE_API const char* moe_status_string(moe_status_t status);
  * succeed immediately give up, which exercises the timeout path. */
 MOE_API void moe_set_wait_limit_ns(uint64_t ns);
 
+/* Testing hook: while on, every grouped-GEMM kernel's MMA warp first waits on
+ * a barrier that nothing arrives on.  Its bounded wait runs out after the
+ * configured limit; the kernel then records MOE_ERR_DEVICE_TIMEOUT, lets the
+ * copies already in flight land, frees its tensor memory and returns.  This
+ * exercises the timeout path without faulting or hanging the GPU. */
+MOE_API void moe_test_inject_stall(int on);
+
 /* Benchmark hook (not thread-safe; for measurement only).
  * moe_profile_enable(1) starts recording, for every kernel kind below, a pair
  * of CUDA events around each of its launches on the launching stream (up to

@@ -52,6 +52,7 @@ struct GemmArgs {
   __nv_bfloat16* lora_t;   // [r, ld_lora] s-scaled rank-r product, transposed
   int ld_lora;
   uint64_t wait_ns;
+  int stall_test;          // testing: make the MMA warp's first wait run out
 };
 
 constexpr int kSmemOptin = 232448;  // max dynamic shared memory per block
@@ -108,12 +109,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-// Bounded wait that ignores the abort flag (used to drain work in flight).
+// Bounded wait that ignores the abort flag, used before exit to let copies
+// and MMAs already in flight land.  Its limit never drops below one second,
+// whatever the configured wait limit, so that a CTA does not leave while its
+// own asynchronous work is still writing into it.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity,
                                            uint64_t limit_ns) {
+  const uint64_t limit = limit_ns > 1000000000ull ? limit_ns : 1000000000ull;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) {
+    if (globaltimer_ns() - t0 > limit) {
       set_status(4);
       return;
     }
@@ -331,7 +336,11 @@ __global__ void __launch_bounds__(192, 1)
       int local = 0;
       int pending = -1;  // local index of the tile whose up-projection is due
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++local) {
+      // Testing hook: wait on a barrier that nothing arrives on before the
+      // end of the kernel, so the bounded wait runs out and the whole CTA
+      // takes its abort path.
+      if (args.stall_test) ok = mbar_wait(drain_bar, 0, s_abort, wait_ns);
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++local) {
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;

@@ -53,6 +53,7 @@ moe_status_t route_scratch_on_current_device(void** out) {
 }
 
 uint64_t g_wait_limit_ns = 1000000000ull;  // one second per bounded wait
+int g_stall_test = 0;                      // testing hook, see moe_test_inject_stall
 
 // ------------------------------------------------ optional per-kernel timing
 // When enabled, each launch site of a kernel kind records a CUDA event before
@@ -308,6 +309,8 @@ void moe_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns = ns ? ns : 1000000000ull;
 }
 
+void moe_test_inject_stall(int on) { g_stall_test = on ? 1 : 0; }
+
 moe_status_t moe_profile_enable(int on) {
   if (on && !g_prof_created) {
     for (int k = 0; k < MOE_PROF_KINDS; ++k)
@@ -344,9 +347,9 @@ moe_status_t moe_get_device_status(moe_stream_t stream) {
 // ------------------------------------------------------------------ route
 size_t moe_route_workspace_bytes(int T, int E, int k) {
   if (T <= 0 || E <= 0 || k <= 0) return 256;
-  const int tpb = route_tokens_per_warp(k) * kRouteWarps;
-  const size_t nblk = (static_cast<size_t>(T) + tpb - 1) / tpb;
-  return align256(nblk * E * 4) + align256(static_cast<size_t>(T) * k * 4);
+  const size_t R = static_cast<size_t>(T) * k;
+  const size_t nblk = (R + kRankChunk - 1) / kRankChunk;
+  return align256(nblk * E * 4) + align256(R * 4);
 }
 
 moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* topk_idx,
@@ -365,19 +368,20 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
   if (!logits || !topk_idx || !topk_w || !dest || !ws) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_route_workspace_bytes(T, E, k)) return MOE_ERR_INVALID_ARG;
   ProfScope prof(MOE_PROF_ROUTE, st);
-  const int tpb = route_tokens_per_warp(k) * kRouteWarps;
-  const int nblk = (T + tpb - 1) / tpb;
+  const int R = T * k;
+  const int nblk = (R + kRankChunk - 1) / kRankChunk;
   int32_t* blk_hist = static_cast<int32_t*>(ws);
   int32_t* local_rank = at<int32_t>(ws, align256(static_cast<size_t>(nblk) * E * 4));
-  const size_t smem = (2 * static_cast<size_t>(tpb) * k + kRouteWarps * E) * 4 +
-                      static_cast<size_t>(kRouteWarps) * k * 4;
+  // 1. top-k + weights, one token per warp
+  const size_t smem1 = static_cast<size_t>(kRouteWarps) * k * 4;
   const int epl = (E + 31) / 32;
+  const int grid1 = (T + kRouteWarps - 1) / kRouteWarps;
   auto launch = [&](auto kern) -> moe_status_t {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+    if (smem1 > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem1)) != cudaSuccess)
       return MOE_ERR_CUDA;
-    kern<<<nblk, kRouteWarps * 32, smem, st>>>(logits, T, E, k, topk_idx, topk_w,
-                                               blk_hist, local_rank);
+    kern<<<grid1, kRouteWarps * 32, smem1, st>>>(logits, T, E, k, topk_idx, topk_w);
     return launch_status();
   };
   moe_status_t s;
@@ -387,15 +391,19 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
   else if (epl <= 8) s = launch(route_topk_kernel<8>);
   else s = launch(route_topk_kernel<16>);
   if (s != MOE_OK) return s;
+  // 2. stable in-chunk ranks + chunk histograms
+  route_rank_kernel<<<nblk, kRankWarps * 32, static_cast<size_t>(kRankWarps) * E * 4, st>>>(
+      topk_idx, R, E, blk_hist, local_rank);
+  if ((s = launch_status()) != MOE_OK) return s;
+  // 3. expert totals, offsets and per-chunk base rows (one CTA)
   const int P = std::max(1, 1024 / E);
   const size_t smem2 = (static_cast<size_t>(P) * E + E + 1) * 4;
-  route_scan_kernel<<<1, 1024, smem2, st>>>(blk_hist, nblk, E, T * k, expert_counts,
+  route_scan_kernel<<<1, 1024, smem2, st>>>(blk_hist, nblk, E, R, expert_counts,
                                             expert_offsets);
   if ((s = launch_status()) != MOE_OK) return s;
-  const int R = T * k;
+  // 4. destination rows
   const int grid = std::min((R + 255) / 256, std::max(1, num_sms()) * 8);
-  route_dest_kernel<<<grid, 256, 0, st>>>(topk_idx, blk_hist, local_rank, R, E, k, tpb,
-                                          dest);
+  route_dest_kernel<<<grid, 256, 0, st>>>(topk_idx, blk_hist, local_rank, R, E, dest);
   return launch_status();
 }
 
@@ -519,6 +527,7 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     g.b_rows = 2 * I; g.lb_rows = 2 * I; g.s = s;
     g.out = h; g.ld_out = I; g.out2 = Z1; g.ld_out2 = 2 * I;
     g.lora_t = xa1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
     if ((stt = launch_gemm<kGateUpFwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   // down
@@ -536,6 +545,7 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     g.b_rows = H; g.lb_rows = H; g.s = s;
     g.out = static_cast<__nv_bfloat16*>(Z2); g.ld_out = H;
     g.lora_t = ha2; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
     if ((stt = launch_gemm<kDownFwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   return MOE_OK;
@@ -612,6 +622,7 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
     g.b_rows = H; g.lb_rows = I; g.s = s;
     g.out = dZ1; g.ld_out = 2 * I; g.aux = Z1; g.ld_aux = 2 * I;
     g.lora_t = dzb2; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
     if ((stt = launch_gemm<kDownBwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   // gate_up backward: dXp = dZ1 W1 + s (dZ1 B1) A1
@@ -629,6 +640,7 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
     g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
     g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
     g.lora_t = dzb1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
     if ((stt = launch_gemm<kGateUpBwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   // LoRA gradients

@@ -12,126 +12,115 @@
 
 namespace moe {
 
-constexpr int kRouteWarps = 8;
-
-__host__ __device__ inline int route_tokens_per_warp(int k) {
-  int t = 128 / k;
-  if (t < 1) t = 1;
-  if (t > 16) t = 16;
-  return t;
-}
+constexpr int kRouteWarps = 8;          // top-k: one token per warp
+constexpr int kRankWarps = 16;          // ranking: 16 warps per CTA
+constexpr int kRankPerWarp = 128;       // flat entries per warp
+constexpr int kRankChunk = kRankWarps * kRankPerWarp;  // entries per CTA
 
 __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
   return va > vb || (va == vb && ea < eb);
 }
 
 // One warp per token.  Lane l holds experts l, l+32, ... (EPL of them).
-// Writes topk idx / w, the block's expert histogram and, for every (t, j) of
-// the block, its rank among earlier same-expert entries of the block.
+// Writes the k selected experts (logit desc, index asc) and their
+// renormalised weights.  Per-warp scratch in shared memory: k values.
 template <int EPL>
 __global__ void __launch_bounds__(kRouteWarps * 32)
     route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                      int32_t* __restrict__ idx_out, float* __restrict__ w_out,
-                      int32_t* __restrict__ blk_hist,
-                      int32_t* __restrict__ local_rank) {
-  const int tpw = route_tokens_per_warp(k);
-  const int tpb = tpw * kRouteWarps;
+                      int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t_block = blockIdx.x * tpb;
-  const int per_warp = tpw * k;
-
-  extern __shared__ int smem_i[];
-  int* s_idx = smem_i;                       // [tpb * k]
-  int* s_rank = s_idx + tpb * k;             // [tpb * k]
-  int* s_cnt = s_rank + tpb * k;             // [kRouteWarps][E]
-  float* s_val = reinterpret_cast<float*>(s_cnt + kRouteWarps * E);  // [warps][k]
-
-  for (int i = threadIdx.x; i < kRouteWarps * E; i += blockDim.x) s_cnt[i] = 0;
-  __syncthreads();
-
-  float* my_val = s_val + warp * k;
-  for (int i = 0; i < tpw; ++i) {
-    const int t = t_block + warp * tpw + i;
-    if (t >= T) break;
-    float v[EPL];
-    uint32_t taken = 0;
+  extern __shared__ float s_val_all[];
+  float* my_val = s_val_all + warp * k;
+  const int t = blockIdx.x * kRouteWarps + warp;
+  if (t >= T) return;
+  float v[EPL];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int q = 0; q < EPL; ++q) {
+    const int e = lane + 32 * q;
+    if (e < E) {
+      const float x = __ldg(logits + static_cast<size_t>(t) * E + e);
+      v[q] = (x != x) ? -INFINITY : x;  // NaN never outranks a number
+    } else {
+      v[q] = -INFINITY;
+      taken |= 1u << q;
+    }
+  }
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
 #pragma unroll
     for (int q = 0; q < EPL; ++q) {
       const int e = lane + 32 * q;
-      if (e < E) {
-        float x = __ldg(logits + static_cast<size_t>(t) * E + e);
-        v[q] = (x != x) ? -INFINITY : x;  // NaN never outranks a number
-      } else {
-        v[q] = -INFINITY;
-        taken |= 1u << q;
+      if (!((taken >> q) & 1u) && better(v[q], e, bv, be)) {
+        bv = v[q];
+        be = e;
       }
     }
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
 #pragma unroll
-      for (int q = 0; q < EPL; ++q) {
-        const int e = lane + 32 * q;
-        if (!((taken >> q) & 1u) && better(v[q], e, bv, be)) {
-          bv = v[q];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (better(ov, oe, bv, be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if (be >= E) {  // cannot happen for k <= E; keep indices in range
-        set_status(5);
-        be = 0;
-      }
-      if (lane == (be & 31)) taken |= 1u << (be >> 5);
-      if (lane == 0) {
-        s_idx[warp * per_warp + i * k + j] = be;
-        my_val[j] = bv;
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (better(ov, oe, bv, be)) {
+        bv = ov;
+        be = oe;
       }
     }
-    __syncwarp();
-    // renormalised softmax over the k kept logits (my_val[0] is the max)
-    float denom = 0.f;
-    const float vmax = my_val[0];
-    for (int j = 0; j < k; ++j) denom += expf(my_val[j] - vmax);
-    for (int j = lane; j < k; j += 32) {
-      const size_t o = static_cast<size_t>(t) * k + j;
-      idx_out[o] = s_idx[warp * per_warp + i * k + j];
-      w_out[o] = expf(my_val[j] - vmax) / denom;
+    if (be >= E) {  // cannot happen for k <= E; keep indices in range
+      set_status(5);
+      be = 0;
     }
-    __syncwarp();
+    if (lane == (be & 31)) taken |= 1u << (be >> 5);
+    if (lane == 0) {
+      my_val[j] = bv;
+      idx_out[static_cast<size_t>(t) * k + j] = be;
+    }
   }
   __syncwarp();
+  // renormalised softmax over the k kept logits (my_val[0] is the max)
+  float denom = 0.f;
+  const float vmax = my_val[0];
+  for (int j = 0; j < k; ++j) denom += expf(my_val[j] - vmax);
+  for (int j = lane; j < k; j += 32)
+    w_out[static_cast<size_t>(t) * k + j] = expf(my_val[j] - vmax) / denom;
+}
 
-  // stable rank of each of this warp's entries among its same-expert entries
-  const int n_tok_w = max(0, min(tpw, T - (t_block + warp * tpw)));
-  const int n_ent = n_tok_w * k;
+// One CTA per kRankChunk consecutive flat entries f = t*k + j: the stable rank
+// of each entry among the chunk's earlier entries of the same expert, and the
+// chunk's expert histogram.
+__global__ void __launch_bounds__(kRankWarps * 32)
+    route_rank_kernel(const int32_t* __restrict__ idx, int R, int E,
+                      int32_t* __restrict__ blk_hist,
+                      int32_t* __restrict__ local_rank) {
+  extern __shared__ int s_cnt[];  // [kRankWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) s_cnt[i] = 0;
+  __syncthreads();
+  const int f0 = blockIdx.x * kRankChunk + warp * kRankPerWarp;
   int* cnt = s_cnt + warp * E;
-  for (int base = 0; base < per_warp; base += 32) {
-    const int f = base + lane;
-    const bool valid = f < n_ent;
-    const int e = valid ? s_idx[warp * per_warp + f] : -1 - lane;
+  int rank[kRankPerWarp / 32];
+  int ex[kRankPerWarp / 32];
+#pragma unroll
+  for (int p = 0; p < kRankPerWarp / 32; ++p) {
+    const int f = f0 + p * 32 + lane;
+    const bool valid = f < R;
+    int e = valid ? idx[f] : -1 - lane;
+    if (valid && (e < 0 || e >= E)) {  // defensive: keep shared indices in range
+      set_status(5);
+      e = 0;
+    }
     const uint32_t m = __match_any_sync(0xffffffffu, e);
-    int rank = 0;
-    if (valid) rank = __popc(m & ((1u << lane) - 1u)) + cnt[e];
+    rank[p] = valid ? __popc(m & ((1u << lane) - 1u)) + cnt[e] : 0;
+    ex[p] = e;
     __syncwarp();
     if (valid && lane == __ffs(m) - 1) cnt[e] += __popc(m);
     __syncwarp();
-    if (valid) s_rank[warp * per_warp + f] = rank;
   }
   __syncthreads();
-
-  // exclusive scan over warps per expert -> block histogram
+  // exclusive scan over warps per expert -> chunk histogram
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
-    for (int w = 0; w < kRouteWarps; ++w) {
+    for (int w = 0; w < kRankWarps; ++w) {
       const int c = s_cnt[w * E + e];
       s_cnt[w * E + e] = run;
       run += c;
@@ -139,12 +128,10 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     blk_hist[static_cast<size_t>(blockIdx.x) * E + e] = run;
   }
   __syncthreads();
-
-  const int n_tok_b = max(0, min(tpb, T - t_block));
-  for (int f = threadIdx.x; f < n_tok_b * k; f += blockDim.x) {
-    const int w = f / per_warp;
-    local_rank[static_cast<size_t>(t_block) * k + f] =
-        s_rank[f] + s_cnt[w * E + s_idx[f]];
+#pragma unroll
+  for (int p = 0; p < kRankPerWarp / 32; ++p) {
+    const int f = f0 + p * 32 + lane;
+    if (f < R) local_rank[f] = rank[p] + cnt[ex[p]];
   }
 }
 
@@ -212,15 +199,14 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-// dest[t, j] = block base of (block of t, expert) + in-block stable rank.
+// dest[f] = base row of (chunk of f, expert) + in-chunk stable rank.
 __global__ void route_dest_kernel(const int32_t* __restrict__ idx,
                                   const int32_t* __restrict__ blk_base,
                                   const int32_t* __restrict__ local_rank,
-                                  int R, int E, int k, int tpb,
-                                  int32_t* __restrict__ dest) {
+                                  int R, int E, int32_t* __restrict__ dest) {
   for (int f = blockIdx.x * blockDim.x + threadIdx.x; f < R;
        f += gridDim.x * blockDim.x) {
-    const int b = (f / k) / tpb;
+    const int b = f / kRankChunk;
     const int e = idx[f];
     int d = blk_base[static_cast<size_t>(b) * E + e] + local_rank[f];
     if (d < 0 || d >= R) {

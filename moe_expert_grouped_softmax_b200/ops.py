@@ -24,7 +24,8 @@ EXPORTS = [
     "moe_route_workspace_bytes", "moe_route_topk", "moe_permute", "moe_unpermute",
     "moe_saved_bytes", "moe_saved_part_offset", "moe_workspace_bytes",
     "moe_lora_mlp_fwd", "moe_lora_mlp_bwd", "moe_get_device_status",
-    "moe_status_string", "moe_set_wait_limit_ns", "moe_profile_enable",
+    "moe_status_string", "moe_set_wait_limit_ns", "moe_test_inject_stall",
+    "moe_profile_enable",
     "moe_profile_collect",
 ]
 
@@ -76,6 +77,8 @@ def lib():
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_set_wait_limit_ns.argtypes = [U64]
         L.moe_set_wait_limit_ns.restype = None
+        L.moe_test_inject_stall.argtypes = [I]
+        L.moe_test_inject_stall.restype = None
         L.moe_profile_enable.argtypes = [I]
         L.moe_profile_enable.restype = I
         L.moe_profile_collect.argtypes = [I, ctypes.POINTER(ctypes.c_float), I]
@@ -115,6 +118,10 @@ def device_status():
 
 def set_wait_limit_ns(ns):
     lib().moe_set_wait_limit_ns(int(ns))
+
+
+def test_inject_stall(on=True):
+    lib().moe_test_inject_stall(1 if on else 0)
 
 
 def profile_enable(on=True):
@@ -288,8 +295,8 @@ class MoeBlock:
     gate_up + SwiGLU, down, weighted unpermute, weighted dY gather, down /
     gate_up backward, LoRA gradients and the dX combine."""
 
-    KERNELS_PER_STEP = 17  # 3 route + 1 permute + 2 fwd + 1 combine +
-    #                        1 gather + 4 transposes + 2 bwd GEMMs + 1 grads
+    KERNELS_PER_STEP = 18  # 4 route + 1 permute + 2 fwd + 1 combine +
+    #                        1 gather + 4 factor copies + 2 bwd GEMMs + 1 grads
     #                        + 1 dX combine
 
     def __init__(self, T, H, I, E, k, r, s, device="cuda", with_dw=False):
