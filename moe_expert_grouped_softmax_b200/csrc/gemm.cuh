@@ -15,8 +15,9 @@
 // faster with Unsloth" (section "Faster LoRA MoE training"): x W^T +
 // s (x A^T) B^T, so W + s B A is never formed.
 //
-// Roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM
-// owner), warps 2..5 = epilogue (TMEM lane quarter = warp % 4).  TMEM holds
+// Roles: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner), then
+// 4 or 8 epilogue warps: TMEM lane quarter = warp % 4; with 8, the two warps
+// of a quarter split the tile's columns.  TMEM holds
 // two accumulators of 256 columns, so the epilogue of one tile overlaps the
 // mainloop of the next.  Tiles are enumerated on the device from
 // expert_offsets (no host synchronisation): m-tiles of all experts in expert
@@ -56,6 +57,37 @@ struct GemmArgs {
 };
 
 constexpr int kSmemOptin = 232448;  // max dynamic shared memory per block
+// Epilogue warps per mode: the SwiGLU-backward epilogue (loads of the saved
+// gate / up and two stores per element) gets two warps per TMEM lane quarter.
+__host__ __device__ constexpr int gemm_epi_warps(int mode) {
+  return mode == 2 ? 8 : 4;
+}
+__host__ __device__ constexpr int gemm_threads(int mode) {
+  return 64 + 32 * gemm_epi_warps(mode);
+}
+
+// Split of a tile's NC epilogue columns between the two warps of a TMEM lane
+// quarter, in multiples of 8 columns.
+template <int NC>
+struct ColSplit {
+  static constexpr int C0 = ((NC / 8 + 1) / 2) * 8;
+  static constexpr int C1 = NC - C0;
+  static_assert(C1 > 0 && C1 % 8 == 0, "column split");
+};
+
+// for_chunks over this warp's share [0, C0) or [C0, NC) of the columns
+// (all of them when the quarter has a single warp).
+template <int NC, bool SPLIT, typename F>
+__device__ __forceinline__ void for_my_chunks(int half, F&& f) {
+  using S = ColSplit<NC>;
+  if constexpr (!SPLIT) {
+    for_chunks<NC>(f);
+  } else if (half == 0) {
+    for_chunks<S::C0>(f);
+  } else {
+    for_chunks<S::C1>([&](int c, auto w) { f(S::C0 + c, w); });
+  }
+}
 
 template <int MODE, int BN, int RK>
 struct GemmCfg {
@@ -169,7 +201,7 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 }
 
 template <int MODE, int BN, int RK>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(gemm_threads(MODE), 1)
     grouped_lora_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmLA,
@@ -215,7 +247,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&lora_full[i], 1);
       mbar_init(&xa_ready[i], 4);
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], gemm_epi_warps(MODE));
     }
     mbar_init(drain_bar, 1);
     *s_abort = 0;
@@ -400,7 +432,9 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp & 3;
+    const int ew = warp & 3;              // TMEM lane quarter
+    constexpr bool kSplit = gemm_epi_warps(MODE) == 8;
+    const int ehalf = (warp - 2) >> 2;    // which share of the columns
     const int row_in_tile = ew * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(ew * 32) << 16;
     int local = 0;
@@ -414,7 +448,9 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
       const uint32_t t_lora = t_acc + BN;
 
-      // rank-r product: TMEM -> bf16 A operand of the up-projection
+      // rank-r product: TMEM -> bf16 A operand of the up-projection (done by
+      // the first four epilogue warps)
+      if (ehalf == 0) {
       if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
       tc_fence_after();
       {
@@ -440,15 +476,20 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&xa_ready[b]);
+      }
       if constexpr (MODE == kDownBwd) {
-        // pull this row's saved gate / up segments into L2 while the
-        // up-projection and the next tile's mainloop run
+        // pull this row's saved gate / up segments (this warp's share of the
+        // columns) into L2 while the up-projection and the next tile's
+        // mainloop run
         if (rvalid) {
-          const int col0 = nt * BN;
-          const int ncol = min(BN, args.N - col0);
-          const __nv_bfloat16* gp = args.aux + static_cast<size_t>(grow) * args.ld_aux + col0;
-          prefetch_l2_bulk(gp, static_cast<uint32_t>(ncol) * 2u);
-          prefetch_l2_bulk(gp + args.I, static_cast<uint32_t>(ncol) * 2u);
+          using S = ColSplit<BN>;
+          const int c0 = nt * BN + (ehalf ? S::C0 : 0);
+          const int ncol = min(ehalf ? S::C1 : S::C0, args.N - c0);
+          if (ncol > 0) {
+            const __nv_bfloat16* gp = args.aux + static_cast<size_t>(grow) * args.ld_aux + c0;
+            prefetch_l2_bulk(gp, static_cast<uint32_t>(ncol) * 2u);
+            prefetch_l2_bulk(gp + args.I, static_cast<uint32_t>(ncol) * 2u);
+          }
         }
       }
 
@@ -459,7 +500,7 @@ __global__ void __launch_bounds__(192, 1)
         const int col0 = nt * HALF;
         __nv_bfloat16* hrow = args.out + static_cast<size_t>(grow) * args.ld_out;
         __nv_bfloat16* zrow = args.out2 + static_cast<size_t>(grow) * args.ld_out2;
-        for_chunks<HALF>([&](int c, auto w) {
+        for_my_chunks<HALF, kSplit>(ehalf, [&](int c, auto w) {
           constexpr int W = decltype(w)::value;
           float g[W], u[W];
           tmem_ld<W>(t_acc + c, g);
@@ -487,7 +528,7 @@ __global__ void __launch_bounds__(192, 1)
         const int col0 = nt * BN;
         const __nv_bfloat16* grow_p = args.aux + static_cast<size_t>(grow) * args.ld_aux;
         __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
-        for_chunks<BN>([&](int c, auto w) {
+        for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
           constexpr int W = decltype(w)::value;
           uint4 gv[W / 8], uv[W / 8];
 #pragma unroll
@@ -530,7 +571,7 @@ __global__ void __launch_bounds__(192, 1)
       } else {
         const int col0 = nt * BN;
         __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
-        for_chunks<BN>([&](int c, auto w) {
+        for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
           constexpr int W = decltype(w)::value;
           float v[W];
           tmem_ld<W>(t_acc + c, v);

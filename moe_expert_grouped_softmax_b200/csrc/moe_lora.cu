@@ -186,7 +186,7 @@ moe_status_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b,
   ProfScope prof(MODE == kGateUpFwd ? MOE_PROF_GATE_UP_FWD
                  : MODE == kDownFwd ? MOE_PROF_DOWN_FWD
                  : MODE == kDownBwd ? MOE_PROF_DOWN_BWD : MOE_PROF_GATE_UP_BWD, st);
-  kern<<<grid, 192, C::SMEM_BYTES, st>>>(a, b, la, lb, args);
+  kern<<<grid, gemm_threads(MODE), C::SMEM_BYTES, st>>>(a, b, la, lb, args);
   return launch_status();
 }
 
