@@ -198,6 +198,12 @@ MOE_API void moe_set_wait_limit_ns(uint64_t ns);
  * exercises the timeout path without faulting or hanging the GPU. */
 MOE_API void moe_test_inject_stall(int on);
 
+/* Kernel choice for the forward grouped GEMMs (not thread-safe; takes effect
+ * at the next moe_lora_mlp_fwd call): 1 runs them on CTA pairs (256-row
+ * tiles on the 2-SM tensor-core instruction), 0 (default) on single CTAs
+ * (128-row tiles).  Both compute the same result. */
+MOE_API void moe_set_forward_pairs(int on);
+
 /* Benchmark hook (not thread-safe; for measurement only).
  * moe_profile_enable(1) starts recording, for every kernel kind below, a pair
  * of CUDA events around each of its launches on the launching stream (up to

@@ -158,11 +158,14 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity,
 }
 
 // Builds the m-tile table in shared memory (one warp): s_off = offsets,
-// s_mstart[e] = first global m-tile of expert e, s_mstart[E] = total.
+// s_mstart[e] = first global m-tile (of 2^bm_shift rows) of expert e,
+// s_mstart[E] = total.
 // Offsets that are not a valid partition of [0, R) give zero tiles.
 __device__ __forceinline__ void build_tile_table(const int32_t* offsets, int E,
                                                  int R, int* s_off,
-                                                 int* s_mstart, int lane) {
+                                                 int* s_mstart, int lane,
+                                                 int bm_shift = 7) {
+  const int bm_round = (1 << bm_shift) - 1;
   const int per = (E + 31) / 32;
   const int lo = min(E, lane * per), hi = min(E, lo + per);
   bool bad = false;
@@ -170,7 +173,7 @@ __device__ __forceinline__ void build_tile_table(const int32_t* offsets, int E,
   for (int e = lo; e < hi; ++e) {
     const int a = offsets[e], b = offsets[e + 1];
     if (b < a) bad = true;
-    local += (b - a + 127) >> 7;
+    local += (b - a + bm_round) >> bm_shift;
   }
   if (lane == 0 && offsets[0] != 0) bad = true;
   if (lane == 0 && offsets[E] != R) bad = true;
@@ -185,7 +188,7 @@ __device__ __forceinline__ void build_tile_table(const int32_t* offsets, int E,
     const int a = offsets[e], b = offsets[e + 1];
     s_off[e] = a;
     s_mstart[e] = run;
-    run += (b - a + 127) >> 7;
+    run += (b - a + bm_round) >> bm_shift;
   }
   const bool any_bad = __any_sync(0xffffffffu, bad);
   if (lane == 31) {
@@ -198,6 +201,147 @@ __device__ __forceinline__ void build_tile_table(const int32_t* offsets, int E,
 __device__ __forceinline__ uint4 pack8(const float* v) {
   return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                     pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+// Epilogue step 1: the rank-r product (TMEM columns [BN, BN + r) of this
+// thread's row) times s, rounded to bf16, into the swizzled K-major shared
+// tile that feeds the up-projection; the first n-tile also saves it
+// (transposed) for the backward.
+template <int RK>
+__device__ __forceinline__ void epi_rank_handoff(const GemmArgs& args, uint32_t t_lora,
+                                                 uint8_t* xt, int row_in_tile, int nt,
+                                                 bool rvalid, int grow) {
+  constexpr uint32_t LSPAN = RK * 2;
+  float xa[RK];
+#pragma unroll
+  for (int c = 0; c < RK; c += 16) tmem_ld16(t_lora + c, xa + c);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < RK; ++i) xa[i] *= args.s;
+#pragma unroll
+  for (int ch = 0; ch < RK / 8; ++ch)
+    *reinterpret_cast<uint4*>(xt + swz_offset(row_in_tile, ch, LSPAN)) = pack8(xa + 8 * ch);
+  if (nt == 0 && rvalid && args.lora_t != nullptr) {
+#pragma unroll
+    for (int q = 0; q < RK; ++q)
+      args.lora_t[static_cast<size_t>(q) * args.ld_lora + grow] = __float2bfloat16_rn(xa[q]);
+  }
+}
+
+// SwiGLU backward: pull this row's saved gate / up segments (this warp's
+// share of the columns) into L2 while the up-projection and the next tile's
+// mainloop run.
+template <int BN>
+__device__ __forceinline__ void epi_prefetch_saved(const GemmArgs& args, int grow,
+                                                   bool rvalid, int nt, int ehalf) {
+  if (!rvalid) return;
+  using S = ColSplit<BN>;
+  const int c0 = nt * BN + (ehalf ? S::C0 : 0);
+  const int ncol = min(ehalf ? S::C1 : S::C0, args.N - c0);
+  if (ncol > 0) {
+    const __nv_bfloat16* gp = args.aux + static_cast<size_t>(grow) * args.ld_aux + c0;
+    prefetch_l2_bulk(gp, static_cast<uint32_t>(ncol) * 2u);
+    prefetch_l2_bulk(gp + args.I, static_cast<uint32_t>(ncol) * 2u);
+  }
+}
+
+// Epilogue step 2: drain the accumulator of this thread's row with the
+// mode's math (SwiGLU; plain store; SwiGLU backward).
+template <int MODE, int BN, bool kSplit>
+__device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, int grow,
+                                          bool rvalid, int nt, int ehalf) {
+  constexpr bool kSwiGLU = (MODE == kGateUpFwd);
+  constexpr int HALF = BN / 2;
+  if constexpr (kSwiGLU) {
+    // gate columns [0, HALF), up columns [HALF, BN) of the tile
+    const int col0 = nt * HALF;
+    __nv_bfloat16* hrow = args.out + static_cast<size_t>(grow) * args.ld_out;
+    __nv_bfloat16* zrow = args.out2 + static_cast<size_t>(grow) * args.ld_out2;
+    for_my_chunks<HALF, kSplit>(ehalf, [&](int c, auto w) {
+      constexpr int W = decltype(w)::value;
+      float g[W], u[W];
+      tmem_ld<W>(t_acc + c, g);
+      tmem_ld<W>(t_acc + HALF + c, u);
+      tmem_ld_wait();
+      if (rvalid) {
+#pragma unroll
+        for (int q = 0; q < W / 8; ++q) {
+          const int col = col0 + c + 8 * q;
+          if (col < args.N) {
+            float h[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float gg = g[8 * q + i];
+              h[i] = gg * sigmoidf_(gg) * u[8 * q + i];
+            }
+            *reinterpret_cast<uint4*>(hrow + col) = pack8(h);
+            *reinterpret_cast<uint4*>(zrow + col) = pack8(g + 8 * q);
+            *reinterpret_cast<uint4*>(zrow + args.I + col) = pack8(u + 8 * q);
+          }
+        }
+      }
+    });
+  } else if constexpr (MODE == kDownBwd) {
+    const int col0 = nt * BN;
+    const __nv_bfloat16* grow_p = args.aux + static_cast<size_t>(grow) * args.ld_aux;
+    __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
+    for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
+      constexpr int W = decltype(w)::value;
+      uint4 gv[W / 8], uv[W / 8];
+#pragma unroll
+      for (int q = 0; q < W / 8; ++q) {  // loads first: in flight during the TMEM read
+        const int col = col0 + c + 8 * q;
+        if (rvalid && col < args.N) {
+          gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
+          uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
+        }
+      }
+      float dh[W];
+      tmem_ld<W>(t_acc + c, dh);
+      tmem_ld_wait();
+      if (rvalid) {
+#pragma unroll
+        for (int q = 0; q < W / 8; ++q) {
+          const int col = col0 + c + 8 * q;
+          if (col < args.N) {
+            const uint32_t ga[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+            const uint32_t ua[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
+            float dg[8], du[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const float gg = h2 ? bf16_hi(ga[i]) : bf16_lo(ga[i]);
+                const float uu = h2 ? bf16_hi(ua[i]) : bf16_lo(ua[i]);
+                const float d = dh[8 * q + 2 * i + h2];
+                const float sg = sigmoidf_(gg);
+                dg[2 * i + h2] = d * uu * sg * (1.f + gg * (1.f - sg));
+                du[2 * i + h2] = d * gg * sg;
+              }
+            }
+            *reinterpret_cast<uint4*>(orow + col) = pack8(dg);
+            *reinterpret_cast<uint4*>(orow + args.I + col) = pack8(du);
+          }
+        }
+      }
+    });
+  } else {
+    const int col0 = nt * BN;
+    __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
+    for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
+      constexpr int W = decltype(w)::value;
+      float v[W];
+      tmem_ld<W>(t_acc + c, v);
+      tmem_ld_wait();
+      if (rvalid) {
+#pragma unroll
+        for (int q = 0; q < W / 8; ++q) {
+          const int col = col0 + c + 8 * q;
+          if (col < args.N) *reinterpret_cast<uint4*>(orow + col) = pack8(v + 8 * q);
+        }
+      }
+    });
+  }
 }
 
 template <int MODE, int BN, int RK>
@@ -451,140 +595,20 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
       // rank-r product: TMEM -> bf16 A operand of the up-projection (done by
       // the first four epilogue warps)
       if (ehalf == 0) {
-      if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
-      tc_fence_after();
-      {
-        float xa[RK];
-#pragma unroll
-        for (int c = 0; c < RK; c += 16) tmem_ld16(t_lora + c, xa + c);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < RK; ++i) xa[i] *= args.s;
-        uint8_t* xt = sXA + b * C::XA_BYTES;
-#pragma unroll
-        for (int ch = 0; ch < RK / 8; ++ch)
-          *reinterpret_cast<uint4*>(xt + swz_offset(row_in_tile, ch, C::LSPAN)) =
-              pack8(xa + 8 * ch);
-        if (nt == 0 && rvalid && args.lora_t != nullptr) {
-#pragma unroll
-          for (int q = 0; q < RK; ++q)
-            args.lora_t[static_cast<size_t>(q) * args.ld_lora + grow] =
-                __float2bfloat16_rn(xa[q]);
-        }
+        if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
+        tc_fence_after();
+        epi_rank_handoff<RK>(args, t_lora, sXA + b * C::XA_BYTES, row_in_tile, nt, rvalid,
+                             grow);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xa_ready[b]);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&xa_ready[b]);
-      }
-      if constexpr (MODE == kDownBwd) {
-        // pull this row's saved gate / up segments (this warp's share of the
-        // columns) into L2 while the up-projection and the next tile's
-        // mainloop run
-        if (rvalid) {
-          using S = ColSplit<BN>;
-          const int c0 = nt * BN + (ehalf ? S::C0 : 0);
-          const int ncol = min(ehalf ? S::C1 : S::C0, args.N - c0);
-          if (ncol > 0) {
-            const __nv_bfloat16* gp = args.aux + static_cast<size_t>(grow) * args.ld_aux + c0;
-            prefetch_l2_bulk(gp, static_cast<uint32_t>(ncol) * 2u);
-            prefetch_l2_bulk(gp + args.I, static_cast<uint32_t>(ncol) * 2u);
-          }
-        }
-      }
+      if constexpr (MODE == kDownBwd) epi_prefetch_saved<BN>(args, grow, rvalid, nt, ehalf);
 
       if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
       tc_fence_after();
-      if constexpr (kSwiGLU) {
-        // gate columns [0, HALF), up columns [HALF, BN) of the tile
-        const int col0 = nt * HALF;
-        __nv_bfloat16* hrow = args.out + static_cast<size_t>(grow) * args.ld_out;
-        __nv_bfloat16* zrow = args.out2 + static_cast<size_t>(grow) * args.ld_out2;
-        for_my_chunks<HALF, kSplit>(ehalf, [&](int c, auto w) {
-          constexpr int W = decltype(w)::value;
-          float g[W], u[W];
-          tmem_ld<W>(t_acc + c, g);
-          tmem_ld<W>(t_acc + HALF + c, u);
-          tmem_ld_wait();
-          if (rvalid) {
-#pragma unroll
-            for (int q = 0; q < W / 8; ++q) {
-              const int col = col0 + c + 8 * q;
-              if (col < args.N) {
-                float h[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float gg = g[8 * q + i];
-                  h[i] = gg * sigmoidf_(gg) * u[8 * q + i];
-                }
-                *reinterpret_cast<uint4*>(hrow + col) = pack8(h);
-                *reinterpret_cast<uint4*>(zrow + col) = pack8(g + 8 * q);
-                *reinterpret_cast<uint4*>(zrow + args.I + col) = pack8(u + 8 * q);
-              }
-            }
-          }
-        });
-      } else if constexpr (MODE == kDownBwd) {
-        const int col0 = nt * BN;
-        const __nv_bfloat16* grow_p = args.aux + static_cast<size_t>(grow) * args.ld_aux;
-        __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
-        for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
-          constexpr int W = decltype(w)::value;
-          uint4 gv[W / 8], uv[W / 8];
-#pragma unroll
-          for (int q = 0; q < W / 8; ++q) {  // loads first: in flight during the TMEM read
-            const int col = col0 + c + 8 * q;
-            if (rvalid && col < args.N) {
-              gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
-              uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
-            }
-          }
-          float dh[W];
-          tmem_ld<W>(t_acc + c, dh);
-          tmem_ld_wait();
-          if (rvalid) {
-#pragma unroll
-            for (int q = 0; q < W / 8; ++q) {
-              const int col = col0 + c + 8 * q;
-              if (col < args.N) {
-                const uint32_t ga[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
-                const uint32_t ua[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
-                float dg[8], du[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-#pragma unroll
-                  for (int h2 = 0; h2 < 2; ++h2) {
-                    const float gg = h2 ? bf16_hi(ga[i]) : bf16_lo(ga[i]);
-                    const float uu = h2 ? bf16_hi(ua[i]) : bf16_lo(ua[i]);
-                    const float d = dh[8 * q + 2 * i + h2];
-                    const float sg = sigmoidf_(gg);
-                    dg[2 * i + h2] = d * uu * sg * (1.f + gg * (1.f - sg));
-                    du[2 * i + h2] = d * gg * sg;
-                  }
-                }
-                *reinterpret_cast<uint4*>(orow + col) = pack8(dg);
-                *reinterpret_cast<uint4*>(orow + args.I + col) = pack8(du);
-              }
-            }
-          }
-        });
-      } else {
-        const int col0 = nt * BN;
-        __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
-        for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
-          constexpr int W = decltype(w)::value;
-          float v[W];
-          tmem_ld<W>(t_acc + c, v);
-          tmem_ld_wait();
-          if (rvalid) {
-#pragma unroll
-            for (int q = 0; q < W / 8; ++q) {
-              const int col = col0 + c + 8 * q;
-              if (col < args.N) *reinterpret_cast<uint4*>(orow + col) = pack8(v + 8 * q);
-            }
-          }
-        });
-      }
+      epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);

@@ -1,0 +1,394 @@
+// a3 / a4 on CTA pairs: the forward grouped GEMMs with 256-row tiles on the
+// 2-SM tensor-core instruction (tcgen05.mma.cta_group::2).
+//
+// A cluster of two CTAs on two SMs computes one 256 x BN tile of one expert.
+// Each CTA stages its own 128 rows of A and half of the B operand
+// [W rows (BN) ; LoRA-down factor rows (r)] (N = BN + r, split into two
+// halves of N/2 rows), so every SM moves a third less operand data per FLOP
+// than the single-CTA 128-row tile.  The even CTA ("leader") issues the
+// MMAs, which read both CTAs' shared memory and write both CTAs' TMEM (each
+// holds its 128 rows x N columns).  The split-LoRA schedule is the one of the
+// single-CTA kernel: rank-r down-projection inside the mainloop MMA,
+// hand-off through shared memory, up-projection (M = 256, K = r) into the
+// same accumulator during the next tile's mainloop.
+//
+// Synchronisation (every wait bounded):
+//  * each CTA's TMA loads complete on its own barriers (so each CTA can
+//    always drain its own copies); the odd CTA ("peer") relays "my half of
+//    stage s has landed" to a second barrier of the leader with a remote
+//    mbarrier arrive, so no asynchronous copy ever signals the other CTA;
+//  * the leader's MMA commits are multicast to both CTAs' barriers
+//    (stage free, rank-r product ready, accumulator ready);
+//  * both CTAs' epilogues arrive on the leader's barriers (hand-off written,
+//    accumulator drained);
+//  * at exit, each CTA waits for the leader's last MMAs (which touch its
+//    shared memory and TMEM), and the leader waits for the peer's final
+//    arrive, so neither leaves while the other can still reach it.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace moe {
+
+template <int MODE, int BN, int RK>
+struct PairCfg {
+  static_assert(MODE == kGateUpFwd || MODE == kDownFwd, "pair kernel: forward only");
+  static constexpr bool kSwiGLU = (MODE == kGateUpFwd);
+  static constexpr int BM = 128, BK = 64;           // rows per CTA
+  static constexpr int NMMA = BN + RK;              // N of the fused MMA
+  static constexpr int NH = NMMA / 2;               // B rows per CTA
+  static constexpr int HALF = BN / 2;
+  // B segments of each CTA (rows): SwiGLU: CTA0 = gate HALF + up U0,
+  // CTA1 = up U1 + factor RK.  Plain: CTA0 = W0 weight rows, CTA1 = W1
+  // weight rows + factor RK.
+  static constexpr int U0 = NH - HALF;              // = RK / 2
+  static constexpr int U1 = HALF - U0;
+  static constexpr int W0 = NH;
+  static constexpr int W1 = BN - NH;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = NH * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int LB_BYTES = HALF * RK * 2;    // this CTA's half of LB
+  static constexpr int XA_BYTES = BM * RK * 2;
+  static constexpr int MISC_BYTES = 512 + 8 * 520;  // barriers, flags, tables
+  static constexpr int FIXED = 2 * LB_BYTES + 2 * XA_BYTES + MISC_BYTES;
+  static constexpr int NS_FIT = (kSmemOptin - 1024 - FIXED) / STAGE_BYTES;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+  static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + FIXED;
+  static constexpr int LSPAN = RK * 2;
+  static constexpr uint32_t LLAYOUT =
+      RK == 16 ? kLayoutSW32 : (RK == 32 ? kLayoutSW64 : kLayoutSW128);
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int ACC_STRIDE = 256;
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static_assert(NS >= 3, "not enough shared memory for three stages");
+  static_assert(SMEM_BYTES <= kSmemOptin, "shared memory over the opt-in limit");
+  static_assert(NMMA <= ACC_STRIDE && NMMA % 16 == 0, "MMA N = BN + r");
+  static_assert(BN % 16 == 0 && NH % 8 == 0, "8-row operand atoms");
+  static_assert(U0 % 8 == 0 && U1 % 8 == 0 && U1 > 0, "SwiGLU segments");
+  static_assert(W1 % 8 == 0 && W1 > 0, "plain segments");
+};
+
+// Host-visible box heights of the weight segments (rows), for the maps.
+template <int MODE, int BN, int RK>
+struct PairBoxes {
+  using C = PairCfg<MODE, BN, RK>;
+  static constexpr int seg0 = C::kSwiGLU ? C::HALF : C::W0;  // CTA0, first
+  static constexpr int seg1 = C::kSwiGLU ? C::U0 : 0;        // CTA0, second
+  static constexpr int seg2 = C::kSwiGLU ? C::U1 : C::W1;    // CTA1, first
+};
+
+template <int MODE, int BN, int RK>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK>::THREADS, 1)
+    grouped_lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                                  const __grid_constant__ CUtensorMap tmW0,
+                                  const __grid_constant__ CUtensorMap tmW1,
+                                  const __grid_constant__ CUtensorMap tmW2,
+                                  const __grid_constant__ CUtensorMap tmLA,
+                                  const __grid_constant__ CUtensorMap tmLB,
+                                  const GemmArgs args) {
+  using C = PairCfg<MODE, BN, RK>;
+  constexpr bool kSwiGLU = C::kSwiGLU;
+  constexpr int HALF = C::HALF;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sStage = smem;
+  uint8_t* sLB = sStage + C::NS * C::STAGE_BYTES;
+  uint8_t* sXA = sLB + 2 * C::LB_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sXA + 2 * C::XA_BYTES);
+  uint64_t* empty = full + C::NS;
+  uint64_t* lb_full = empty + C::NS;
+  uint64_t* lb_empty = lb_full + 2;
+  uint64_t* lora_full = lb_empty + 2;
+  uint64_t* xa_ready = lora_full + 2;
+  uint64_t* acc_full = xa_ready + 2;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* peer_full = acc_empty + 2;       // leader: peer's half landed
+  uint64_t* peer_lb = peer_full + C::NS;      // leader: peer's LB half landed
+  uint64_t* final_bar = peer_lb + 2;
+  uint64_t* peer_done = final_bar + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(peer_done + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_off = reinterpret_cast<int*>(s_tmem + 4);
+  int* s_mstart = s_off + 520;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int E = args.E;
+  const uint64_t wait_ns = args.wait_ns;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&peer_full[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&lb_full[i], 1);
+      mbar_init(&peer_lb[i], 1);
+      mbar_init(&lb_empty[i], 1);
+      mbar_init(&lora_full[i], 1);
+      mbar_init(&xa_ready[i], 2 * C::EPI_WARPS);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 2 * C::EPI_WARPS);
+    }
+    mbar_init(final_bar, 1);
+    mbar_init(peer_done, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmW0);
+    prefetch_tmap(&tmW1);
+    prefetch_tmap(&tmW2);
+    prefetch_tmap(&tmLA);
+    prefetch_tmap(&tmLB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(s_tmem, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 2) build_tile_table(args.offsets, E, args.R, s_off, s_mstart, lane, 8);
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated
+  tc_fence_after();
+
+  const uint32_t tmem_base = *s_tmem;
+  const int total_tiles = s_mstart[E] * args.n_tiles;
+  const int k_iters = (args.K + C::BK - 1) / C::BK;
+  // cluster addresses of the leader's copies of the barriers
+  auto lead = [&](uint64_t* bar) { return mapa_shared(smem_u32(bar), 0); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed_stages = 0;
+      uint32_t lb_armed = 0;
+      uint32_t lb_par[2] = {0, 0};
+      bool ok = true;
+      int local = 0;
+      for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++local) {
+        int e, mt, nt;
+        decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+        const int row0 = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * C::BM;
+        const int b = local & 1;
+        const uint32_t use = (local >> 1) & 1;
+        if (!mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
+        mbar_arrive_expect_tx(&lb_full[b], C::LB_BYTES);
+        lb_armed |= 1u << b;
+        lb_par[b] = use;
+        // this CTA's half of the up-projection factor: output columns
+        // [rank * BN/2, (rank + 1) * BN/2) of the tile
+        const int lb_row = kSwiGLU ? e * args.lb_rows + (rank ? args.I : 0) + nt * HALF
+                                   : e * args.lb_rows + nt * BN + static_cast<int>(rank) * HALF;
+        tma_load_2d(sLB + b * C::LB_BYTES, &tmLB, &lb_full[b], 0, lb_row);
+        for (int kt = 0; kt < k_iters; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, wait_ns)) { ok = false; break; }
+          uint8_t* st = sStage + stage * C::STAGE_BYTES;
+          uint8_t* sb = st + C::A_BYTES;
+          const int kx = kt * C::BK;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(st, &tmA, &full[stage], kx, row0);
+          if (kSwiGLU) {
+            const int gate = e * args.b_rows + nt * HALF;
+            const int up = e * args.b_rows + args.I + nt * HALF;
+            if (rank == 0) {
+              tma_load_2d(sb, &tmW0, &full[stage], kx, gate);
+              tma_load_2d(sb + HALF * 128, &tmW1, &full[stage], kx, up);
+            } else {
+              tma_load_2d(sb, &tmW2, &full[stage], kx, up + C::U0);
+              tma_load_2d(sb + C::U1 * 128, &tmLA, &full[stage], kx, e * RK);
+            }
+          } else {
+            const int w = e * args.b_rows + nt * BN;
+            if (rank == 0) {
+              tma_load_2d(sb, &tmW0, &full[stage], kx, w);
+            } else {
+              tma_load_2d(sb, &tmW2, &full[stage], kx, w + C::W0);
+              tma_load_2d(sb + C::W1 * 128, &tmLA, &full[stage], kx, e * RK);
+            }
+          }
+          if (armed_stages < C::NS) ++armed_stages;
+          if (++stage == C::NS) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // own loads complete on own barriers: wait for all of them to land
+      for (int i = 0; i < armed_stages; ++i) {
+        int s = stage - 1 - i;
+        uint32_t ph = phase;
+        if (s < 0) {
+          s += C::NS;
+          ph ^= 1;
+        }
+        drain_wait(&full[s], ph, wait_ns);
+      }
+      for (int bb = 0; bb < 2; ++bb)
+        if (lb_armed & (1u << bb)) drain_wait(&lb_full[bb], lb_par[bb], wait_ns);
+    }
+  } else if (warp == 1) {
+    if (!leader) {
+      // ---------------------------------------------------------- relay (peer)
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int local = 0;
+        bool ok = true;
+        for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++local) {
+          const int b = local & 1;
+          const uint32_t use = (local >> 1) & 1;
+          if (!mbar_wait(&lb_full[b], use, s_abort, wait_ns)) { ok = false; break; }
+          mbar_arrive_cluster(lead(&peer_lb[b]));
+          for (int kt = 0; kt < k_iters; ++kt) {
+            if (!mbar_wait(&full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
+            mbar_arrive_cluster(lead(&peer_full[stage]));
+            if (++stage == C::NS) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+      }
+    } else if (lane == 0) {
+      // ---------------------------------------------------------- MMA (leader)
+      constexpr uint32_t kIdesc = idesc_bf16_f32(256, C::NMMA, false, false);
+      constexpr uint32_t kIdescUp = idesc_bf16_f32(256, BN, false, false);
+      constexpr uint16_t kBoth = 0x3;
+      auto issue_up = [&](int b) {
+        const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
+        const uint32_t xa0 = smem_u32(sXA + b * C::XA_BYTES);
+        const uint32_t lb0 = smem_u32(sLB + b * C::LB_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < RK / 16; ++kk)
+          umma_bf16_pair(t_acc, smem_desc(xa0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
+                         smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), kIdescUp, 1u);
+        umma_commit_pair_mc(&lb_empty[b], kBoth);
+        umma_commit_pair_mc(&acc_full[b], kBoth);
+      };
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      int pending = -1;
+      bool ok = true;
+      if (args.stall_test) ok = mbar_wait(final_bar, 0, s_abort, wait_ns);
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs, ++local) {
+        const int b = local & 1;
+        const uint32_t use = (local >> 1) & 1;
+        const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
+        if (!mbar_wait_cluster(&acc_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        for (int kt = 0; kt < k_iters; ++kt) {
+          if (!mbar_wait(&full[stage], phase, s_abort, wait_ns) ||
+              !mbar_wait_cluster(&peer_full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sStage + stage * C::STAGE_BYTES);
+          const uint32_t b0 = a0 + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk)
+            umma_bf16_pair(t_acc, smem_desc(a0 + kk * 32, 16, 1024, kLayoutSW128),
+                           smem_desc(b0 + kk * 32, 16, 1024, kLayoutSW128), kIdesc,
+                           (kt | kk) ? 1u : 0u);
+          umma_commit_pair_mc(&empty[stage], kBoth);
+          if (++stage == C::NS) {
+            stage = 0;
+            phase ^= 1;
+          }
+          if (pending >= 0) {
+            const int pb = pending & 1;
+            const uint32_t pu = (pending >> 1) & 1;
+            if (mbar_test_wait_cluster(&xa_ready[pb], pu) &&
+                mbar_test_wait(&lb_full[pb], pu) && mbar_test_wait_cluster(&peer_lb[pb], pu)) {
+              tc_fence_after();
+              issue_up(pb);
+              pending = -1;
+            }
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(&lora_full[b], kBoth);
+        if (pending >= 0) {
+          const int pb = pending & 1;
+          const uint32_t pu = (pending >> 1) & 1;
+          if (!mbar_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) ||
+              !mbar_wait(&lb_full[pb], pu, s_abort, wait_ns) ||
+              !mbar_wait_cluster(&peer_lb[pb], pu, s_abort, wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          issue_up(pb);
+        }
+        pending = local;
+      }
+      if (ok && pending >= 0) {
+        const int pb = pending & 1;
+        const uint32_t pu = (pending >> 1) & 1;
+        if (mbar_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) &&
+            mbar_wait(&lb_full[pb], pu, s_abort, wait_ns) &&
+            mbar_wait_cluster(&peer_lb[pb], pu, s_abort, wait_ns)) {
+          tc_fence_after();
+          issue_up(pb);
+        }
+      }
+      // all of the leader's MMAs complete -> both CTAs' final_bar
+      umma_commit_pair_mc(final_bar, kBoth);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp & 3;
+    const int row_in_tile = ew * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(ew * 32) << 16;
+    int local = 0;
+    for (int tile = pair; tile < total_tiles; tile += npairs, ++local) {
+      int e, mt, nt;
+      decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+      const int b = local & 1;
+      const uint32_t use = (local >> 1) & 1;
+      const int grow = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * C::BM + row_in_tile;
+      const bool rvalid = grow < s_off[e + 1];
+      const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
+      if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
+      tc_fence_after();
+      epi_rank_handoff<RK>(args, t_acc + BN, sXA + b * C::XA_BYTES, row_in_tile, nt, rvalid,
+                           grow);
+      fence_proxy_async_all();  // the leader's MMA reads this tile
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead(&xa_ready[b]));
+      if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
+      tc_fence_after();
+      epi_drain<MODE, BN, false>(args, t_acc, grow, rvalid, nt, 0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead(&acc_empty[b]));
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // the leader's MMAs read this CTA's shared memory and write its TMEM
+    drain_wait(final_bar, 0, wait_ns);
+    if (!leader) {
+      mbar_arrive_cluster(lead(peer_done));  // no more arrives from this CTA
+    } else {
+      drain_wait(peer_done, 0, wait_ns);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace moe

@@ -15,6 +15,7 @@
 #include "route.cuh"
 #include "permute.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "lora_grad.cuh"
 
 using namespace moe;
@@ -54,6 +55,7 @@ moe_status_t route_scratch_on_current_device(void** out) {
 
 uint64_t g_wait_limit_ns = 1000000000ull;  // one second per bounded wait
 int g_stall_test = 0;                      // testing hook, see moe_test_inject_stall
+int g_forward_pairs = 0;                   // forward GEMMs on CTA pairs
 
 // ------------------------------------------------ optional per-kernel timing
 // When enabled, each launch site of a kernel kind records a CUDA event before
@@ -208,6 +210,47 @@ moe_status_t launch_gemm(int bn, int r, const CUtensorMap& a, const CUtensorMap&
   return MOE_ERR_UNSUPPORTED;
 }
 
+// Forward GEMM on CTA pairs (256-row tiles, BN = 256 - r).  A: [R, K]
+// activations; W: the base weight as [E * b_rows, K]; LA: the down factor as
+// [E * r, K]; LB: the up factor as [E * lb_rows, r].
+template <int MODE, int BN, int RK>
+moe_status_t launch_pair_t(const void* A, const void* W, const void* LA, const void* LB,
+                           const GemmArgs& args, cudaStream_t st) {
+  using C = PairCfg<MODE, BN, RK>;
+  using Bx = PairBoxes<MODE, BN, RK>;
+  const uint64_t K = static_cast<uint64_t>(args.K);
+  const uint64_t EU = static_cast<uint64_t>(args.E);
+  CUtensorMap ta, tw0, tw1, tw2, tla, tlb;
+  bool ok = tmap_2d(&ta, A, K, args.R, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && tmap_2d(&tw0, W, K, EU * args.b_rows, K * 2, 64, Bx::seg0, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && tmap_2d(&tw1, W, K, EU * args.b_rows, K * 2, 64, Bx::seg1 > 0 ? Bx::seg1 : 8,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && tmap_2d(&tw2, W, K, EU * args.b_rows, K * 2, 64, Bx::seg2, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && tmap_2d(&tla, LA, K, EU * RK, K * 2, 64, RK, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && tmap_2d(&tlb, LB, RK, EU * args.lb_rows, RK * 2ull, RK, C::HALF, lora_swizzle(RK));
+  if (!ok) return MOE_ERR_CUDA;
+  auto kern = grouped_lora_gemm_pair_kernel<MODE, BN, RK>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_BYTES) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const long long max_pairs =
+      (static_cast<long long>(args.R) / 256 + args.E) * args.n_tiles;
+  const int pairs = static_cast<int>(std::min<long long>(num_sms() / 2, max_pairs));
+  if (pairs <= 0) return MOE_ERR_CUDA;
+  ProfScope prof(MODE == kGateUpFwd ? MOE_PROF_GATE_UP_FWD : MOE_PROF_DOWN_FWD, st);
+  kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tw0, tw1, tw2, tla, tlb, args);
+  return launch_status();
+}
+
+template <int MODE>
+moe_status_t launch_pair(int r, const void* A, const void* W, const void* LA,
+                         const void* LB, const GemmArgs& args, cudaStream_t st) {
+  if (r == 16) return launch_pair_t<MODE, 240, 16>(A, W, LA, LB, args, st);
+  if (r == 32) return launch_pair_t<MODE, 224, 32>(A, W, LA, LB, args, st);
+  if (r == 64) return launch_pair_t<MODE, 192, 64>(A, W, LA, LB, args, st);
+  return MOE_ERR_UNSUPPORTED;
+}
+
 template <int RK>
 moe_status_t launch_grad_t(const CUtensorMap* u, const CUtensorMap* v,
                            const GradArgs& args, cudaStream_t st) {
@@ -310,6 +353,8 @@ void moe_set_wait_limit_ns(uint64_t ns) {
 }
 
 void moe_test_inject_stall(int on) { g_stall_test = on ? 1 : 0; }
+
+void moe_set_forward_pairs(int on) { g_forward_pairs = on ? 1 : 0; }
 
 moe_status_t moe_profile_enable(int on) {
   if (on && !g_prof_created) {
@@ -440,9 +485,14 @@ moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
   const int warps = 8;
   const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
   ProfScope prof(MOE_PROF_PERMUTE, stream);
-  permute_kernel<<<grid, warps * 32, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
-      static_cast<__nv_bfloat16*>(Xp), static_cast<const __nv_bfloat16*>(Zp), dw);
+  if (dw == nullptr)
+    permute_rows_kernel<<<grid, warps * 32, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
+        static_cast<__nv_bfloat16*>(Xp));
+  else
+    permute_kernel<<<grid, warps * 32, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
+        static_cast<__nv_bfloat16*>(Xp), static_cast<const __nv_bfloat16*>(Zp), dw);
   return launch_status();
 }
 
@@ -513,7 +563,17 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
   const uint64_t EU = static_cast<uint64_t>(E);
 
   // gate_up + SwiGLU
-  {
+  if (g_forward_pairs) {
+    const int bn = 256 - r, half = bn / 2;
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + half - 1) / half; g.I = I;
+    g.b_rows = 2 * I; g.lb_rows = 2 * I; g.s = s;
+    g.out = h; g.ld_out = I; g.out2 = Z1; g.ld_out2 = 2 * I;
+    g.lora_t = xa1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
+    if ((stt = launch_pair<kGateUpFwd>(r, Xp, W1, A1, B1, g, st)) != MOE_OK) return stt;
+  } else {
     const int bn = pick_bn(I, true, r, false), half = bn / 2;
     CUtensorMap ta, tb, tla, tlb;
     bool ok = tmap_2d(&ta, Xp, H, R, H * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -531,7 +591,17 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     if ((stt = launch_gemm<kGateUpFwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   // down
-  {
+  if (g_forward_pairs) {
+    const int bn = 256 - r;
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
+    g.b_rows = H; g.lb_rows = H; g.s = s;
+    g.out = static_cast<__nv_bfloat16*>(Z2); g.ld_out = H;
+    g.lora_t = ha2; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
+    if ((stt = launch_pair<kDownFwd>(r, h, W2, A2, B2, g, st)) != MOE_OK) return stt;
+  } else {
     const int bn = pick_bn(H, false, r, false);
     CUtensorMap ta, tb, tla, tlb;
     bool ok = tmap_2d(&ta, h, I, R, I * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);

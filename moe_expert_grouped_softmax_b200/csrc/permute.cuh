@@ -48,8 +48,58 @@ __device__ __forceinline__ float dot8(uint4 a, uint4 b) {
 
 constexpr int kCopyUnroll = 4;
 
-// Xp[dest[t,j]] = (scale ? scale[t,j] : 1) * X[t]; optional dw[t,j] =
-// <X[t], Zp[dest[t,j]]>.  One warp per token, grid-stride over tokens.
+constexpr int kRowVec = 8;  // 16-byte vectors per lane held at once
+
+// Xp[dest[t,j]] = (scale ? scale[t,j] : 1) * X[t].  One warp per token: the
+// row is read once into registers (kRowVec vectors per lane in flight) and
+// written to all k destinations.
+__global__ void __launch_bounds__(256)
+    permute_rows_kernel(const __nv_bfloat16* __restrict__ X,
+                        const int32_t* __restrict__ dest,
+                        const float* __restrict__ scale, int T, int H, int k,
+                        __nv_bfloat16* __restrict__ Xp) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int nvec = H >> 3;
+  const int R = T * k;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+    const char* xrow = reinterpret_cast<const char*>(X + static_cast<size_t>(t) * H);
+    for (int v0 = lane; v0 < nvec; v0 += 32 * kRowVec) {
+      uint4 x[kRowVec];
+#pragma unroll
+      for (int u = 0; u < kRowVec; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < nvec) x[u] = ld_nc_v4(xrow + 16 * static_cast<size_t>(v));
+      }
+      for (int j = 0; j < k; ++j) {
+        const int d = dest[static_cast<size_t>(t) * k + j];
+        if (d < 0 || d >= R) {
+          if (lane == 0 && v0 == lane) set_status(5);
+          continue;
+        }
+        char* orow = reinterpret_cast<char*>(Xp + static_cast<size_t>(d) * H);
+        const float c = scale ? scale[static_cast<size_t>(t) * k + j] : 1.f;
+#pragma unroll
+        for (int u = 0; u < kRowVec; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nvec) {
+            uint4 y = x[u];
+            if (scale) {
+              y.x = scale2(y.x, c);
+              y.y = scale2(y.y, c);
+              y.z = scale2(y.z, c);
+              y.w = scale2(y.w, c);
+            }
+            st_v4(orow + 16 * static_cast<size_t>(v), y);
+          }
+        }
+      }
+    }
+  }
+}
+
+// Same with the routing-weight gradient dw[t,j] = <X[t], Zp[dest[t,j]]>.
+// One warp per token, grid-stride over tokens.
 __global__ void __launch_bounds__(256)
     permute_kernel(const __nv_bfloat16* __restrict__ X,
                    const int32_t* __restrict__ dest,
@@ -114,7 +164,10 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+constexpr int kCombVec = 4;  // 16-byte vectors per lane per source row
+
 // Y[t] = sum_j (w ? w[t,j] : 1) * Yp[dest[t,j]], fp32 in j order -> bf16.
+// One warp per token; kCombVec x k loads in flight per lane.
 __global__ void __launch_bounds__(256)
     unpermute_kernel(const __nv_bfloat16* __restrict__ Yp,
                      const int32_t* __restrict__ dest,
@@ -126,10 +179,10 @@ __global__ void __launch_bounds__(256)
   const int R = T * k;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     char* yrow = reinterpret_cast<char*>(Y + static_cast<size_t>(t) * H);
-    for (int v0 = lane; v0 < nvec; v0 += 64) {
-      float acc[2][8];
+    for (int v0 = lane; v0 < nvec; v0 += 32 * kCombVec) {
+      float acc[kCombVec][8];
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+      for (int u = 0; u < kCombVec; ++u)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
       for (int j = 0; j < k; ++j) {
@@ -141,7 +194,7 @@ __global__ void __launch_bounds__(256)
         const float c = w ? w[static_cast<size_t>(t) * k + j] : 1.f;
         const char* zrow = reinterpret_cast<const char*>(Yp + static_cast<size_t>(d) * H);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < kCombVec; ++u) {
           const int v = v0 + 32 * u;
           if (v < nvec) {
             const uint4 z = ld_nc_v4(zrow + 16 * static_cast<size_t>(v));
@@ -157,7 +210,7 @@ __global__ void __launch_bounds__(256)
         }
       }
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < kCombVec; ++u) {
         const int v = v0 + 32 * u;
         if (v < nvec) {
           uint4 o;

@@ -25,7 +25,7 @@ EXPORTS = [
     "moe_saved_bytes", "moe_saved_part_offset", "moe_workspace_bytes",
     "moe_lora_mlp_fwd", "moe_lora_mlp_bwd", "moe_get_device_status",
     "moe_status_string", "moe_set_wait_limit_ns", "moe_test_inject_stall",
-    "moe_profile_enable",
+    "moe_set_forward_pairs", "moe_profile_enable",
     "moe_profile_collect",
 ]
 
@@ -77,6 +77,8 @@ def lib():
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_set_wait_limit_ns.argtypes = [U64]
         L.moe_set_wait_limit_ns.restype = None
+        L.moe_set_forward_pairs.argtypes = [I]
+        L.moe_set_forward_pairs.restype = None
         L.moe_test_inject_stall.argtypes = [I]
         L.moe_test_inject_stall.restype = None
         L.moe_profile_enable.argtypes = [I]
@@ -118,6 +120,11 @@ def device_status():
 
 def set_wait_limit_ns(ns):
     lib().moe_set_wait_limit_ns(int(ns))
+
+
+def set_forward_pairs(on=True):
+    """Forward GEMMs on CTA pairs (256-row tiles) or single CTAs."""
+    lib().moe_set_forward_pairs(1 if on else 0)
 
 
 def test_inject_stall(on=True):

@@ -125,20 +125,32 @@ BLOCK_CASES = {
 }
 
 
-@pytest.fixture(scope="module", params=list(BLOCK_CASES))
+# every case on the default single-CTA forward kernels; the cases marked
+# "/pairs" again with the CTA-pair forward kernels
+BLOCK_RUNS = [(c, False) for c in BLOCK_CASES] + [
+    (c, True) for c in ("tiny", "ragged", "rank32", "rank64", "skew_empty")]
+
+
+@pytest.fixture(scope="module", params=BLOCK_RUNS,
+                ids=lambda p: p[0] + ("/pairs" if p[1] else ""))
 def block_run(request, cuda_ok):
-    cfg = BLOCK_CASES[request.param]
+    name, pairs = request.param
+    cfg = BLOCK_CASES[name]
     inp = S.make_inputs(cfg)
     Y, ctx, grads = oracle_block(inp, cfg["k"])
     g = _cuda(inp)
     blk = ops.MoeBlock(cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"], cfg["r"], cfg["s"],
                        with_dw=True)
     W = _weights(g)
-    blk.step(g["X"], g["logits"], g["dY"], W)
-    torch.cuda.synchronize()
+    ops.set_forward_pairs(pairs)
+    try:
+        blk.step(g["X"], g["logits"], g["dY"], W)
+        torch.cuda.synchronize()
+    finally:
+        ops.set_forward_pairs(False)
     status = ops.device_status()
-    return dict(name=request.param, cfg=cfg, inp=inp, Y=Y, ctx=ctx, grads=grads, blk=blk,
-                status=status)
+    return dict(name=name, pairs=pairs, cfg=cfg, inp=inp, Y=Y, ctx=ctx, grads=grads,
+                blk=blk, status=status)
 
 
 def test_block_status(block_run):
@@ -199,6 +211,10 @@ def test_block_deterministic(block_run):
     g = _cuda(block_run["inp"])
     W = _weights(g)
     first = [t.clone() for t in (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2)]
-    b.step(g["X"], g["logits"], g["dY"], W)
+    ops.set_forward_pairs(block_run["pairs"])
+    try:
+        b.step(g["X"], g["logits"], g["dY"], W)
+    finally:
+        ops.set_forward_pairs(False)
     for x, y in zip(first, (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2)):
         assert torch.equal(x, y)
