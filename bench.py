@@ -138,6 +138,8 @@ def run_ours(args, cfg):
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
+    if args.forward_pairs >= 0:
+        ops.set_forward_pairs(bool(args.forward_pairs))
     dev = torch.device("cuda", local)
     if ws > 1:
         dist.init_process_group("nccl", device_id=dev,
@@ -317,6 +319,9 @@ def main():
     ap.add_argument("--cpu-sample-tokens", type=int, default=128)
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (small cases for profiler captures)")
+    ap.add_argument("--forward-pairs", type=int, default=-1,
+                    help="1: forward GEMMs on CTA pairs, 0: single CTAs, "
+                         "-1: library default")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

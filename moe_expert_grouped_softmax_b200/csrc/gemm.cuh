@@ -57,6 +57,14 @@ struct GemmArgs {
 };
 
 constexpr int kSmemOptin = 232448;  // max dynamic shared memory per block
+
+// K-slice of one pipeline stage of the single-CTA kernel: 64 bf16 = 128-byte
+// rows, 128-byte swizzle for the K-major operands.  (Measured: halving it to
+// 32 doubles the TMA requests per FLOP and slows the mainloop.)
+constexpr int kGemmBK = 64;
+constexpr uint32_t kKmajLayout = kGemmBK == 64 ? kLayoutSW128 : kLayoutSW64;
+constexpr int kKmajSBO = 8 * kGemmBK * 2;        // 8 rows of 64 bytes
+constexpr int kMnAtomBytes = kGemmBK * 128;      // 64 columns x BK rows (MN-major)
 // Epilogue warps per mode: the SwiGLU-backward epilogue (loads of the saved
 // gate / up and two stores per element) gets two warps per TMEM lane quarter.
 __host__ __device__ constexpr int gemm_epi_warps(int mode) {
@@ -92,13 +100,15 @@ __device__ __forceinline__ void for_my_chunks(int half, F&& f) {
 template <int MODE, int BN, int RK>
 struct GemmCfg {
   static constexpr bool kBMN = (MODE == kDownBwd || MODE == kGateUpBwd);
-  static constexpr int BM = 128, BK = 64;
+  static constexpr int BM = 128, BK = kGemmBK;
   static constexpr int NMMA = BN + RK;  // N of the fused mainloop MMA
   static constexpr int A_BYTES = BM * BK * 2;
-  // K-major: BN weight rows then r factor rows, 128 B each.  MN-major: BN/64
-  // weight atoms then one 64-column atom holding the (zero-padded) factor.
-  static constexpr int B_BYTES = kBMN ? (BN / 64 + 1) * 8192 : NMMA * 128;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  // K-major: BN weight rows then r factor rows, BK*2 bytes each.  MN-major:
+  // BN/64 weight atoms then one 64-column atom holding the (zero-padded)
+  // factor.
+  static constexpr int B_BYTES = kBMN ? (BN / 64 + 1) * kMnAtomBytes : NMMA * BK * 2;
+  // stages start on 1024-byte boundaries (the widest swizzle period)
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int LB_BYTES = BN * RK * 2;
   static constexpr int XA_BYTES = BM * RK * 2;
   static constexpr int MISC_BYTES = 256 + 8 * 520;  // barriers, flags, tables
@@ -198,6 +208,31 @@ __device__ __forceinline__ void build_tile_table(const int32_t* offsets, int E,
   if (any_bad && lane == 0) set_status(5);
 }
 
+// Optional wait-time instrumentation (compiled in only with MOE_GEMM_TRACE):
+// clock cycles per CTA and role spent in each wait, by GEMM mode.
+#ifdef MOE_GEMM_TRACE
+constexpr int kTraceSlots = 16;
+__device__ unsigned long long g_gemm_trace[4][160][kTraceSlots];
+#define MOE_TIMED(mode, slot, expr)                                           \
+  ([&]() {                                                                    \
+    const long long _t = clock64();                                           \
+    auto _r = (expr);                                                         \
+    atomicAdd(&g_gemm_trace[mode][blockIdx.x % 160][slot],                    \
+              static_cast<unsigned long long>(clock64() - _t));               \
+    return _r;                                                                \
+  }())
+#define MOE_TIMED_VOID(mode, slot, stmt)                                      \
+  do {                                                                        \
+    const long long _t = clock64();                                           \
+    stmt;                                                                     \
+    atomicAdd(&g_gemm_trace[mode][blockIdx.x % 160][slot],                    \
+              static_cast<unsigned long long>(clock64() - _t));               \
+  } while (0)
+#else
+#define MOE_TIMED(mode, slot, expr) (expr)
+#define MOE_TIMED_VOID(mode, slot, stmt) stmt
+#endif
+
 __device__ __forceinline__ uint4 pack8(const float* v) {
   return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                     pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
@@ -252,6 +287,7 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
                                           bool rvalid, int nt, int ehalf) {
   constexpr bool kSwiGLU = (MODE == kGateUpFwd);
   constexpr int HALF = BN / 2;
+  const uint64_t pol = policy_evict_first();  // outputs stream out of L2
   if constexpr (kSwiGLU) {
     // gate columns [0, HALF), up columns [HALF, BN) of the tile
     const int col0 = nt * HALF;
@@ -274,9 +310,9 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
               const float gg = g[8 * q + i];
               h[i] = gg * sigmoidf_(gg) * u[8 * q + i];
             }
-            *reinterpret_cast<uint4*>(hrow + col) = pack8(h);
-            *reinterpret_cast<uint4*>(zrow + col) = pack8(g + 8 * q);
-            *reinterpret_cast<uint4*>(zrow + args.I + col) = pack8(u + 8 * q);
+            st_global_v4_hint(hrow + col, pack8(h), pol);
+            st_global_v4_hint(zrow + col, pack8(g + 8 * q), pol);
+            st_global_v4_hint(zrow + args.I + col, pack8(u + 8 * q), pol);
           }
         }
       }
@@ -319,8 +355,8 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
                 du[2 * i + h2] = d * gg * sg;
               }
             }
-            *reinterpret_cast<uint4*>(orow + col) = pack8(dg);
-            *reinterpret_cast<uint4*>(orow + args.I + col) = pack8(du);
+            st_global_v4_hint(orow + col, pack8(dg), pol);
+            st_global_v4_hint(orow + args.I + col, pack8(du), pol);
           }
         }
       }
@@ -337,7 +373,7 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
 #pragma unroll
         for (int q = 0; q < W / 8; ++q) {
           const int col = col0 + c + 8 * q;
-          if (col < args.N) *reinterpret_cast<uint4*>(orow + col) = pack8(v + 8 * q);
+          if (col < args.N) st_global_v4_hint(orow + col, pack8(v + 8 * q), pol);
         }
       }
     });
@@ -419,6 +455,10 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // weights are reused by every m-tile of an expert: keep them in L2;
+      // activations stream through once per n-tile wave
+      const uint64_t pol_w = policy_evict_last();
+      const uint64_t pol_a = policy_evict_first();
       int stage = 0;
       uint32_t phase = 0;
       int armed_stages = 0;      // stages armed at least once
@@ -433,42 +473,45 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
         const int row0 = s_off[e] + mt * C::BM;
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
-        if (!mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
+        if (!MOE_TIMED(MODE, 5, mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
         mbar_arrive_expect_tx(&lb_full[b], C::LB_BYTES);
         lb_armed |= 1u << b;
         lb_par[b] = use;
         uint8_t* lb = sLB + b * C::LB_BYTES;
         if (kSwiGLU) {
-          tma_load_2d(lb, &tmLB, &lb_full[b], 0, e * args.lb_rows + nt * HALF);
-          tma_load_2d(lb + HALF * C::LSPAN, &tmLB, &lb_full[b], 0,
-                      e * args.lb_rows + args.I + nt * HALF);
+          tma_load_2d_hint(lb, &tmLB, &lb_full[b], 0, e * args.lb_rows + nt * HALF, pol_w);
+          tma_load_2d_hint(lb + HALF * C::LSPAN, &tmLB, &lb_full[b], 0,
+                           e * args.lb_rows + args.I + nt * HALF, pol_w);
         } else {
-          tma_load_2d(lb, &tmLB, &lb_full[b], 0, e * args.lb_rows + nt * BN);
+          tma_load_2d_hint(lb, &tmLB, &lb_full[b], 0, e * args.lb_rows + nt * BN, pol_w);
         }
         for (int kt = 0; kt < k_iters; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, wait_ns)) { ok = false; break; }
+          if (!MOE_TIMED(MODE, 4, mbar_wait(&empty[stage], phase ^ 1, s_abort, wait_ns))) { ok = false; break; }
           uint8_t* st = sStage + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(st, &tmA, &full[stage], kt * C::BK, row0);
+          tma_load_2d_hint(st, &tmA, &full[stage], kt * C::BK, row0, pol_a);
           uint8_t* sb = st + C::A_BYTES;
           if (kBMN) {
 #pragma unroll
             for (int i = 0; i < BN / 64; ++i)
-              tma_load_2d(sb + i * 8192, &tmB, &full[stage], nt * BN + 64 * i,
-                          e * args.b_rows + kt * C::BK);
+              tma_load_2d_hint(sb + i * kMnAtomBytes, &tmB, &full[stage], nt * BN + 64 * i,
+                               e * args.b_rows + kt * C::BK, pol_w);
             // factor atom: [K rows, 64 columns] zero-padded past r
-            tma_load_2d(sb + (BN / 64) * 8192, &tmLA, &full[stage], 0,
-                        e * args.b_rows + kt * C::BK);
+            tma_load_2d_hint(sb + (BN / 64) * kMnAtomBytes, &tmLA, &full[stage], 0,
+                             e * args.b_rows + kt * C::BK, pol_w);
           } else {
             if (kSwiGLU) {
-              tma_load_2d(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * HALF);
-              tma_load_2d(sb + HALF * 128, &tmB, &full[stage], kt * C::BK,
-                          e * args.b_rows + args.I + nt * HALF);
+              tma_load_2d_hint(sb, &tmB, &full[stage], kt * C::BK,
+                               e * args.b_rows + nt * HALF, pol_w);
+              tma_load_2d_hint(sb + HALF * C::BK * 2, &tmB, &full[stage], kt * C::BK,
+                               e * args.b_rows + args.I + nt * HALF, pol_w);
             } else {
-              tma_load_2d(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * BN);
+              tma_load_2d_hint(sb, &tmB, &full[stage], kt * C::BK, e * args.b_rows + nt * BN,
+                               pol_w);
             }
             // factor rows right after the weight rows: one operand of N = BN + r
-            tma_load_2d(sb + BN * 128, &tmLA, &full[stage], kt * C::BK, e * RK);
+            tma_load_2d_hint(sb + BN * C::BK * 2, &tmLA, &full[stage], kt * C::BK, e * RK,
+                             pol_w);
           }
           if (armed_stages < C::NS) ++armed_stages;
           if (++stage == C::NS) {
@@ -507,7 +550,18 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
         umma_commit(&lb_empty[b]);
         umma_commit(&acc_full[b]);
       };
+      // Stage-0 operand descriptors; a stage / K-step moves only the 14-bit
+      // start-address field (shared addresses are < 256 KB, so adding the
+      // byte offset >> 4 never carries out of it).
+      const uint64_t a_desc0 = smem_desc(smem_u32(sStage), 16, kKmajSBO, kKmajLayout);
+      const uint64_t b_desc0 =
+          kBMN ? smem_desc(smem_u32(sStage) + C::A_BYTES, kMnAtomBytes, 1024, kLayoutSW128)
+               : smem_desc(smem_u32(sStage) + C::A_BYTES, 16, kKmajSBO, kKmajLayout);
+      constexpr uint64_t kStageInc = C::STAGE_BYTES >> 4;
+      constexpr uint64_t kAStep = 32 >> 4;                     // 16 K of K-major
+      constexpr uint64_t kBStep = kBMN ? (2048 >> 4) : (32 >> 4);  // 16 K rows / cols
       int stage = 0;
+      uint64_t soff = 0;
       uint32_t phase = 0;
       int local = 0;
       int pending = -1;  // local index of the tile whose up-projection is due
@@ -516,27 +570,30 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
       // end of the kernel, so the bounded wait runs out and the whole CTA
       // takes its abort path.
       if (args.stall_test) ok = mbar_wait(drain_bar, 0, s_abort, wait_ns);
+#ifdef MOE_GEMM_TRACE
+      const long long t_role = clock64();
+#endif
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++local) {
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
-        if (!mbar_wait(&acc_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
+        if (!MOE_TIMED(MODE, 1, mbar_wait(&acc_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < k_iters; ++kt) {
-          if (!mbar_wait(&full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sStage + stage * C::STAGE_BYTES);
-          const uint32_t b0 = a0 + C::A_BYTES;
+          // (TMA -> MMA ordering comes with the barrier; no tcgen05 fence)
+          if (!MOE_TIMED(MODE, 0, mbar_wait(&full[stage], phase, s_abort, wait_ns))) { ok = false; break; }
+          const uint64_t da = a_desc0 + soff, db = b_desc0 + soff;
+          MOE_TIMED_VOID(MODE, 6, ({
+            umma_bf16(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk) {
-            const uint64_t da = smem_desc(a0 + kk * 32, 16, 1024, kLayoutSW128);
-            const uint64_t db = kBMN ? smem_desc(b0 + kk * 2048, 8192, 1024, kLayoutSW128)
-                                     : smem_desc(b0 + kk * 32, 16, 1024, kLayoutSW128);
-            umma_bf16(t_acc, da, db, kIdesc, (kt | kk) ? 1u : 0u);
-          }
-          umma_commit(&empty[stage]);
+            for (int kk = 1; kk < C::BK / 16; ++kk)
+              umma_bf16(t_acc, da + kk * kAStep, db + kk * kBStep, kIdesc, 1u);
+            umma_commit(&empty[stage]);
+          }));
+          soff += kStageInc;
           if (++stage == C::NS) {
             stage = 0;
+            soff = 0;
             phase ^= 1;
           }
           if (pending >= 0) {  // previous tile's up-projection, once it is ready
@@ -554,8 +611,8 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
         if (pending >= 0) {
           const int pb = pending & 1;
           const uint32_t pu = (pending >> 1) & 1;
-          if (!mbar_wait(&xa_ready[pb], pu, s_abort, wait_ns) ||
-              !mbar_wait(&lb_full[pb], pu, s_abort, wait_ns)) { ok = false; break; }
+          if (!MOE_TIMED(MODE, 2, mbar_wait(&xa_ready[pb], pu, s_abort, wait_ns)) ||
+              !MOE_TIMED(MODE, 3, mbar_wait(&lb_full[pb], pu, s_abort, wait_ns))) { ok = false; break; }
           tc_fence_after();
           issue_up(pb);
         }
@@ -570,6 +627,10 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
           issue_up(pb);
         }
       }
+#ifdef MOE_GEMM_TRACE
+      atomicAdd(&g_gemm_trace[MODE][blockIdx.x % 160][7],
+                static_cast<unsigned long long>(clock64() - t_role));
+#endif
       // every MMA issued by this thread must be complete before TMEM is freed
       umma_commit(drain_bar);
       drain_wait(drain_bar, 0, wait_ns);
@@ -595,7 +656,7 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
       // rank-r product: TMEM -> bf16 A operand of the up-projection (done by
       // the first four epilogue warps)
       if (ehalf == 0) {
-        if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
+        if (!MOE_TIMED(MODE, 8, warp_wait(&lora_full[b], use, s_abort, wait_ns))) break;
         tc_fence_after();
         epi_rank_handoff<RK>(args, t_lora, sXA + b * C::XA_BYTES, row_in_tile, nt, rvalid,
                              grow);
@@ -606,9 +667,9 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
       }
       if constexpr (MODE == kDownBwd) epi_prefetch_saved<BN>(args, grow, rvalid, nt, ehalf);
 
-      if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
+      if (!MOE_TIMED(MODE, 9, warp_wait(&acc_full[b], use, s_abort, wait_ns))) break;
       tc_fence_after();
-      epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
+      MOE_TIMED_VOID(MODE, 10, (epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf)));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);

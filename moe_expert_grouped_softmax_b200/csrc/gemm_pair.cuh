@@ -248,10 +248,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           const int b = local & 1;
           const uint32_t use = (local >> 1) & 1;
           if (!mbar_wait(&lb_full[b], use, s_abort, wait_ns)) { ok = false; break; }
-          mbar_arrive_cluster(lead(&peer_lb[b]));
+          mbar_arrive_cluster_relaxed(lead(&peer_lb[b]));
           for (int kt = 0; kt < k_iters; ++kt) {
             if (!mbar_wait(&full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
-            mbar_arrive_cluster(lead(&peer_full[stage]));
+            mbar_arrive_cluster_relaxed(lead(&peer_full[stage]));
             if (++stage == C::NS) {
               stage = 0;
               phase ^= 1;
@@ -275,7 +275,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         umma_commit_pair_mc(&lb_empty[b], kBoth);
         umma_commit_pair_mc(&acc_full[b], kBoth);
       };
+      const uint64_t a_desc0 = smem_desc(smem_u32(sStage), 16, 1024, kLayoutSW128);
+      const uint64_t b_desc0 = smem_desc(smem_u32(sStage) + C::A_BYTES, 16, 1024, kLayoutSW128);
+      constexpr uint64_t kStageInc = C::STAGE_BYTES >> 4;
       int stage = 0;
+      uint64_t soff = 0;
       uint32_t phase = 0;
       int local = 0;
       int pending = -1;
@@ -290,17 +294,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         for (int kt = 0; kt < k_iters; ++kt) {
           if (!mbar_wait(&full[stage], phase, s_abort, wait_ns) ||
               !mbar_wait_cluster(&peer_full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sStage + stage * C::STAGE_BYTES);
-          const uint32_t b0 = a0 + C::A_BYTES;
+          const uint64_t da = a_desc0 + soff, db = b_desc0 + soff;
+          umma_bf16_pair(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)
-            umma_bf16_pair(t_acc, smem_desc(a0 + kk * 32, 16, 1024, kLayoutSW128),
-                           smem_desc(b0 + kk * 32, 16, 1024, kLayoutSW128), kIdesc,
-                           (kt | kk) ? 1u : 0u);
+          for (int kk = 1; kk < C::BK / 16; ++kk)
+            umma_bf16_pair(t_acc, da + 2 * kk, db + 2 * kk, kIdesc, 1u);
           umma_commit_pair_mc(&empty[stage], kBoth);
+          soff += kStageInc;
           if (++stage == C::NS) {
             stage = 0;
+            soff = 0;
             phase ^= 1;
           }
           if (pending >= 0) {

@@ -134,6 +134,10 @@ CUtensorMapSwizzle lora_swizzle(int r) {
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// swizzle of the single-CTA kernel's K-major operand boxes (kGemmBK wide)
+constexpr CUtensorMapSwizzle kKmajSwz =
+    kGemmBK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
 inline int ld_rank(int R) { return (R + 63) & ~63; }  // row pitch of [r, R] parts
 
 moe_status_t launch_status() {
@@ -381,6 +385,19 @@ int moe_profile_collect(int kind, float* ms, int max_n) {
   return n;
 }
 
+#ifdef MOE_GEMM_TRACE
+// Instrumented builds only: copies (and clears) the per-CTA wait counters.
+MOE_API int moe_debug_read_trace(unsigned long long* out, int n) {
+  const int total = static_cast<int>(sizeof(g_gemm_trace) / sizeof(unsigned long long));
+  if (n < total) return -total;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(out, g_gemm_trace, sizeof(g_gemm_trace)) != cudaSuccess) return -1;
+  static unsigned long long zeros[sizeof(g_gemm_trace) / sizeof(unsigned long long)];
+  if (cudaMemcpyToSymbol(g_gemm_trace, zeros, sizeof(g_gemm_trace)) != cudaSuccess) return -1;
+  return total;
+}
+#endif
+
 moe_status_t moe_get_device_status(moe_stream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
   int v = 0, zero = 0;
@@ -576,9 +593,9 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
   } else {
     const int bn = pick_bn(I, true, r, false), half = bn / 2;
     CUtensorMap ta, tb, tla, tlb;
-    bool ok = tmap_2d(&ta, Xp, H, R, H * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, half, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, A1, H, EU * r, H * 2ull, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = tmap_2d(&ta, Xp, H, R, H * 2ull, kGemmBK, 128, kKmajSwz);
+    ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, kGemmBK, half, kKmajSwz);
+    ok = ok && tmap_2d(&tla, A1, H, EU * r, H * 2ull, kGemmBK, r, kKmajSwz);
     ok = ok && tmap_2d(&tlb, B1, r, EU * 2 * I, r * 2ull, r, half, lsw);
     if (!ok) return MOE_ERR_CUDA;
     GemmArgs g{};
@@ -604,9 +621,9 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
   } else {
     const int bn = pick_bn(H, false, r, false);
     CUtensorMap ta, tb, tla, tlb;
-    bool ok = tmap_2d(&ta, h, I, R, I * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tb, W2, I, EU * H, I * 2ull, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, A2, I, EU * r, I * 2ull, 64, r, CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = tmap_2d(&ta, h, I, R, I * 2ull, kGemmBK, 128, kKmajSwz);
+    ok = ok && tmap_2d(&tb, W2, I, EU * H, I * 2ull, kGemmBK, bn, kKmajSwz);
+    ok = ok && tmap_2d(&tla, A2, I, EU * r, I * 2ull, kGemmBK, r, kKmajSwz);
     ok = ok && tmap_2d(&tlb, B2, r, EU * H, r * 2ull, r, bn, lsw);
     if (!ok) return MOE_ERR_CUDA;
     GemmArgs g{};
@@ -681,9 +698,9 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
   {
     const int bn = pick_bn(I, false, r, true);
     CUtensorMap ta, tb, tla, tlb;
-    bool ok = tmap_2d(&ta, dZ2, H, R, H * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tb, W2, I, EU * H, I * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, B2p, 64, EU * H, 128, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = tmap_2d(&ta, dZ2, H, R, H * 2ull, kGemmBK, 128, kKmajSwz);
+    ok = ok && tmap_2d(&tb, W2, I, EU * H, I * 2ull, 64, kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, B2p, 64, EU * H, 128, 64, kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && tmap_2d(&tlb, A2t, r, EU * I, r * 2ull, r, bn, lsw);
     if (!ok) return MOE_ERR_CUDA;
     GemmArgs g{};
@@ -699,9 +716,9 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
   {
     const int bn = pick_bn(H, false, r, true);
     CUtensorMap ta, tb, tla, tlb;
-    bool ok = tmap_2d(&ta, dZ1, 2 * I, R, 4ull * I, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, B1p, 64, EU * 2 * I, 128, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = tmap_2d(&ta, dZ1, 2 * I, R, 4ull * I, kGemmBK, 128, kKmajSwz);
+    ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, B1p, 64, EU * 2 * I, 128, 64, kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && tmap_2d(&tlb, A1t, r, EU * H, r * 2ull, r, bn, lsw);
     if (!ok) return MOE_ERR_CUDA;
     GemmArgs g{};
