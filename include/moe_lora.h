@@ -199,10 +199,13 @@ MOE_API void moe_set_wait_limit_ns(uint64_t ns);
 MOE_API void moe_test_inject_stall(int on);
 
 /* Kernel choice for the forward grouped GEMMs (not thread-safe; takes effect
- * at the next moe_lora_mlp_fwd call): 1 runs them on CTA pairs (256-row
- * tiles on the 2-SM tensor-core instruction), 0 (default) on single CTAs
- * (128-row tiles).  Both compute the same result. */
-MOE_API void moe_set_forward_pairs(int on);
+ * at the next moe_lora_mlp_fwd call): mode > 0 runs them on CTA pairs
+ * (256-row tiles on the 2-SM tensor-core instruction), mode == 0 on single
+ * CTAs (128-row tiles), mode < 0 (the default) chooses per GEMM: pairs when
+ * the mean rows per expert R / E is at least 768 (little padding on each
+ * expert's ragged last 256-row tile) and the GEMM's K (H for gate_up, I for
+ * down) is at least 1024.  All compute the same result. */
+MOE_API void moe_set_forward_pairs(int mode);
 
 /* Benchmark hook (not thread-safe; for measurement only).
  * moe_profile_enable(1) starts recording, for every kernel kind below, a pair

@@ -191,6 +191,20 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// drain_wait for a barrier that other CTAs of the cluster arrive on with
+// release semantics (acquire at cluster scope).
+__device__ __forceinline__ void drain_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                   uint64_t limit_ns) {
+  const uint64_t limit = limit_ns > 1000000000ull ? limit_ns : 1000000000ull;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit) {
+      set_status(4);
+      return;
+    }
+  }
+}
+
 // Builds the m-tile table in shared memory (one warp): s_off = offsets,
 // s_mstart[e] = first global m-tile (of 2^bm_shift rows) of expert e,
 // s_mstart[E] = total.

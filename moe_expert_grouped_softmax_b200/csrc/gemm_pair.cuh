@@ -13,22 +13,44 @@
 // same accumulator during the next tile's mainloop.
 //
 // Synchronisation (every wait bounded):
-//  * each CTA's TMA loads complete on its own barriers (so each CTA can
-//    always drain its own copies); the odd CTA ("peer") relays "my half of
-//    stage s has landed" to a second barrier of the leader with a remote
-//    mbarrier arrive, so no asynchronous copy ever signals the other CTA;
+//  * both CTAs' TMA loads of a stage complete on the leader's barrier (the
+//    pair form of the tensor copy signals a barrier of either CTA); only the
+//    leader arms it, for the bytes of both halves;
 //  * the leader's MMA commits are multicast to both CTAs' barriers
 //    (stage free, rank-r product ready, accumulator ready);
 //  * both CTAs' epilogues arrive on the leader's barriers (hand-off written,
 //    accumulator drained);
 //  * at exit, each CTA waits for the leader's last MMAs (which touch its
-//    shared memory and TMEM), and the leader waits for the peer's final
-//    arrive, so neither leaves while the other can still reach it.
+//    shared memory and TMEM); the peer then tells the leader how many copies
+//    it issued, the leader balances and waits out every copy either CTA has
+//    in flight (all complete on its barriers) and releases the peer, so
+//    neither leaves while a copy, an MMA or an arrive can still reach it.
 #pragma once
 
 #include "gemm.cuh"
 
 namespace moe {
+
+// Teardown of the leader: every copy of either CTA completes on the
+// leader's barriers bars[0..n) (phase q / n of barrier q % n for the q-th
+// copy).  The leader armed its first `mine` phases for both halves; the
+// peer issued its first `peers` halves.  Arm what only the peer issued,
+// balance what the peer never issued, and wait out the last n phases
+// (earlier ones completed before any later copy could be issued).
+__device__ __forceinline__ void drain_pair_copies(uint64_t* bars, int n, uint32_t bytes,
+                                                  int mine, int peers, uint64_t limit_ns) {
+  const int hi = mine > peers ? mine : peers;
+  const int lo = hi - n > 0 ? hi - n : 0;
+  for (int q = lo; q < hi; ++q) {
+    uint64_t* bar = &bars[q % n];
+    if (q >= mine) {
+      mbar_arrive_expect_tx(bar, bytes);
+    } else if (q >= peers) {
+      mbar_complete_tx(bar, bytes);
+    }
+    drain_wait(bar, static_cast<uint32_t>(q / n) & 1u, limit_ns);
+  }
+}
 
 template <int MODE, int BN, int RK>
 struct PairCfg {
@@ -50,7 +72,7 @@ struct PairCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int LB_BYTES = HALF * RK * 2;    // this CTA's half of LB
   static constexpr int XA_BYTES = BM * RK * 2;
-  static constexpr int MISC_BYTES = 512 + 8 * 520;  // barriers, flags, tables
+  static constexpr int MISC_BYTES = 512 + 8 * 520;  // barriers, counts, tables
   static constexpr int FIXED = 2 * LB_BYTES + 2 * XA_BYTES + MISC_BYTES;
   static constexpr int NS_FIT = (kSmemOptin - 1024 - FIXED) / STAGE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
@@ -106,13 +128,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
   uint64_t* xa_ready = lora_full + 2;
   uint64_t* acc_full = xa_ready + 2;
   uint64_t* acc_empty = acc_full + 2;
-  uint64_t* peer_full = acc_empty + 2;       // leader: peer's half landed
-  uint64_t* peer_lb = peer_full + C::NS;      // leader: peer's LB half landed
-  uint64_t* final_bar = peer_lb + 2;
-  uint64_t* peer_done = final_bar + 1;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(peer_done + 1);
+  uint64_t* final_bar = acc_empty + 2;
+  uint64_t* peer_done = final_bar + 1;       // leader: the peer is done
+  uint64_t* drained = peer_done + 1;         // peer: its copies have landed
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  int* s_off = reinterpret_cast<int*>(s_tmem + 4);
+  // copies issued by this CTA's producer: [0] stages, [1] up-factor halves;
+  // [2], [3]: the same counts of the peer (written into the leader)
+  int* s_issued = reinterpret_cast<int*>(s_tmem + 4);
+  int* s_off = s_issued + 4;
   int* s_mstart = s_off + 520;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,11 +150,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
-      mbar_init(&peer_full[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&lb_full[i], 1);
-      mbar_init(&peer_lb[i], 1);
       mbar_init(&lb_empty[i], 1);
       mbar_init(&lora_full[i], 1);
       mbar_init(&xa_ready[i], 2 * C::EPI_WARPS);
@@ -139,6 +161,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
     }
     mbar_init(final_bar, 1);
     mbar_init(peer_done, 1);
+    mbar_init(drained, 1);
+    for (int i = 0; i < 4; ++i) s_issued[i] = 0;
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -163,16 +187,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
   const int total_tiles = s_mstart[E] * args.n_tiles;
   const int k_iters = (args.K + C::BK - 1) / C::BK;
   // cluster addresses of the leader's copies of the barriers
-  auto lead = [&](uint64_t* bar) { return mapa_shared(smem_u32(bar), 0); };
+  auto lead = [&](const void* p) { return mapa_shared(smem_u32(p), 0); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int armed_stages = 0;
-      uint32_t lb_armed = 0;
-      uint32_t lb_par[2] = {0, 0};
+      int n_st = 0, n_lb = 0;
       bool ok = true;
       int local = 0;
       for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++local) {
@@ -182,84 +204,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         if (!mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
-        mbar_arrive_expect_tx(&lb_full[b], C::LB_BYTES);
-        lb_armed |= 1u << b;
-        lb_par[b] = use;
+        if (leader) mbar_arrive_expect_tx(&lb_full[b], 2 * C::LB_BYTES);
         // this CTA's half of the up-projection factor: output columns
         // [rank * BN/2, (rank + 1) * BN/2) of the tile
         const int lb_row = kSwiGLU ? e * args.lb_rows + (rank ? args.I : 0) + nt * HALF
                                    : e * args.lb_rows + nt * BN + static_cast<int>(rank) * HALF;
-        tma_load_2d(sLB + b * C::LB_BYTES, &tmLB, &lb_full[b], 0, lb_row);
+        tma_load_2d_pair(sLB + b * C::LB_BYTES, &tmLB, lead(&lb_full[b]), 0, lb_row);
+        ++n_lb;
         for (int kt = 0; kt < k_iters; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, wait_ns)) { ok = false; break; }
           uint8_t* st = sStage + stage * C::STAGE_BYTES;
           uint8_t* sb = st + C::A_BYTES;
           const int kx = kt * C::BK;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(st, &tmA, &full[stage], kx, row0);
+          const uint32_t fb = lead(&full[stage]);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(st, &tmA, fb, kx, row0);
           if (kSwiGLU) {
             const int gate = e * args.b_rows + nt * HALF;
             const int up = e * args.b_rows + args.I + nt * HALF;
             if (rank == 0) {
-              tma_load_2d(sb, &tmW0, &full[stage], kx, gate);
-              tma_load_2d(sb + HALF * 128, &tmW1, &full[stage], kx, up);
+              tma_load_2d_pair(sb, &tmW0, fb, kx, gate);
+              tma_load_2d_pair(sb + HALF * 128, &tmW1, fb, kx, up);
             } else {
-              tma_load_2d(sb, &tmW2, &full[stage], kx, up + C::U0);
-              tma_load_2d(sb + C::U1 * 128, &tmLA, &full[stage], kx, e * RK);
+              tma_load_2d_pair(sb, &tmW2, fb, kx, up + C::U0);
+              tma_load_2d_pair(sb + C::U1 * 128, &tmLA, fb, kx, e * RK);
             }
           } else {
             const int w = e * args.b_rows + nt * BN;
             if (rank == 0) {
-              tma_load_2d(sb, &tmW0, &full[stage], kx, w);
+              tma_load_2d_pair(sb, &tmW0, fb, kx, w);
             } else {
-              tma_load_2d(sb, &tmW2, &full[stage], kx, w + C::W0);
-              tma_load_2d(sb + C::W1 * 128, &tmLA, &full[stage], kx, e * RK);
+              tma_load_2d_pair(sb, &tmW2, fb, kx, w + C::W0);
+              tma_load_2d_pair(sb + C::W1 * 128, &tmLA, fb, kx, e * RK);
             }
           }
-          if (armed_stages < C::NS) ++armed_stages;
+          ++n_st;
           if (++stage == C::NS) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      // own loads complete on own barriers: wait for all of them to land
-      for (int i = 0; i < armed_stages; ++i) {
-        int s = stage - 1 - i;
-        uint32_t ph = phase;
-        if (s < 0) {
-          s += C::NS;
-          ph ^= 1;
-        }
-        drain_wait(&full[s], ph, wait_ns);
-      }
-      for (int bb = 0; bb < 2; ++bb)
-        if (lb_armed & (1u << bb)) drain_wait(&lb_full[bb], lb_par[bb], wait_ns);
+      // every copy lands on the leader's barriers; the teardown waits them out
+      s_issued[0] = n_st;
+      s_issued[1] = n_lb;
     }
   } else if (warp == 1) {
-    if (!leader) {
-      // ---------------------------------------------------------- relay (peer)
-      if (lane == 0) {
-        int stage = 0;
-        uint32_t phase = 0;
-        int local = 0;
-        bool ok = true;
-        for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++local) {
-          const int b = local & 1;
-          const uint32_t use = (local >> 1) & 1;
-          if (!mbar_wait(&lb_full[b], use, s_abort, wait_ns)) { ok = false; break; }
-          mbar_arrive_cluster_relaxed(lead(&peer_lb[b]));
-          for (int kt = 0; kt < k_iters; ++kt) {
-            if (!mbar_wait(&full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
-            mbar_arrive_cluster_relaxed(lead(&peer_full[stage]));
-            if (++stage == C::NS) {
-              stage = 0;
-              phase ^= 1;
-            }
-          }
-        }
-      }
-    } else if (lane == 0) {
+    if (leader && lane == 0) {
       // ---------------------------------------------------------- MMA (leader)
       constexpr uint32_t kIdesc = idesc_bf16_f32(256, C::NMMA, false, false);
       constexpr uint32_t kIdescUp = idesc_bf16_f32(256, BN, false, false);
@@ -285,15 +276,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       int pending = -1;
       bool ok = true;
       if (args.stall_test) ok = mbar_wait(final_bar, 0, s_abort, wait_ns);
+#ifdef MOE_GEMM_TRACE
+      const long long t_role = clock64();
+#endif
       for (int tile = pair; ok && tile < total_tiles; tile += npairs, ++local) {
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
-        if (!mbar_wait_cluster(&acc_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
+        if (!MOE_TIMED(MODE, 14, mbar_wait_cluster(&acc_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < k_iters; ++kt) {
-          if (!mbar_wait(&full[stage], phase, s_abort, wait_ns) ||
-              !mbar_wait_cluster(&peer_full[stage], phase, s_abort, wait_ns)) { ok = false; break; }
+          if (!MOE_TIMED(MODE, 11, mbar_wait(&full[stage], phase, s_abort, wait_ns))) { ok = false; break; }
           const uint64_t da = a_desc0 + soff, db = b_desc0 + soff;
           umma_bf16_pair(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
 #pragma unroll
@@ -309,8 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           if (pending >= 0) {
             const int pb = pending & 1;
             const uint32_t pu = (pending >> 1) & 1;
-            if (mbar_test_wait_cluster(&xa_ready[pb], pu) &&
-                mbar_test_wait(&lb_full[pb], pu) && mbar_test_wait_cluster(&peer_lb[pb], pu)) {
+            if (mbar_test_wait_cluster(&xa_ready[pb], pu) && mbar_test_wait(&lb_full[pb], pu)) {
               tc_fence_after();
               issue_up(pb);
               pending = -1;
@@ -323,8 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           const int pb = pending & 1;
           const uint32_t pu = (pending >> 1) & 1;
           if (!mbar_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) ||
-              !mbar_wait(&lb_full[pb], pu, s_abort, wait_ns) ||
-              !mbar_wait_cluster(&peer_lb[pb], pu, s_abort, wait_ns)) { ok = false; break; }
+              !mbar_wait(&lb_full[pb], pu, s_abort, wait_ns)) { ok = false; break; }
           tc_fence_after();
           issue_up(pb);
         }
@@ -334,12 +325,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         const int pb = pending & 1;
         const uint32_t pu = (pending >> 1) & 1;
         if (mbar_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) &&
-            mbar_wait(&lb_full[pb], pu, s_abort, wait_ns) &&
-            mbar_wait_cluster(&peer_lb[pb], pu, s_abort, wait_ns)) {
+            mbar_wait(&lb_full[pb], pu, s_abort, wait_ns)) {
           tc_fence_after();
           issue_up(pb);
         }
       }
+#ifdef MOE_GEMM_TRACE
+      atomicAdd(&g_gemm_trace[MODE][blockIdx.x % 160][13],
+                static_cast<unsigned long long>(clock64() - t_role));
+#endif
       // all of the leader's MMAs complete -> both CTAs' final_bar
       umma_commit_pair_mc(final_bar, kBoth);
     }
@@ -381,9 +375,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
     // the leader's MMAs read this CTA's shared memory and write its TMEM
     drain_wait(final_bar, 0, wait_ns);
     if (!leader) {
-      mbar_arrive_cluster(lead(peer_done));  // no more arrives from this CTA
+      // publish this CTA's copy counts; the release orders them before the
+      // arrive, after which nothing else arrives from this CTA
+      st_shared_cluster_s32(lead(&s_issued[2]), s_issued[0]);
+      st_shared_cluster_s32(lead(&s_issued[3]), s_issued[1]);
+      mbar_arrive_cluster(lead(peer_done));
+      drain_wait(drained, 0, wait_ns);        // the leader saw every copy land
     } else {
-      drain_wait(peer_done, 0, wait_ns);
+      drain_wait_cluster(peer_done, 0, wait_ns);
+      drain_pair_copies(full, C::NS, C::STAGE_BYTES, s_issued[0], s_issued[2], wait_ns);
+      drain_pair_copies(lb_full, 2, C::LB_BYTES, s_issued[1], s_issued[3], wait_ns);
+      mbar_arrive_cluster(mapa_shared(smem_u32(drained), 1));
     }
   }
   __syncthreads();

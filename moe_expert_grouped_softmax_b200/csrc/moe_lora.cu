@@ -55,7 +55,17 @@ moe_status_t route_scratch_on_current_device(void** out) {
 
 uint64_t g_wait_limit_ns = 1000000000ull;  // one second per bounded wait
 int g_stall_test = 0;                      // testing hook, see moe_test_inject_stall
-int g_forward_pairs = 0;                   // forward GEMMs on CTA pairs
+int g_forward_pairs = -1;                  // forward GEMMs on CTA pairs: <0 auto
+// Automatic choice: CTA pairs when the mean rows per expert fill at least
+// three 256-row tiles (little padding on each expert's ragged last tile) and
+// K is long enough (16 k-steps) for the per-tile hand-offs to stay hidden.
+constexpr int kPairMinRowsPerExpert = 768;
+constexpr int kPairMinK = 1024;
+bool use_pairs(int R, int E, int K) {
+  if (g_forward_pairs >= 0) return g_forward_pairs > 0;
+  return static_cast<int64_t>(R) >= static_cast<int64_t>(kPairMinRowsPerExpert) * E &&
+         K >= kPairMinK;
+}
 
 // ------------------------------------------------ optional per-kernel timing
 // When enabled, each launch site of a kernel kind records a CUDA event before
@@ -358,7 +368,7 @@ void moe_set_wait_limit_ns(uint64_t ns) {
 
 void moe_test_inject_stall(int on) { g_stall_test = on ? 1 : 0; }
 
-void moe_set_forward_pairs(int on) { g_forward_pairs = on ? 1 : 0; }
+void moe_set_forward_pairs(int mode) { g_forward_pairs = mode > 0 ? 1 : (mode == 0 ? 0 : -1); }
 
 moe_status_t moe_profile_enable(int on) {
   if (on && !g_prof_created) {
@@ -580,7 +590,7 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
   const uint64_t EU = static_cast<uint64_t>(E);
 
   // gate_up + SwiGLU
-  if (g_forward_pairs) {
+  if (use_pairs(R, E, H)) {
     const int bn = 256 - r, half = bn / 2;
     GemmArgs g{};
     g.offsets = expert_offsets;
@@ -608,7 +618,7 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     if ((stt = launch_gemm<kGateUpFwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   // down
-  if (g_forward_pairs) {
+  if (use_pairs(R, E, I)) {
     const int bn = 256 - r;
     GemmArgs g{};
     g.offsets = expert_offsets;

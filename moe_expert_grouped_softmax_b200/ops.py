@@ -123,8 +123,9 @@ def set_wait_limit_ns(ns):
 
 
 def set_forward_pairs(on=True):
-    """Forward GEMMs on CTA pairs (256-row tiles) or single CTAs."""
-    lib().moe_set_forward_pairs(1 if on else 0)
+    """Forward GEMMs on CTA pairs (True, 256-row tiles), single CTAs (False)
+    or chosen per call from the mean rows per expert (None, the default)."""
+    lib().moe_set_forward_pairs(-1 if on is None else (1 if on else 0))
 
 
 def test_inject_stall(on=True):

@@ -125,8 +125,9 @@ BLOCK_CASES = {
 }
 
 
-# every case on the default single-CTA forward kernels; the cases marked
-# "/pairs" again with the CTA-pair forward kernels
+# every case forced onto the single-CTA forward kernels; the cases marked
+# "/pairs" again forced onto the CTA-pair forward kernels (the default
+# chooses between them from the mean rows per expert)
 BLOCK_RUNS = [(c, False) for c in BLOCK_CASES] + [
     (c, True) for c in ("tiny", "ragged", "rank32", "rank64", "skew_empty")]
 
@@ -147,7 +148,7 @@ def block_run(request, cuda_ok):
         blk.step(g["X"], g["logits"], g["dY"], W)
         torch.cuda.synchronize()
     finally:
-        ops.set_forward_pairs(False)
+        ops.set_forward_pairs(None)
     status = ops.device_status()
     return dict(name=name, pairs=pairs, cfg=cfg, inp=inp, Y=Y, ctx=ctx, grads=grads,
                 blk=blk, status=status)
@@ -215,6 +216,6 @@ def test_block_deterministic(block_run):
     try:
         b.step(g["X"], g["logits"], g["dY"], W)
     finally:
-        ops.set_forward_pairs(False)
+        ops.set_forward_pairs(None)
     for x, y in zip(first, (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2)):
         assert torch.equal(x, y)
