@@ -167,8 +167,8 @@ def run_ours(args, cfg):
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
-    if args.forward_pairs >= 0:
-        ops.set_forward_pairs(bool(args.forward_pairs))
+    if args.cta_pairs >= 0:
+        ops.set_cta_pairs(bool(args.cta_pairs))
     dev = torch.device("cuda", local)
     if ws > 1:
         dist.init_process_group("nccl", device_id=dev,
@@ -203,11 +203,13 @@ def run_ours(args, cfg):
     barrier()
     torch.cuda.synchronize()
     clk.t_begin = time.time()
+    launches0 = ops.kernel_launches()
     for i in range(K):
         flush.zero_()                      # L2 flush, outside the timed span
         ev0[i].record(stream)
         blk.step(X, logits, dY, W)
         ev1[i].record(stream)
+    launches = ops.kernel_launches() - launches0
     torch.cuda.synchronize()
     clk.t_end = time.time()
     barrier()
@@ -307,7 +309,7 @@ def run_ours(args, cfg):
         dist.destroy_process_group()
     return dict(ms_total=ms_total, ms_steps=ms_steps, kern=kern, e2e=e2e,
                 clocks=clk.summary(), counts=counts, ws=ws, rank=rank,
-                launches=ops.MoeBlock.KERNELS_PER_STEP * K)
+                launches=launches)
 
 
 _CPU_INPUTS = {}
@@ -348,8 +350,8 @@ def main():
     ap.add_argument("--cpu-sample-tokens", type=int, default=128)
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (small cases for profiler captures)")
-    ap.add_argument("--forward-pairs", type=int, default=-1,
-                    help="1: forward GEMMs on CTA pairs, 0: single CTAs, "
+    ap.add_argument("--cta-pairs", type=int, default=-1,
+                    help="1: grouped GEMMs on CTA pairs, 0: single CTAs, "
                          "-1: library default")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -198,14 +198,19 @@ MOE_API void moe_set_wait_limit_ns(uint64_t ns);
  * exercises the timeout path without faulting or hanging the GPU. */
 MOE_API void moe_test_inject_stall(int on);
 
-/* Kernel choice for the forward grouped GEMMs (not thread-safe; takes effect
- * at the next moe_lora_mlp_fwd call): mode > 0 runs them on CTA pairs
- * (256-row tiles on the 2-SM tensor-core instruction), mode == 0 on single
- * CTAs (128-row tiles), mode < 0 (the default) chooses per GEMM: pairs when
- * the mean rows per expert R / E is at least 768 (little padding on each
- * expert's ragged last 256-row tile) and the GEMM's K (H for gate_up, I for
- * down) is at least 1024.  All compute the same result. */
-MOE_API void moe_set_forward_pairs(int mode);
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams), counted on the host at each launch; for measurement. */
+MOE_API unsigned long long moe_kernel_launches(void);
+
+/* Kernel choice for the four grouped GEMMs (not thread-safe; takes effect at
+ * the next moe_lora_mlp_fwd / moe_lora_mlp_bwd call): mode > 0 runs them on
+ * CTA pairs (256-row tiles on the 2-SM tensor-core instruction), mode == 0
+ * on single CTAs (128-row tiles), mode < 0 (the default) chooses per GEMM:
+ * a forward GEMM runs on pairs when the mean rows per expert R / E is at
+ * least 768 (little padding on each expert's ragged last 256-row tile) and
+ * its K is at least 1024 (H for gate_up, I for down); the backward GEMMs run
+ * on single CTAs.  All compute the same result. */
+MOE_API void moe_set_cta_pairs(int mode);
 
 /* Benchmark hook (not thread-safe; for measurement only).
  * moe_profile_enable(1) starts recording, for every kernel kind below, a pair

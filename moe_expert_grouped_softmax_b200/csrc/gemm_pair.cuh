@@ -1,11 +1,16 @@
-// a3 / a4 on CTA pairs: the forward grouped GEMMs with 256-row tiles on the
+// a3, a4, a7, a8 on CTA pairs: the grouped GEMMs with 256-row tiles on the
 // 2-SM tensor-core instruction (tcgen05.mma.cta_group::2).
 //
 // A cluster of two CTAs on two SMs computes one 256 x BN tile of one expert.
 // Each CTA stages its own 128 rows of A and half of the B operand
-// [W rows (BN) ; LoRA-down factor rows (r)] (N = BN + r, split into two
-// halves of N/2 rows), so every SM moves a third less operand data per FLOP
-// than the single-CTA 128-row tile.  The even CTA ("leader") issues the
+// [W (BN columns) ; LoRA-down factor (r columns)] (N = BN + r, split into two
+// halves of N/2), so every SM moves a third less operand data per FLOP
+// than the single-CTA 128-row tile, through shared memory as well as from L2.
+// Forward (K-major B): the halves are row blocks of W and of the factor.
+// Backward (MN-major B, W read in place as [K, N]): 32-column atoms with the
+// 64-byte swizzle, one TMA box of 32 columns x 64 K-rows each; the r factor
+// columns (B2 or B1, zero-padded to a multiple of 32 columns when r = 16) fill
+// whole atoms next to the weight columns, so BN = 256 - round_up(r, 32).  The even CTA ("leader") issues the
 // MMAs, which read both CTAs' shared memory and write both CTAs' TMEM (each
 // holds its 128 rows x N columns).  The split-LoRA schedule is the one of the
 // single-CTA kernel: rank-r down-projection inside the mainloop MMA,
@@ -54,15 +59,17 @@ __device__ __forceinline__ void drain_pair_copies(uint64_t* bars, int n, uint32_
 
 template <int MODE, int BN, int RK>
 struct PairCfg {
-  static_assert(MODE == kGateUpFwd || MODE == kDownFwd, "pair kernel: forward only");
   static constexpr bool kSwiGLU = (MODE == kGateUpFwd);
+  static constexpr bool kBMN = (MODE == kDownBwd || MODE == kGateUpBwd);
   static constexpr int BM = 128, BK = 64;           // rows per CTA
-  static constexpr int NMMA = BN + RK;              // N of the fused MMA
+  // factor columns in the fused B operand (MN-major: whole 32-column atoms)
+  static constexpr int FPAD = kBMN ? (RK + 31) / 32 * 32 : RK;
+  static constexpr int NMMA = BN + FPAD;            // N of the fused MMA
   static constexpr int NH = NMMA / 2;               // B rows per CTA
   static constexpr int HALF = BN / 2;
-  // B segments of each CTA (rows): SwiGLU: CTA0 = gate HALF + up U0,
-  // CTA1 = up U1 + factor RK.  Plain: CTA0 = W0 weight rows, CTA1 = W1
-  // weight rows + factor RK.
+  // B segments of each CTA (rows of N): SwiGLU: CTA0 = gate HALF + up U0,
+  // CTA1 = up U1 + factor RK.  Plain and backward: CTA0 = W0 weight
+  // columns, CTA1 = W1 weight columns + factor RK.
   static constexpr int U0 = NH - HALF;              // = RK / 2
   static constexpr int U1 = HALF - U0;
   static constexpr int W0 = NH;
@@ -82,13 +89,18 @@ struct PairCfg {
       RK == 16 ? kLayoutSW32 : (RK == 32 ? kLayoutSW64 : kLayoutSW128);
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_STRIDE = 256;
-  static constexpr int EPI_WARPS = 4;
+  static constexpr int EPI_WARPS = gemm_epi_warps(MODE);
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  // MN-major B: one 32-column x BK-row box (64-byte swizzle) per atom
+  static constexpr int MN_COLS = 32;
+  static constexpr int MN_BOX = MN_COLS * BK * 2;
+  static_assert(!kBMN || (W0 % MN_COLS == 0 && W1 % MN_COLS == 0 && NMMA == 256),
+                "MN-major halves in whole 32-column atoms");
   static_assert(NS >= 3, "not enough shared memory for three stages");
   static_assert(SMEM_BYTES <= kSmemOptin, "shared memory over the opt-in limit");
   static_assert(NMMA <= ACC_STRIDE && NMMA % 16 == 0, "MMA N = BN + r");
   static_assert(BN % 16 == 0 && NH % 8 == 0, "8-row operand atoms");
-  static_assert(U0 % 8 == 0 && U1 % 8 == 0 && U1 > 0, "SwiGLU segments");
+  static_assert(!kSwiGLU || (U0 % 8 == 0 && U1 % 8 == 0 && U1 > 0), "SwiGLU segments");
   static_assert(W1 % 8 == 0 && W1 > 0, "plain segments");
 };
 
@@ -112,6 +124,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
                                   const GemmArgs args) {
   using C = PairCfg<MODE, BN, RK>;
   constexpr bool kSwiGLU = C::kSwiGLU;
+  constexpr bool kBMN = C::kBMN;
   constexpr int HALF = C::HALF;
 
   extern __shared__ uint8_t smem_raw[];
@@ -155,7 +168,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       mbar_init(&lb_full[i], 1);
       mbar_init(&lb_empty[i], 1);
       mbar_init(&lora_full[i], 1);
-      mbar_init(&xa_ready[i], 2 * C::EPI_WARPS);
+      mbar_init(&xa_ready[i], 2 * 4);
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 2 * C::EPI_WARPS);
     }
@@ -219,7 +232,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           const uint32_t fb = lead(&full[stage]);
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           tma_load_2d_pair(st, &tmA, fb, kx, row0);
-          if (kSwiGLU) {
+          if constexpr (kBMN) {
+            // W [K, N] in place: this CTA's weight columns, then (CTA1) the
+            // factor's columns, one 32-column atom per box
+            constexpr int A = C::MN_COLS;
+            const int nw = rank ? C::W1 : C::W0;
+            const int n0 = nt * BN + (rank ? C::W0 : 0);
+            const int krow = e * args.b_rows + kx;
+            for (int i = 0; i < nw / A; ++i)
+              tma_load_2d_pair(sb + i * C::MN_BOX, &tmW0, fb, n0 + A * i, krow);
+            if (rank) {
+#pragma unroll
+              for (int i = 0; i < C::FPAD / A; ++i)
+                tma_load_2d_pair(sb + (nw / A + i) * C::MN_BOX, &tmLA, fb, A * i, krow);
+            }
+          } else if (kSwiGLU) {
             const int gate = e * args.b_rows + nt * HALF;
             const int up = e * args.b_rows + args.I + nt * HALF;
             if (rank == 0) {
@@ -252,7 +279,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
   } else if (warp == 1) {
     if (leader && lane == 0) {
       // ---------------------------------------------------------- MMA (leader)
-      constexpr uint32_t kIdesc = idesc_bf16_f32(256, C::NMMA, false, false);
+      constexpr uint32_t kIdesc = idesc_bf16_f32(256, C::NMMA, false, kBMN);
       constexpr uint32_t kIdescUp = idesc_bf16_f32(256, BN, false, false);
       constexpr uint16_t kBoth = 0x3;
       auto issue_up = [&](int b) {
@@ -267,8 +294,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         umma_commit_pair_mc(&acc_full[b], kBoth);
       };
       const uint64_t a_desc0 = smem_desc(smem_u32(sStage), 16, 1024, kLayoutSW128);
-      const uint64_t b_desc0 = smem_desc(smem_u32(sStage) + C::A_BYTES, 16, 1024, kLayoutSW128);
+      // MN-major: LBO = next 32-column atom, SBO = next 8 K-rows (8 x 64 B)
+      const uint64_t b_desc0 =
+          kBMN ? smem_desc(smem_u32(sStage) + C::A_BYTES, C::MN_BOX, 512, kLayoutSW64)
+               : smem_desc(smem_u32(sStage) + C::A_BYTES, 16, 1024, kLayoutSW128);
       constexpr uint64_t kStageInc = C::STAGE_BYTES >> 4;
+      constexpr uint64_t kBStep = kBMN ? (1024 >> 4) : (32 >> 4);  // 16 K
       int stage = 0;
       uint64_t soff = 0;
       uint32_t phase = 0;
@@ -291,7 +322,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           umma_bf16_pair(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 1; kk < C::BK / 16; ++kk)
-            umma_bf16_pair(t_acc, da + 2 * kk, db + 2 * kk, kIdesc, 1u);
+            umma_bf16_pair(t_acc, da + 2 * kk, db + kk * kBStep, kIdesc, 1u);
           umma_commit_pair_mc(&empty[stage], kBoth);
           soff += kStageInc;
           if (++stage == C::NS) {
@@ -339,7 +370,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp & 3;
+    const int ew = warp & 3;              // TMEM lane quarter
+    constexpr bool kSplit = C::EPI_WARPS == 8;
+    const int ehalf = (warp - 2) >> 2;    // which share of the columns
     const int row_in_tile = ew * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(ew * 32) << 16;
     int local = 0;
@@ -351,17 +384,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       const int grow = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * C::BM + row_in_tile;
       const bool rvalid = grow < s_off[e + 1];
       const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
-      if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
-      tc_fence_after();
-      epi_rank_handoff<RK>(args, t_acc + BN, sXA + b * C::XA_BYTES, row_in_tile, nt, rvalid,
-                           grow);
-      fence_proxy_async_all();  // the leader's MMA reads this tile
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead(&xa_ready[b]));
+      if (ehalf == 0) {  // rank-r hand-off: the first four epilogue warps
+        if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
+        tc_fence_after();
+        epi_rank_handoff<RK>(args, t_acc + BN, sXA + b * C::XA_BYTES, row_in_tile, nt,
+                             rvalid, grow);
+        fence_proxy_async_all();  // the leader's MMA reads this tile
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead(&xa_ready[b]));
+      }
+      if constexpr (MODE == kDownBwd) epi_prefetch_saved<BN>(args, grow, rvalid, nt, ehalf);
       if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
       tc_fence_after();
-      epi_drain<MODE, BN, false>(args, t_acc, grow, rvalid, nt, 0);
+      epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead(&acc_empty[b]));

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -54,16 +55,23 @@ moe_status_t route_scratch_on_current_device(void** out) {
 }
 
 uint64_t g_wait_limit_ns = 1000000000ull;  // one second per bounded wait
+std::atomic<unsigned long long> g_launches{0};  // kernels launched by the library
+inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 int g_stall_test = 0;                      // testing hook, see moe_test_inject_stall
-int g_forward_pairs = -1;                  // forward GEMMs on CTA pairs: <0 auto
-// Automatic choice: CTA pairs when the mean rows per expert fill at least
-// three 256-row tiles (little padding on each expert's ragged last tile) and
-// K is long enough (16 k-steps) for the per-tile hand-offs to stay hidden.
+int g_cta_pairs = -1;                      // grouped GEMMs on CTA pairs: <0 auto
+// Automatic choice (measured): the forward GEMMs run on CTA pairs when the
+// mean rows per expert fill at least three 256-row tiles (little padding on
+// each expert's ragged last tile) and K is long enough (16 k-steps) for the
+// per-tile hand-offs to stay hidden.  The backward GEMMs stay on single CTAs:
+// their MN-major weight operand needs 32-column atoms in the pair kernel,
+// which pads the fused factor columns, and with the 256-row padding that
+// costs more than the pair saves.
 constexpr int kPairMinRowsPerExpert = 768;
 constexpr int kPairMinK = 1024;
-bool use_pairs(int R, int E, int K) {
-  if (g_forward_pairs >= 0) return g_forward_pairs > 0;
-  return static_cast<int64_t>(R) >= static_cast<int64_t>(kPairMinRowsPerExpert) * E &&
+bool use_pairs(int R, int E, int K, bool backward) {
+  if (g_cta_pairs >= 0) return g_cta_pairs > 0;
+  return !backward &&
+         static_cast<int64_t>(R) >= static_cast<int64_t>(kPairMinRowsPerExpert) * E &&
          K >= kPairMinK;
 }
 
@@ -203,6 +211,7 @@ moe_status_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b,
                  : MODE == kDownFwd ? MOE_PROF_DOWN_FWD
                  : MODE == kDownBwd ? MOE_PROF_DOWN_BWD : MOE_PROF_GATE_UP_BWD, st);
   kern<<<grid, gemm_threads(MODE), C::SMEM_BYTES, st>>>(a, b, la, lb, args);
+  count_launch();
   return launch_status();
 }
 
@@ -236,11 +245,26 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* LA, const v
   const uint64_t EU = static_cast<uint64_t>(args.E);
   CUtensorMap ta, tw0, tw1, tw2, tla, tlb;
   bool ok = tmap_2d(&ta, A, K, args.R, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok = ok && tmap_2d(&tw0, W, K, EU * args.b_rows, K * 2, 64, Bx::seg0, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok = ok && tmap_2d(&tw1, W, K, EU * args.b_rows, K * 2, 64, Bx::seg1 > 0 ? Bx::seg1 : 8,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-  ok = ok && tmap_2d(&tw2, W, K, EU * args.b_rows, K * 2, 64, Bx::seg2, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok = ok && tmap_2d(&tla, LA, K, EU * RK, K * 2, 64, RK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if constexpr (C::kBMN) {
+    // W [E * K, N] in place and the down-projection factor [E * K, FPAD]
+    // (zero-padded copy when r < FPAD), 32-column x 64-row boxes (64-byte
+    // swizzle)
+    const uint64_t N = static_cast<uint64_t>(args.N);
+    ok = ok && tmap_2d(&tw0, W, N, EU * args.b_rows, N * 2, C::MN_COLS, 64,
+                       CU_TENSOR_MAP_SWIZZLE_64B);
+    ok = ok && tmap_2d(&tla, LA, C::FPAD, EU * args.b_rows, C::FPAD * 2ull, C::MN_COLS, 64,
+                       CU_TENSOR_MAP_SWIZZLE_64B);
+    tw1 = tw0;
+    tw2 = tw0;
+  } else {
+    ok = ok && tmap_2d(&tw0, W, K, EU * args.b_rows, K * 2, 64, Bx::seg0,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tw1, W, K, EU * args.b_rows, K * 2, 64, Bx::seg1 > 0 ? Bx::seg1 : 8,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tw2, W, K, EU * args.b_rows, K * 2, 64, Bx::seg2,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, LA, K, EU * RK, K * 2, 64, RK, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
   ok = ok && tmap_2d(&tlb, LB, RK, EU * args.lb_rows, RK * 2ull, RK, C::HALF, lora_swizzle(RK));
   if (!ok) return MOE_ERR_CUDA;
   auto kern = grouped_lora_gemm_pair_kernel<MODE, BN, RK>;
@@ -251,17 +275,29 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* LA, const v
       (static_cast<long long>(args.R) / 256 + args.E) * args.n_tiles;
   const int pairs = static_cast<int>(std::min<long long>(num_sms() / 2, max_pairs));
   if (pairs <= 0) return MOE_ERR_CUDA;
-  ProfScope prof(MODE == kGateUpFwd ? MOE_PROF_GATE_UP_FWD : MOE_PROF_DOWN_FWD, st);
+  ProfScope prof(MODE == kGateUpFwd   ? MOE_PROF_GATE_UP_FWD
+                 : MODE == kDownFwd   ? MOE_PROF_DOWN_FWD
+                 : MODE == kDownBwd   ? MOE_PROF_DOWN_BWD
+                                      : MOE_PROF_GATE_UP_BWD,
+                 st);
   kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tw0, tw1, tw2, tla, tlb, args);
+  count_launch();
   return launch_status();
+}
+
+// Tile width of the CTA-pair kernels: N = BN + r fills the 256-column MMA
+// (forward, K-major factor rows); backward: BN + round_up(r, 32) = 256.
+constexpr bool pair_backward(int mode) { return mode == kDownBwd || mode == kGateUpBwd; }
+constexpr int pair_bn(int mode, int r) {
+  return 256 - (pair_backward(mode) ? (r + 31) / 32 * 32 : r);
 }
 
 template <int MODE>
 moe_status_t launch_pair(int r, const void* A, const void* W, const void* LA,
                          const void* LB, const GemmArgs& args, cudaStream_t st) {
-  if (r == 16) return launch_pair_t<MODE, 240, 16>(A, W, LA, LB, args, st);
-  if (r == 32) return launch_pair_t<MODE, 224, 32>(A, W, LA, LB, args, st);
-  if (r == 64) return launch_pair_t<MODE, 192, 64>(A, W, LA, LB, args, st);
+  if (r == 16) return launch_pair_t<MODE, pair_bn(MODE, 16), 16>(A, W, LA, LB, args, st);
+  if (r == 32) return launch_pair_t<MODE, pair_bn(MODE, 32), 32>(A, W, LA, LB, args, st);
+  if (r == 64) return launch_pair_t<MODE, pair_bn(MODE, 64), 64>(A, W, LA, LB, args, st);
   return MOE_ERR_UNSUPPORTED;
 }
 
@@ -278,6 +314,7 @@ moe_status_t launch_grad_t(const CUtensorMap* u, const CUtensorMap* v,
   ProfScope prof(MOE_PROF_LORA_GRAD, st);
   kern<<<grid, 192, C::SMEM_BYTES, st>>>(u[0], u[1], u[2], u[3], v[0], v[1], v[2],
                                          v[3], args);
+  count_launch();
   return launch_status();
 }
 
@@ -301,9 +338,9 @@ void bwd_layout(int R, int E, int H, int I, int r, size_t off[8]) {
   off[0] = 0;                                                  // dZ1 [R, 2I]
   off[1] = off[0] + align256(dz1);                             // dZB2t [r, ldR]
   off[2] = off[1] + align256(vt);                              // dZB1t [r, ldR]
-  off[3] = off[2] + align256(vt);                              // B2p [E*H, 64]
+  off[3] = off[2] + align256(vt);                              // B2p [E*H, <= 64]
   off[4] = off[3] + align256(static_cast<size_t>(E) * H * 64 * 2);     // A2t [E, I, r]
-  off[5] = off[4] + align256(static_cast<size_t>(E) * I * r * 2);      // B1p [E*2I, 64]
+  off[5] = off[4] + align256(static_cast<size_t>(E) * I * r * 2);      // B1p [E*2I, <= 64]
   off[6] = off[5] + align256(static_cast<size_t>(E) * 2 * I * 64 * 2);  // A1t [E, H, r]
   off[7] = off[6] + align256(static_cast<size_t>(E) * H * r * 2);
 }
@@ -329,12 +366,14 @@ moe_status_t zero_rank_padding(void* p, int R, int r, cudaStream_t st) {
 
 // out [rows, 64] = in [rows, r] followed by zero columns (one MN-major
 // 64-column atom per K-slice for the backward's fused rank-r operand).
-moe_status_t pad_cols64(const void* in, void* out, long long rows, int r, cudaStream_t st) {
-  const long long n = rows * 8;  // 16-byte chunks of the output
+moe_status_t pad_cols(const void* in, void* out, long long rows, int r, int width,
+                      cudaStream_t st) {
+  const long long n = rows * (width / 8);  // 16-byte chunks of the output
   const int grid = static_cast<int>(std::min<long long>((n + 255) / 256, 148ll * 16));
   ProfScope prof(MOE_PROF_TRANSPOSE, st);
-  pad_cols64_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in),
-                                          static_cast<__nv_bfloat16*>(out), rows, r);
+  pad_cols_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in),
+                                        static_cast<__nv_bfloat16*>(out), rows, r, width);
+  count_launch();
   return launch_status();
 }
 
@@ -343,6 +382,7 @@ moe_status_t transpose(const void* in, void* out, int nb, int P, int Q, cudaStre
   ProfScope prof(MOE_PROF_TRANSPOSE, st);
   transpose_kernel<<<grid, dim3(32, 8), 0, st>>>(static_cast<const __nv_bfloat16*>(in),
                                                  static_cast<__nv_bfloat16*>(out), P, Q);
+  count_launch();
   return launch_status();
 }
 
@@ -368,7 +408,11 @@ void moe_set_wait_limit_ns(uint64_t ns) {
 
 void moe_test_inject_stall(int on) { g_stall_test = on ? 1 : 0; }
 
-void moe_set_forward_pairs(int mode) { g_forward_pairs = mode > 0 ? 1 : (mode == 0 ? 0 : -1); }
+unsigned long long moe_kernel_launches(void) {
+  return g_launches.load(std::memory_order_relaxed);
+}
+
+void moe_set_cta_pairs(int mode) { g_cta_pairs = mode > 0 ? 1 : (mode == 0 ? 0 : -1); }
 
 moe_status_t moe_profile_enable(int on) {
   if (on && !g_prof_created) {
@@ -454,6 +498,7 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
                              static_cast<int>(smem1)) != cudaSuccess)
       return MOE_ERR_CUDA;
     kern<<<grid1, kRouteWarps * 32, smem1, st>>>(logits, T, E, k, topk_idx, topk_w);
+    count_launch();
     return launch_status();
   };
   moe_status_t s;
@@ -466,16 +511,19 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
   // 2. stable in-chunk ranks + chunk histograms
   route_rank_kernel<<<nblk, kRankWarps * 32, static_cast<size_t>(kRankWarps) * E * 4, st>>>(
       topk_idx, R, E, blk_hist, local_rank);
+  count_launch();
   if ((s = launch_status()) != MOE_OK) return s;
   // 3. expert totals, offsets and per-chunk base rows (one CTA)
   const int P = std::max(1, 1024 / E);
   const size_t smem2 = (static_cast<size_t>(P) * E + E + 1) * 4;
   route_scan_kernel<<<1, 1024, smem2, st>>>(blk_hist, nblk, E, R, expert_counts,
                                             expert_offsets);
+  count_launch();
   if ((s = launch_status()) != MOE_OK) return s;
   // 4. destination rows
   const int grid = std::min((R + 255) / 256, std::max(1, num_sms()) * 8);
   route_dest_kernel<<<grid, 256, 0, st>>>(topk_idx, blk_hist, local_rank, R, E, dest);
+  count_launch();
   return launch_status();
 }
 
@@ -520,6 +568,7 @@ moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
     permute_kernel<<<grid, warps * 32, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
         static_cast<__nv_bfloat16*>(Xp), static_cast<const __nv_bfloat16*>(Zp), dw);
+  count_launch();
   return launch_status();
 }
 
@@ -537,6 +586,7 @@ moe_status_t moe_unpermute(const void* Yp, const int32_t* dest, const float* w, 
   unpermute_kernel<<<grid, warps * 32, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(Yp), dest, w, T, H, k,
       static_cast<__nv_bfloat16*>(Y));
+  count_launch();
   return launch_status();
 }
 
@@ -590,8 +640,8 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
   const uint64_t EU = static_cast<uint64_t>(E);
 
   // gate_up + SwiGLU
-  if (use_pairs(R, E, H)) {
-    const int bn = 256 - r, half = bn / 2;
+  if (use_pairs(R, E, H, false)) {
+    const int bn = pair_bn(kGateUpFwd, r), half = bn / 2;
     GemmArgs g{};
     g.offsets = expert_offsets;
     g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + half - 1) / half; g.I = I;
@@ -618,8 +668,8 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     if ((stt = launch_gemm<kGateUpFwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   // down
-  if (use_pairs(R, E, I)) {
-    const int bn = 256 - r;
+  if (use_pairs(R, E, I, false)) {
+    const int bn = pair_bn(kDownFwd, r);
     GemmArgs g{};
     g.offsets = expert_offsets;
     g.E = E; g.R = R; g.K = I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
@@ -683,21 +733,29 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
   __nv_bfloat16* dZ1 = at<__nv_bfloat16>(ws, wo[0]);
   __nv_bfloat16* dzb2 = at<__nv_bfloat16>(ws, wo[1]);
   __nv_bfloat16* dzb1 = at<__nv_bfloat16>(ws, wo[2]);
-  const void* B2p = B2;  // [E*H, 64]: B2 itself when r = 64, else a padded copy
-  const void* B1p = B1;  // [E*2I, 64]
+  const void* B2p = B2;  // [E*H, 64 or 32]: B2 itself when r fills the width
+  const void* B1p = B1;  // [E*2I, 64 or 32]
   __nv_bfloat16* A2t = at<__nv_bfloat16>(ws, wo[4]);
   __nv_bfloat16* A1t = at<__nv_bfloat16>(ws, wo[6]);
   moe_status_t stt;
   if ((stt = zero_rank_padding(dzb2, R, r, st)) != MOE_OK) return stt;
   if ((stt = zero_rank_padding(dzb1, R, r, st)) != MOE_OK) return stt;
-  // Operand copies of the LoRA factors: the down-projection factors B2, B1 as
-  // 64-column MN-major atoms (fused into the base MMA), the up-projection
-  // factors A2, A1 transposed to K-major.
-  if (r < 64) {
+  // Operand copies of the LoRA factors: the down-projection factors B2, B1
+  // zero-padded to whole MN-major atoms (64 columns for the single-CTA
+  // kernels, 32 for the CTA-pair kernels; fused into the base MMA), the
+  // up-projection factors A2, A1 transposed to K-major (both kernels).
+  const bool pair_down = use_pairs(R, E, H, true);
+  const bool pair_gate_up = use_pairs(R, E, 2 * I, true);
+  const int wdown = pair_down ? 32 : 64, wgate = pair_gate_up ? 32 : 64;
+  if (r < wdown) {
     B2p = at<__nv_bfloat16>(ws, wo[3]);
+    if ((stt = pad_cols(B2, const_cast<void*>(B2p), 1ll * E * H, r, wdown, st)) != MOE_OK)
+      return stt;
+  }
+  if (r < wgate) {
     B1p = at<__nv_bfloat16>(ws, wo[5]);
-    if ((stt = pad_cols64(B2, const_cast<void*>(B2p), 1ll * E * H, r, st)) != MOE_OK) return stt;
-    if ((stt = pad_cols64(B1, const_cast<void*>(B1p), 2ll * E * I, r, st)) != MOE_OK) return stt;
+    if ((stt = pad_cols(B1, const_cast<void*>(B1p), 2ll * E * I, r, wgate, st)) != MOE_OK)
+      return stt;
   }
   if ((stt = transpose(A2, A2t, E, r, I, st)) != MOE_OK) return stt;
   if ((stt = transpose(A1, A1t, E, r, H, st)) != MOE_OK) return stt;
@@ -705,7 +763,17 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
   const uint64_t EU = static_cast<uint64_t>(E);
 
   // down backward: dh = dZ2 W2 + s (dZ2 B2) A2, SwiGLU backward -> dZ1
-  {
+  if (pair_down) {
+    const int bn = pair_bn(kDownBwd, r);
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + bn - 1) / bn; g.I = I;
+    g.b_rows = H; g.lb_rows = I; g.s = s;
+    g.out = dZ1; g.ld_out = 2 * I; g.aux = Z1; g.ld_aux = 2 * I;
+    g.lora_t = dzb2; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
+    if ((stt = launch_pair<kDownBwd>(r, dZ2, W2, B2p, A2t, g, st)) != MOE_OK) return stt;
+  } else {
     const int bn = pick_bn(I, false, r, true);
     CUtensorMap ta, tb, tla, tlb;
     bool ok = tmap_2d(&ta, dZ2, H, R, H * 2ull, kGemmBK, 128, kKmajSwz);
@@ -723,7 +791,17 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
     if ((stt = launch_gemm<kDownBwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   // gate_up backward: dXp = dZ1 W1 + s (dZ1 B1) A1
-  {
+  if (pair_gate_up) {
+    const int bn = pair_bn(kGateUpBwd, r);
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
+    g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
+    g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
+    g.lora_t = dzb1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
+    if ((stt = launch_pair<kGateUpBwd>(r, dZ1, W1, B1p, A1t, g, st)) != MOE_OK) return stt;
+  } else {
     const int bn = pick_bn(H, false, r, true);
     CUtensorMap ta, tb, tla, tlb;
     bool ok = tmap_2d(&ta, dZ1, 2 * I, R, 4ull * I, kGemmBK, 128, kKmajSwz);

@@ -225,18 +225,20 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// out[row][0:64] = (in[row][0:r], zeros) for bf16 rows (LoRA factors only).
-__global__ void pad_cols64_kernel(const __nv_bfloat16* __restrict__ in,
-                                  __nv_bfloat16* __restrict__ out, long long rows,
-                                  int r) {
-  const long long n = rows * 8;
+// out[row][0:width] = (in[row][0:r], zeros) for bf16 rows (LoRA factors
+// only; width a multiple of 8 and >= r).
+__global__ void pad_cols_kernel(const __nv_bfloat16* __restrict__ in,
+                                __nv_bfloat16* __restrict__ out, long long rows, int r,
+                                int width) {
+  const int chunks = width / 8;  // 16-byte chunks per output row
+  const long long n = rows * chunks;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
        i < n; i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = i >> 3;
-    const int c8 = static_cast<int>(i & 7) * 8;  // first column of this chunk
+    const long long row = i / chunks;
+    const int c8 = static_cast<int>(i - row * chunks) * 8;  // first column of this chunk
     uint4 v = make_uint4(0, 0, 0, 0);
     if (c8 < r) v = *reinterpret_cast<const uint4*>(in + row * r + c8);
-    *reinterpret_cast<uint4*>(out + row * 64 + c8) = v;
+    *reinterpret_cast<uint4*>(out + row * width + c8) = v;
   }
 }
 

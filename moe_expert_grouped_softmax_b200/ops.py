@@ -25,7 +25,7 @@ EXPORTS = [
     "moe_saved_bytes", "moe_saved_part_offset", "moe_workspace_bytes",
     "moe_lora_mlp_fwd", "moe_lora_mlp_bwd", "moe_get_device_status",
     "moe_status_string", "moe_set_wait_limit_ns", "moe_test_inject_stall",
-    "moe_set_forward_pairs", "moe_profile_enable",
+    "moe_set_cta_pairs", "moe_kernel_launches", "moe_profile_enable",
     "moe_profile_collect",
 ]
 
@@ -77,8 +77,10 @@ def lib():
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_set_wait_limit_ns.argtypes = [U64]
         L.moe_set_wait_limit_ns.restype = None
-        L.moe_set_forward_pairs.argtypes = [I]
-        L.moe_set_forward_pairs.restype = None
+        L.moe_set_cta_pairs.argtypes = [I]
+        L.moe_set_cta_pairs.restype = None
+        L.moe_kernel_launches.argtypes = []
+        L.moe_kernel_launches.restype = ctypes.c_ulonglong
         L.moe_test_inject_stall.argtypes = [I]
         L.moe_test_inject_stall.restype = None
         L.moe_profile_enable.argtypes = [I]
@@ -122,10 +124,15 @@ def set_wait_limit_ns(ns):
     lib().moe_set_wait_limit_ns(int(ns))
 
 
-def set_forward_pairs(on=True):
-    """Forward GEMMs on CTA pairs (True, 256-row tiles), single CTAs (False)
-    or chosen per call from the mean rows per expert (None, the default)."""
-    lib().moe_set_forward_pairs(-1 if on is None else (1 if on else 0))
+def kernel_launches():
+    """Kernels this library has launched in this process (host-side count)."""
+    return int(lib().moe_kernel_launches())
+
+
+def set_cta_pairs(on=True):
+    """Grouped GEMMs on CTA pairs (True, 256-row tiles), single CTAs (False)
+    or chosen per GEMM from the rows per expert and K (None, the default)."""
+    lib().moe_set_cta_pairs(-1 if on is None else (1 if on else 0))
 
 
 def test_inject_stall(on=True):
@@ -302,10 +309,6 @@ class MoeBlock:
     end-to-end tests).  ``step`` runs, on the current stream: route, permute,
     gate_up + SwiGLU, down, weighted unpermute, weighted dY gather, down /
     gate_up backward, LoRA gradients and the dX combine."""
-
-    KERNELS_PER_STEP = 18  # 4 route + 1 permute + 2 fwd + 1 combine +
-    #                        1 gather + 4 factor copies + 2 bwd GEMMs + 1 grads
-    #                        + 1 dX combine
 
     def __init__(self, T, H, I, E, k, r, s, device="cuda", with_dw=False):
         self.T, self.H, self.I, self.E, self.k, self.r, self.s = T, H, I, E, k, r, s

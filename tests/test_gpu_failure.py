@@ -1,7 +1,8 @@
 """Device-side failure detection without faulting the GPU.
 
 * Every wait in the pipelined kernels is bounded.  With the stall hook on,
-  each grouped-GEMM kernel waits on a barrier that nothing arrives on; after
+  each grouped-GEMM kernel (single-CTA or CTA-pair) waits on a barrier that
+  nothing arrives on; after
   the (shortened) limit it records MOE_ERR_DEVICE_TIMEOUT, drains its own
   copies and MMAs, frees its tensor memory and returns.  The context must stay
   usable: the next run without the hook is correct.
@@ -33,12 +34,14 @@ def _setup():
     return cfg, inp, g, blk
 
 
-def test_wait_timeout_is_reported_and_context_survives(cuda_ok):
+@pytest.mark.parametrize("pairs", [False, True], ids=["single", "pairs"])
+def test_wait_timeout_is_reported_and_context_survives(cuda_ok, pairs):
     cfg, inp, g, blk = _setup()
     W = [g[n] for n in NAMES]
     assert ops.device_status() == 0
     ops.set_wait_limit_ns(2_000_000)  # 2 ms
     ops.test_inject_stall(True)
+    ops.set_cta_pairs(pairs)
     try:
         blk.step(g["X"], g["logits"], g["dY"], W)
         torch.cuda.synchronize()
@@ -46,6 +49,7 @@ def test_wait_timeout_is_reported_and_context_survives(cuda_ok):
     finally:
         ops.test_inject_stall(False)
         ops.set_wait_limit_ns(0)
+        ops.set_cta_pairs(None)
     assert st == 4, ops.STATUS_NAMES.get(st, st)
     # same process, same context: a normal run is correct
     blk.step(g["X"], g["logits"], g["dY"], W)

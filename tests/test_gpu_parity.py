@@ -125,11 +125,10 @@ BLOCK_CASES = {
 }
 
 
-# every case forced onto the single-CTA forward kernels; the cases marked
-# "/pairs" again forced onto the CTA-pair forward kernels (the default
-# chooses between them from the mean rows per expert)
-BLOCK_RUNS = [(c, False) for c in BLOCK_CASES] + [
-    (c, True) for c in ("tiny", "ragged", "rank32", "rank64", "skew_empty")]
+# every case forced onto the single-CTA GEMM kernels, and again ("/pairs")
+# onto the CTA-pair GEMM kernels (the default chooses between them per GEMM
+# from the rows per expert and K)
+BLOCK_RUNS = [(c, False) for c in BLOCK_CASES] + [(c, True) for c in BLOCK_CASES]
 
 
 @pytest.fixture(scope="module", params=BLOCK_RUNS,
@@ -143,12 +142,12 @@ def block_run(request, cuda_ok):
     blk = ops.MoeBlock(cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"], cfg["r"], cfg["s"],
                        with_dw=True)
     W = _weights(g)
-    ops.set_forward_pairs(pairs)
+    ops.set_cta_pairs(pairs)
     try:
         blk.step(g["X"], g["logits"], g["dY"], W)
         torch.cuda.synchronize()
     finally:
-        ops.set_forward_pairs(None)
+        ops.set_cta_pairs(None)
     status = ops.device_status()
     return dict(name=name, pairs=pairs, cfg=cfg, inp=inp, Y=Y, ctx=ctx, grads=grads,
                 blk=blk, status=status)
@@ -212,10 +211,10 @@ def test_block_deterministic(block_run):
     g = _cuda(block_run["inp"])
     W = _weights(g)
     first = [t.clone() for t in (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2)]
-    ops.set_forward_pairs(block_run["pairs"])
+    ops.set_cta_pairs(block_run["pairs"])
     try:
         b.step(g["X"], g["logits"], g["dY"], W)
     finally:
-        ops.set_forward_pairs(None)
+        ops.set_cta_pairs(None)
     for x, y in zip(first, (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2)):
         assert torch.equal(x, y)
