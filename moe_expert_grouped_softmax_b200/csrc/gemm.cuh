@@ -175,6 +175,19 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// warp_wait for a barrier that other CTAs of the cluster arrive on.
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag,
+                                                  uint64_t limit_ns) {
+  const bool ok = mbar_wait_cluster(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Lane 0's view of a non-blocking barrier test, for the whole warp.
+__device__ __forceinline__ bool warp_uniform(bool v) {
+  return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0;
+}
+
 // Bounded wait that ignores the abort flag, used before exit to let copies
 // and MMAs already in flight land.  Its limit never drops below one second,
 // whatever the configured wait limit, so that a CTA does not leave while its
@@ -255,16 +268,18 @@ __device__ unsigned long long g_gemm_trace[4][160][kTraceSlots];
   ([&]() {                                                                    \
     const long long _t = clock64();                                           \
     auto _r = (expr);                                                         \
-    atomicAdd(&g_gemm_trace[mode][blockIdx.x % 160][slot],                    \
-              static_cast<unsigned long long>(clock64() - _t));               \
+    if ((threadIdx.x & 31) == 0)                                              \
+      atomicAdd(&g_gemm_trace[mode][blockIdx.x % 160][slot],                  \
+                static_cast<unsigned long long>(clock64() - _t));             \
     return _r;                                                                \
   }())
 #define MOE_TIMED_VOID(mode, slot, stmt)                                      \
   do {                                                                        \
     const long long _t = clock64();                                           \
     stmt;                                                                     \
-    atomicAdd(&g_gemm_trace[mode][blockIdx.x % 160][slot],                    \
-              static_cast<unsigned long long>(clock64() - _t));               \
+    if ((threadIdx.x & 31) == 0)                                              \
+      atomicAdd(&g_gemm_trace[mode][blockIdx.x % 160][slot],                  \
+                static_cast<unsigned long long>(clock64() - _t));             \
   } while (0)
 #else
 #define MOE_TIMED(mode, slot, expr) (expr)
@@ -580,7 +595,9 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (its state stays warp-uniform); one
+    // elected lane issues the tensor-core instructions.
+    {
       constexpr uint32_t kIdesc = idesc_bf16_f32(128, C::NMMA, false, kBMN);
       constexpr uint32_t kIdescUp = idesc_bf16_f32(128, BN, false, false);
       // acc[b] += xa[b] * LB[b]^T, then release LB[b] and publish acc[b]
@@ -594,6 +611,11 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
                     smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), kIdescUp, 1u);
         umma_commit(&lb_empty[b]);
         umma_commit(&acc_full[b]);
+      };
+      auto up_when_ready = [&](int pb) {
+        tc_fence_after();
+        if (elect_one()) issue_up(pb);
+        __syncwarp();
       };
       // Stage-0 operand descriptors; a stage / K-step moves only the 14-bit
       // start-address field (shared addresses are < 256 KB, so adding the
@@ -614,7 +636,7 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
       // Testing hook: wait on a barrier that nothing arrives on before the
       // end of the kernel, so the bounded wait runs out and the whole CTA
       // takes its abort path.
-      if (args.stall_test) ok = mbar_wait(drain_bar, 0, s_abort, wait_ns);
+      if (args.stall_test) ok = warp_wait(drain_bar, 0, s_abort, wait_ns);
 #ifdef MOE_GEMM_TRACE
       const long long t_role = clock64();
 #endif
@@ -622,17 +644,20 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
-        if (!MOE_TIMED(MODE, 1, mbar_wait(&acc_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
+        if (!MOE_TIMED(MODE, 1, warp_wait(&acc_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < k_iters; ++kt) {
           // (TMA -> MMA ordering comes with the barrier; no tcgen05 fence)
-          if (!MOE_TIMED(MODE, 0, mbar_wait(&full[stage], phase, s_abort, wait_ns))) { ok = false; break; }
+          if (!MOE_TIMED(MODE, 0, warp_wait(&full[stage], phase, s_abort, wait_ns))) { ok = false; break; }
           const uint64_t da = a_desc0 + soff, db = b_desc0 + soff;
-          umma_bf16(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
+          if (elect_one()) {
+            umma_bf16(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 1; kk < C::BK / 16; ++kk)
-            umma_bf16(t_acc, da + kk * kAStep, db + kk * kBStep, kIdesc, 1u);
-          umma_commit(&empty[stage]);
+            for (int kk = 1; kk < C::BK / 16; ++kk)
+              umma_bf16(t_acc, da + kk * kAStep, db + kk * kBStep, kIdesc, 1u);
+            umma_commit(&empty[stage]);
+          }
+          __syncwarp();
           soff += kStageInc;
           if (++stage == C::NS) {
             stage = 0;
@@ -642,40 +667,40 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
           if (pending >= 0) {  // previous tile's up-projection, once it is ready
             const int pb = pending & 1;
             const uint32_t pu = (pending >> 1) & 1;
-            if (mbar_test_wait(&xa_ready[pb], pu) && mbar_test_wait(&lb_full[pb], pu)) {
-              tc_fence_after();
-              issue_up(pb);
+            if (warp_uniform(mbar_test_wait(&xa_ready[pb], pu) &&
+                             mbar_test_wait(&lb_full[pb], pu))) {
+              up_when_ready(pb);
               pending = -1;
             }
           }
         }
         if (!ok) break;
-        umma_commit(&lora_full[b]);
+        if (elect_one()) umma_commit(&lora_full[b]);
+        __syncwarp();
         if (pending >= 0) {
           const int pb = pending & 1;
           const uint32_t pu = (pending >> 1) & 1;
-          if (!MOE_TIMED(MODE, 2, mbar_wait(&xa_ready[pb], pu, s_abort, wait_ns)) ||
-              !MOE_TIMED(MODE, 3, mbar_wait(&lb_full[pb], pu, s_abort, wait_ns))) { ok = false; break; }
-          tc_fence_after();
-          issue_up(pb);
+          if (!MOE_TIMED(MODE, 2, warp_wait(&xa_ready[pb], pu, s_abort, wait_ns)) ||
+              !MOE_TIMED(MODE, 3, warp_wait(&lb_full[pb], pu, s_abort, wait_ns))) { ok = false; break; }
+          up_when_ready(pb);
         }
         pending = local;
       }
       if (ok && pending >= 0) {
         const int pb = pending & 1;
         const uint32_t pu = (pending >> 1) & 1;
-        if (mbar_wait(&xa_ready[pb], pu, s_abort, wait_ns) &&
-            mbar_wait(&lb_full[pb], pu, s_abort, wait_ns)) {
-          tc_fence_after();
-          issue_up(pb);
-        }
+        if (warp_wait(&xa_ready[pb], pu, s_abort, wait_ns) &&
+            warp_wait(&lb_full[pb], pu, s_abort, wait_ns))
+          up_when_ready(pb);
       }
 #ifdef MOE_GEMM_TRACE
-      atomicAdd(&g_gemm_trace[MODE][blockIdx.x % 160][7],
-                static_cast<unsigned long long>(clock64() - t_role));
+      if (lane == 0)
+        atomicAdd(&g_gemm_trace[MODE][blockIdx.x % 160][7],
+                  static_cast<unsigned long long>(clock64() - t_role));
 #endif
-      // every MMA issued by this thread must be complete before TMEM is freed
-      umma_commit(drain_bar);
+      // every MMA issued by this warp must be complete before TMEM is freed
+      if (elect_one()) umma_commit(drain_bar);
+      __syncwarp();
       drain_wait(drain_bar, 0, wait_ns);
     }
   } else {

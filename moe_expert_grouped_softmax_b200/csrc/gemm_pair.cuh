@@ -277,8 +277,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       s_issued[1] = n_lb;
     }
   } else if (warp == 1) {
-    if (leader && lane == 0) {
+    if (leader) {
       // ---------------------------------------------------------- MMA (leader)
+      // The whole warp runs the loop (its state stays warp-uniform); one
+      // elected lane issues the tensor-core instructions.
       constexpr uint32_t kIdesc = idesc_bf16_f32(256, C::NMMA, false, kBMN);
       constexpr uint32_t kIdescUp = idesc_bf16_f32(256, BN, false, false);
       constexpr uint16_t kBoth = 0x3;
@@ -293,6 +295,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         umma_commit_pair_mc(&lb_empty[b], kBoth);
         umma_commit_pair_mc(&acc_full[b], kBoth);
       };
+      auto up_when_ready = [&](int b) {
+        tc_fence_after();
+        if (elect_one()) issue_up(b);
+        __syncwarp();
+      };
       const uint64_t a_desc0 = smem_desc(smem_u32(sStage), 16, 1024, kLayoutSW128);
       // MN-major: LBO = next 32-column atom, SBO = next 8 K-rows (8 x 64 B)
       const uint64_t b_desc0 =
@@ -306,7 +313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       int local = 0;
       int pending = -1;
       bool ok = true;
-      if (args.stall_test) ok = mbar_wait(final_bar, 0, s_abort, wait_ns);
+      if (args.stall_test) ok = warp_wait(final_bar, 0, s_abort, wait_ns);
 #ifdef MOE_GEMM_TRACE
       const long long t_role = clock64();
 #endif
@@ -314,16 +321,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
-        if (!MOE_TIMED(MODE, 14, mbar_wait_cluster(&acc_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
+        if (!MOE_TIMED(MODE, 14, warp_wait_cluster(&acc_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < k_iters; ++kt) {
-          if (!MOE_TIMED(MODE, 11, mbar_wait(&full[stage], phase, s_abort, wait_ns))) { ok = false; break; }
+          if (!MOE_TIMED(MODE, 11, warp_wait(&full[stage], phase, s_abort, wait_ns))) { ok = false; break; }
           const uint64_t da = a_desc0 + soff, db = b_desc0 + soff;
-          umma_bf16_pair(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
+          if (elect_one()) {
+            umma_bf16_pair(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 1; kk < C::BK / 16; ++kk)
-            umma_bf16_pair(t_acc, da + 2 * kk, db + kk * kBStep, kIdesc, 1u);
-          umma_commit_pair_mc(&empty[stage], kBoth);
+            for (int kk = 1; kk < C::BK / 16; ++kk)
+              umma_bf16_pair(t_acc, da + 2 * kk, db + kk * kBStep, kIdesc, 1u);
+            umma_commit_pair_mc(&empty[stage], kBoth);
+          }
+          __syncwarp();
           soff += kStageInc;
           if (++stage == C::NS) {
             stage = 0;
@@ -333,40 +343,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           if (pending >= 0) {
             const int pb = pending & 1;
             const uint32_t pu = (pending >> 1) & 1;
-            if (mbar_test_wait_cluster(&xa_ready[pb], pu) && mbar_test_wait(&lb_full[pb], pu)) {
-              tc_fence_after();
-              issue_up(pb);
+            if (warp_uniform(mbar_test_wait_cluster(&xa_ready[pb], pu) &&
+                             mbar_test_wait(&lb_full[pb], pu))) {
+              up_when_ready(pb);
               pending = -1;
             }
           }
         }
         if (!ok) break;
-        umma_commit_pair_mc(&lora_full[b], kBoth);
+        if (elect_one()) umma_commit_pair_mc(&lora_full[b], kBoth);
+        __syncwarp();
         if (pending >= 0) {
           const int pb = pending & 1;
           const uint32_t pu = (pending >> 1) & 1;
-          if (!mbar_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) ||
-              !mbar_wait(&lb_full[pb], pu, s_abort, wait_ns)) { ok = false; break; }
-          tc_fence_after();
-          issue_up(pb);
+          if (!warp_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) ||
+              !warp_wait(&lb_full[pb], pu, s_abort, wait_ns)) { ok = false; break; }
+          up_when_ready(pb);
         }
         pending = local;
       }
       if (ok && pending >= 0) {
         const int pb = pending & 1;
         const uint32_t pu = (pending >> 1) & 1;
-        if (mbar_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) &&
-            mbar_wait(&lb_full[pb], pu, s_abort, wait_ns)) {
-          tc_fence_after();
-          issue_up(pb);
-        }
+        if (warp_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) &&
+            warp_wait(&lb_full[pb], pu, s_abort, wait_ns))
+          up_when_ready(pb);
       }
 #ifdef MOE_GEMM_TRACE
-      atomicAdd(&g_gemm_trace[MODE][blockIdx.x % 160][13],
-                static_cast<unsigned long long>(clock64() - t_role));
+      if (lane == 0)
+        atomicAdd(&g_gemm_trace[MODE][blockIdx.x % 160][13],
+                  static_cast<unsigned long long>(clock64() - t_role));
 #endif
       // all of the leader's MMAs complete -> both CTAs' final_bar
-      umma_commit_pair_mc(final_bar, kBoth);
+      if (elect_one()) umma_commit_pair_mc(final_bar, kBoth);
+      __syncwarp();
     }
   } else {
     // ------------------------------------------------------------ epilogue
