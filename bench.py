@@ -87,6 +87,24 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(x, dev):
+    """Max of the float x over all ranks of the default process group (every
+    rank calls it with its own x); x itself without a group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(T, steps, ws, ms_total):
+    """Whole-job throughput: every rank processes T tokens per step (weak
+    scaling); ms_total is the slowest rank's total time of the timed steps."""
+    return T * steps * ws / (ms_total / 1e3)
+
+
 class Clocks:
     """Samples SM clocks and throttle reasons with nvidia-smi (every 50 ms,
     into a file) and keeps the samples taken inside [t_begin, t_end]."""
@@ -226,10 +244,7 @@ def run_ours(args, cfg):
     st = ops.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after timed steps")
-    if ws > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
 
     # ---- end to end through the public API with host buffers: every step
     # copies its X, logits and dY from pinned host memory and reads back Y,
@@ -288,14 +303,10 @@ def run_ours(args, cfg):
         t1.record(s_in)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = float(t0.elapsed_time(t1))
-        if ws > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(float(t0.elapsed_time(t1)), dev)
         h2d = sum(h.numel() * h.element_size() for h in hin[0])
         d2h = sum(h.numel() * h.element_size() for h in hout[0])
-        e2e = {"value": T * K * ws / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": job_tokens_per_s(T, K, ws, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / K,
                "note": "pinned host buffers; copies on two streams overlap the "
@@ -405,7 +416,7 @@ def main():
         return
     K = args.steps
     ms_per_step = res["ms_total"] / K
-    tokens_s = T * K * res["ws"] / (res["ms_total"] / 1e3)
+    tokens_s = job_tokens_per_s(T, K, res["ws"], res["ms_total"])
     tflops = flops / (ms_per_step / 1e3) / 1e12
     # dominant kernel by measured share
     kern = res["kern"]
