@@ -291,6 +291,49 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
                     pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
 
+// Stores the bf16 roundings of v[0, W) to p[0, W) (a row segment of a
+// tile), skipping columns [nvalid, W) (nvalid a multiple of 8, may be <= 0).
+// Each thread writes its own row, so 32-byte stores where the address allows
+// (whole L2 sectors, half the transactions of 16-byte ones), else 16 bytes.
+template <int Q>
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float* v, int nvalid,
+                                       uint64_t pol) {
+  if (8 * Q < nvalid) st_global_v4_hint(p + 8 * Q, pack8(v + 8 * Q), pol);
+}
+template <int Q>
+__device__ __forceinline__ void store16(__nv_bfloat16* p, const float* v, int nvalid,
+                                        uint64_t pol) {
+  if (8 * Q + 16 <= nvalid)
+    st_global_v8_hint(p + 8 * Q, pack8(v + 8 * Q), pack8(v + 8 * Q + 8), pol);
+  else
+    store8<Q>(p, v, nvalid, pol);
+}
+template <int Q, int NQ>
+__device__ __forceinline__ void store_pairs(__nv_bfloat16* p, const float* v, int nvalid,
+                                            uint64_t pol) {
+  if constexpr (Q + 1 < NQ) {
+    store16<Q>(p, v, nvalid, pol);
+    store_pairs<Q + 2, NQ>(p, v, nvalid, pol);
+  } else if constexpr (Q < NQ) {
+    store8<Q>(p, v, nvalid, pol);
+  }
+}
+
+// Stores the bf16 roundings of v[0, W) to p[0, W) (a row segment of a
+// tile), skipping columns [nvalid, W) (nvalid a multiple of 8, may be <= 0).
+// Each thread writes its own row, so 32-byte stores where the address allows
+// (whole L2 sectors, half the transactions of 16-byte ones), else 16 bytes.
+template <int W>
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* p, const float* v, int nvalid,
+                                               uint64_t pol) {
+  if ((reinterpret_cast<uintptr_t>(p) & 31u) == 0) {
+    store_pairs<0, W / 8>(p, v, nvalid, pol);
+  } else {
+    store8<0>(p, v, nvalid, pol);
+    store_pairs<1, W / 8>(p, v, nvalid, pol);
+  }
+}
+
 // Epilogue step 1: the rank-r product (TMEM columns [BN, BN + r) of this
 // thread's row) times s, rounded to bf16, into the swizzled K-major shared
 // tile that feeds the up-projection; the first n-tile also saves it
@@ -353,21 +396,13 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
       tmem_ld<W>(t_acc + HALF + c, u);
       tmem_ld_wait();
       if (rvalid) {
+        float h[W];
 #pragma unroll
-        for (int q = 0; q < W / 8; ++q) {
-          const int col = col0 + c + 8 * q;
-          if (col < args.N) {
-            float h[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float gg = g[8 * q + i];
-              h[i] = gg * sigmoidf_(gg) * u[8 * q + i];
-            }
-            st_global_v4_hint(hrow + col, pack8(h), pol);
-            st_global_v4_hint(zrow + col, pack8(g + 8 * q), pol);
-            st_global_v4_hint(zrow + args.I + col, pack8(u + 8 * q), pol);
-          }
-        }
+        for (int i = 0; i < W; ++i) h[i] = g[i] * sigmoidf_(g[i]) * u[i];
+        const int col = col0 + c, nv = args.N - col;
+        store_row_bf16<W>(hrow + col, h, nv, pol);
+        store_row_bf16<W>(zrow + col, g, nv, pol);
+        store_row_bf16<W>(zrow + args.I + col, u, nv, pol);
       }
     });
   } else if constexpr (MODE == kDownBwd) {
@@ -380,6 +415,7 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
 #pragma unroll
       for (int q = 0; q < W / 8; ++q) {  // loads first: in flight during the TMEM read
         const int col = col0 + c + 8 * q;
+        gv[q] = uv[q] = make_uint4(0, 0, 0, 0);
         if (rvalid && col < args.N) {
           gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
           uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
@@ -389,29 +425,27 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
       tmem_ld<W>(t_acc + c, dh);
       tmem_ld_wait();
       if (rvalid) {
+        float dg[W], du[W];
 #pragma unroll
         for (int q = 0; q < W / 8; ++q) {
-          const int col = col0 + c + 8 * q;
-          if (col < args.N) {
-            const uint32_t ga[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
-            const uint32_t ua[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
-            float dg[8], du[8];
+          const uint32_t ga[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+          const uint32_t ua[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < 4; ++i) {
 #pragma unroll
-              for (int h2 = 0; h2 < 2; ++h2) {
-                const float gg = h2 ? bf16_hi(ga[i]) : bf16_lo(ga[i]);
-                const float uu = h2 ? bf16_hi(ua[i]) : bf16_lo(ua[i]);
-                const float d = dh[8 * q + 2 * i + h2];
-                const float sg = sigmoidf_(gg);
-                dg[2 * i + h2] = d * uu * sg * (1.f + gg * (1.f - sg));
-                du[2 * i + h2] = d * gg * sg;
-              }
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const float gg = h2 ? bf16_hi(ga[i]) : bf16_lo(ga[i]);
+              const float uu = h2 ? bf16_hi(ua[i]) : bf16_lo(ua[i]);
+              const int j = 8 * q + 2 * i + h2;
+              const float sg = sigmoidf_(gg);
+              dg[j] = dh[j] * uu * sg * (1.f + gg * (1.f - sg));
+              du[j] = dh[j] * gg * sg;
             }
-            st_global_v4_hint(orow + col, pack8(dg), pol);
-            st_global_v4_hint(orow + args.I + col, pack8(du), pol);
           }
         }
+        const int col = col0 + c, nv = args.N - col;
+        store_row_bf16<W>(orow + col, dg, nv, pol);
+        store_row_bf16<W>(orow + args.I + col, du, nv, pol);
       }
     });
   } else {
@@ -422,13 +456,7 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
       float v[W];
       tmem_ld<W>(t_acc + c, v);
       tmem_ld_wait();
-      if (rvalid) {
-#pragma unroll
-        for (int q = 0; q < W / 8; ++q) {
-          const int col = col0 + c + 8 * q;
-          if (col < args.N) st_global_v4_hint(orow + col, pack8(v + 8 * q), pol);
-        }
-      }
+      if (rvalid) store_row_bf16<W>(orow + c + col0, v, args.N - col0 - c, pol);
     });
   }
 }

@@ -263,6 +263,16 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// 32-byte global store (8 x 32 bits) with an L2 cache policy; p must be
+// 32-byte aligned.
+__device__ __forceinline__ void st_global_v8_hint(void* p, uint4 a, uint4 b, uint64_t policy) {
+  asm volatile(
+      "st.global.L2::cache_hint.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8}, %9;" ::"l"(p),
+      "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w),
+      "l"(policy)
+      : "memory");
+}
+
 // 16-byte global store with an L2 cache policy.
 __device__ __forceinline__ void st_global_v4_hint(void* p, uint4 v, uint64_t policy) {
   asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p),
