@@ -219,7 +219,8 @@ MOE_API void moe_set_cta_pairs(int mode);
  * moe_profile_enable(0) stops recording.  moe_profile_collect synchronises on
  * the recorded events and writes the durations (ms) of up to max_n launches
  * of `kind` into ms[], returning how many (or -1 on a CUDA error).  Route
- * covers its three kernels together. */
+ * covers its four kernels together; MOE_PROF_TRANSPOSE is the one launch
+ * that makes the backward's operand copies of the LoRA factors. */
 #define MOE_PROF_ROUTE 0
 #define MOE_PROF_PERMUTE 1
 #define MOE_PROF_GATE_UP_FWD 2

@@ -366,25 +366,40 @@ moe_status_t zero_rank_padding(void* p, int R, int r, cudaStream_t st) {
 
 // out [rows, 64] = in [rows, r] followed by zero columns (one MN-major
 // 64-column atom per K-slice for the backward's fused rank-r operand).
-moe_status_t pad_cols(const void* in, void* out, long long rows, int r, int width,
-                      cudaStream_t st) {
-  const long long n = rows * (width / 8);  // 16-byte chunks of the output
-  const int grid = static_cast<int>(std::min<long long>((n + 255) / 256, 148ll * 16));
-  ProfScope prof(MOE_PROF_TRANSPOSE, st);
-  pad_cols_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in),
-                                        static_cast<__nv_bfloat16*>(out), rows, r, width);
-  count_launch();
-  return launch_status();
-}
-
-moe_status_t transpose(const void* in, void* out, int nb, int P, int Q, cudaStream_t st) {
-  dim3 grid((Q + 31) / 32, (P + 31) / 32, nb);
-  ProfScope prof(MOE_PROF_TRANSPOSE, st);
-  transpose_kernel<<<grid, dim3(32, 8), 0, st>>>(static_cast<const __nv_bfloat16*>(in),
-                                                 static_cast<__nv_bfloat16*>(out), P, Q);
-  count_launch();
-  return launch_status();
-}
+// Jobs of factor_prep_kernel, launched together.
+struct FactorPrep {
+  FactorJobs jobs{};
+  int total = 0;
+  void pad(const void* in, void* out, long long rows, int r, int width) {
+    FactorJob& J = jobs.job[jobs.n++];
+    J.in = static_cast<const __nv_bfloat16*>(in);
+    J.out = static_cast<__nv_bfloat16*>(out);
+    J.kind = 0;
+    J.rows = rows;
+    J.r = r;
+    J.width = width;
+    J.blocks = static_cast<int>(std::min<long long>((rows * (width / 8) + 255) / 256, 148ll * 4));
+    total += J.blocks;
+  }
+  void transpose(const void* in, void* out, int nb, int P, int Q) {
+    FactorJob& J = jobs.job[jobs.n++];
+    J.in = static_cast<const __nv_bfloat16*>(in);
+    J.out = static_cast<__nv_bfloat16*>(out);
+    J.kind = 1;
+    J.nb = nb;
+    J.P = P;
+    J.Q = Q;
+    J.blocks = ((Q + 31) / 32) * ((P + 31) / 32) * nb;
+    total += J.blocks;
+  }
+  moe_status_t launch(cudaStream_t st) {
+    if (total == 0) return MOE_OK;
+    ProfScope prof(MOE_PROF_TRANSPOSE, st);
+    factor_prep_kernel<<<total, 256, 0, st>>>(jobs);
+    count_launch();
+    return launch_status();
+  }
+};
 
 }  // namespace
 
@@ -747,18 +762,18 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
   const bool pair_down = use_pairs(R, E, H, true);
   const bool pair_gate_up = use_pairs(R, E, 2 * I, true);
   const int wdown = pair_down ? 32 : 64, wgate = pair_gate_up ? 32 : 64;
+  FactorPrep prep;
   if (r < wdown) {
     B2p = at<__nv_bfloat16>(ws, wo[3]);
-    if ((stt = pad_cols(B2, const_cast<void*>(B2p), 1ll * E * H, r, wdown, st)) != MOE_OK)
-      return stt;
+    prep.pad(B2, const_cast<void*>(B2p), 1ll * E * H, r, wdown);
   }
   if (r < wgate) {
     B1p = at<__nv_bfloat16>(ws, wo[5]);
-    if ((stt = pad_cols(B1, const_cast<void*>(B1p), 2ll * E * I, r, wgate, st)) != MOE_OK)
-      return stt;
+    prep.pad(B1, const_cast<void*>(B1p), 2ll * E * I, r, wgate);
   }
-  if ((stt = transpose(A2, A2t, E, r, I, st)) != MOE_OK) return stt;
-  if ((stt = transpose(A1, A1t, E, r, H, st)) != MOE_OK) return stt;
+  prep.transpose(A2, A2t, E, r, I);
+  prep.transpose(A1, A1t, E, r, H);
+  if ((stt = prep.launch(st)) != MOE_OK) return stt;
   const CUtensorMapSwizzle lsw = lora_swizzle(r);
   const uint64_t EU = static_cast<uint64_t>(E);
 

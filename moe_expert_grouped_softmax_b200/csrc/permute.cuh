@@ -225,39 +225,60 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// out[row][0:width] = (in[row][0:r], zeros) for bf16 rows (LoRA factors
-// only; width a multiple of 8 and >= r).
-__global__ void pad_cols_kernel(const __nv_bfloat16* __restrict__ in,
-                                __nv_bfloat16* __restrict__ out, long long rows, int r,
-                                int width) {
-  const int chunks = width / 8;  // 16-byte chunks per output row
-  const long long n = rows * chunks;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
-       i < n; i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = i / chunks;
-    const int c8 = static_cast<int>(i - row * chunks) * 8;  // first column of this chunk
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (c8 < r) v = *reinterpret_cast<const uint4*>(in + row * r + c8);
-    *reinterpret_cast<uint4*>(out + row * width + c8) = v;
-  }
-}
+// The backward's operand copies of the LoRA factors in one launch: a list
+// of jobs, each either a zero-padding copy (out[row][0:width] = (in[row][0:r],
+// zeros); width a multiple of 8, >= r) or a batched transpose
+// ([nb, P, Q] -> [nb, Q, P]).  Each CTA (256 threads) works for one job.
+struct FactorJob {
+  const __nv_bfloat16* in;
+  __nv_bfloat16* out;
+  int kind;          // 0: pad, 1: transpose
+  int blocks;        // CTAs given to this job
+  long long rows;    // pad
+  int r, width;      // pad
+  int nb, P, Q;      // transpose
+};
+constexpr int kMaxFactorJobs = 4;
+struct FactorJobs {
+  FactorJob job[kMaxFactorJobs];
+  int n;
+};
 
-// out[b][q][p] = in[b][p][q] for bf16 matrices [nb][P][Q] (LoRA factors only).
-__global__ void transpose_kernel(const __nv_bfloat16* __restrict__ in,
-                                 __nv_bfloat16* __restrict__ out, int P, int Q) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const size_t b = blockIdx.z;
-  const __nv_bfloat16* src = in + b * static_cast<size_t>(P) * Q;
-  __nv_bfloat16* dst = out + b * static_cast<size_t>(P) * Q;
-  const int q0 = blockIdx.x * 32, p0 = blockIdx.y * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int p = p0 + i, q = q0 + threadIdx.x;
-    if (p < P && q < Q) tile[i][threadIdx.x] = src[static_cast<size_t>(p) * Q + q];
+__global__ void __launch_bounds__(256) factor_prep_kernel(const FactorJobs jobs) {
+  int b = blockIdx.x, ji = 0;
+  while (ji < jobs.n && b >= jobs.job[ji].blocks) {
+    b -= jobs.job[ji].blocks;
+    ++ji;
   }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int q = q0 + i, p = p0 + threadIdx.x;
-    if (p < P && q < Q) dst[static_cast<size_t>(q) * P + p] = tile[threadIdx.x][i];
+  if (ji >= jobs.n) return;
+  const FactorJob& J = jobs.job[ji];
+  if (J.kind == 0) {
+    const int chunks = J.width / 8;  // 16-byte chunks per output row
+    const long long n = J.rows * chunks;
+    for (long long i = b * 256ll + threadIdx.x; i < n; i += static_cast<long long>(J.blocks) * 256) {
+      const long long row = i / chunks;
+      const int c8 = static_cast<int>(i - row * chunks) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (c8 < J.r) v = *reinterpret_cast<const uint4*>(J.in + row * J.r + c8);
+      *reinterpret_cast<uint4*>(J.out + row * J.width + c8) = v;
+    }
+  } else {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int qt = (J.Q + 31) / 32, pt = (J.P + 31) / 32;
+    const int q0 = (b % qt) * 32, p0 = ((b / qt) % pt) * 32;
+    const size_t bb = static_cast<size_t>(b / (qt * pt));
+    const __nv_bfloat16* src = J.in + bb * static_cast<size_t>(J.P) * J.Q;
+    __nv_bfloat16* dst = J.out + bb * static_cast<size_t>(J.P) * J.Q;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int i = ty; i < 32; i += 8) {
+      const int p = p0 + i, q = q0 + tx;
+      if (p < J.P && q < J.Q) tile[i][tx] = src[static_cast<size_t>(p) * J.Q + q];
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+      const int q = q0 + i, p = p0 + tx;
+      if (p < J.P && q < J.Q) dst[static_cast<size_t>(q) * J.P + p] = tile[tx][i];
+    }
   }
 }
 
