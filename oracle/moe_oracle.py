@@ -20,6 +20,10 @@ Sources (web pages; cited by title and section):
   - section "Implementation details": a LoRA adapter on an (m, n) weight is a
     pair of (m, r) and (r, n) matrices, the router is not fine-tuned, and the
     recommended ``lora_alpha = 2 r`` gives the standard scale s = alpha / r.
+  - the page's opening list of what the kernels support: LoRA and full
+    fine-tuning (FFT).  With the base weights trainable, each projection
+    ``y = x W^T`` also yields ``dW = dy^T x`` (chain rule; unchanged by the
+    split order of the LoRA term).
 * [P5] aiflowlearn codex tutorial "Meet Unsloth", section on ``fast_lora.py``
   (``LoRA_MLP``): SwiGLU is ``e = X G; f = e * sigmoid(e); g = X U;
   h = f * g; out = h W``.
@@ -61,6 +65,7 @@ __all__ = [
     "expert_backward",
     "grouped_forward",
     "grouped_backward",
+    "grouped_base_grads",
     "block_forward",
     "block_backward",
 ]
@@ -237,7 +242,17 @@ def expert_backward(dZ2, cache, W1, A1, B1, W2, A2, B2, s):
     dX = dZ1 @ W1 + s * (dZB1 @ A1)      # [M, H]
     dA1 = s * (dZB1.T @ X)               # [r, H]
     dB1 = s * (dZ1.T @ (X @ A1.T))       # [2I, r]
+    cache["dZ1"] = dZ1                   # for the base-weight gradients
     return dX, dA1, dB1, dA2, dB2
+
+
+def expert_base_grads(dZ2, cache):
+    """Base-weight gradients of one expert when W1, W2 are trainable (full
+    fine-tuning, [P1] opening list): for ``y = x W^T``, ``dW = dy^T x``, so
+    ``dW2 = dZ2^T h`` [H, I] and ``dW1 = dZ1^T X`` [2I, H].  ``cache`` must have
+    been through :func:`expert_backward` (which leaves dZ1 in it)."""
+    dZ2 = _f64(dZ2)
+    return cache["dZ1"].T @ cache["X"], dZ2.T @ cache["h"]
 
 
 # --------------------------------------------------------------------------
@@ -280,6 +295,22 @@ def grouped_backward(dZ2p, offsets, caches, W1, A1, B1, W2, A2, B2, s):
     return dXp, dA1, dB1, dA2, dB2
 
 
+def grouped_base_grads(dZ2p, offsets, caches, H, I):
+    """dW1 [E, 2I, H] and dW2 [E, H, I] over the experts (after
+    :func:`grouped_backward` on the same caches); empty experts get exact
+    zeros."""
+    dZ2p = _f64(dZ2p)
+    E = len(offsets) - 1
+    dW1 = np.zeros((E, 2 * I, H))
+    dW2 = np.zeros((E, H, I))
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if b == a:
+            continue
+        dW1[e], dW2[e] = expert_base_grads(dZ2p[a:b], caches[e])
+    return dW1, dW2
+
+
 # --------------------------------------------------------------------------
 # the whole block
 # --------------------------------------------------------------------------
@@ -306,8 +337,9 @@ def block_forward(X, logits, k, W1, A1, B1, W2, A2, B2, s, route=None):
     return Y, ctx
 
 
-def block_backward(dY, ctx):
-    """Gradients of ``<dY, Y>``: dX, dA1, dB1, dA2, dB2 and dw.
+def block_backward(dY, ctx, base=False):
+    """Gradients of ``<dY, Y>``: dX, dA1, dB1, dA2, dB2 and dw (and, with
+    ``base``, the base-weight gradients dW1, dW2).
 
     weighted dY gather ``dZ2p[dest[t, j]] = w[t, j] dY[t]``;
     ``dw[t, j] = <dY[t], Z2p[dest[t, j]]>``; expert backward;
@@ -325,5 +357,10 @@ def block_backward(dY, ctx):
     dXp, dA1, dB1, dA2, dB2 = grouped_backward(
         dZ2p, ctx["offsets"], ctx["caches"], W1, A1, B1, W2, A2, B2, ctx["s"])
     dX = unpermute(dXp, dest, None)
-    return dict(dX=dX, dA1=dA1, dB1=dB1, dA2=dA2, dB2=dB2, dw=dw,
-                dZ2p=dZ2p, dXp=dXp)
+    out = dict(dX=dX, dA1=dA1, dB1=dB1, dA2=dA2, dB2=dB2, dw=dw,
+               dZ2p=dZ2p, dXp=dXp)
+    if base:
+        H, I = np.shape(W2)[1], np.shape(W2)[2]
+        out["dW1"], out["dW2"] = grouped_base_grads(dZ2p, ctx["offsets"], ctx["caches"],
+                                                    H, I)
+    return out

@@ -246,15 +246,16 @@ def test_backward_matches_torch_autograd_of_merged_weights():
     P = _params(E, H, I, r, rng)
     dY = rng.normal(size=(T, H))
     _, ctx = O.block_forward(X, L, k, *P, s)
-    g = O.block_backward(dY, ctx)
+    g = O.block_backward(dY, ctx, base=True)
     tX = torch.tensor(X, requires_grad=True)
     tw = torch.tensor(ctx["w"], requires_grad=True)
     tP = [torch.tensor(p, requires_grad=True) for p in P]
     loss = _torch_merged_loss(tX, tw, ctx["idx"], tP, s, torch.tensor(dY))
     gX, gw, gW1, gA1, gB1, gW2, gA2, gB2 = torch.autograd.grad(
         loss, [tX, tw] + tP)
+    # (the merged weight W + sBA has the base-weight gradient of W itself)
     for name, want in [("dX", gX), ("dw", gw), ("dA1", gA1), ("dB1", gB1),
-                       ("dA2", gA2), ("dB2", gB2)]:
+                       ("dA2", gA2), ("dB2", gB2), ("dW1", gW1), ("dW2", gW2)]:
         np.testing.assert_allclose(g[name], want.numpy(), rtol=1e-10,
                                    atol=1e-10, err_msg=name)
 
@@ -267,7 +268,7 @@ def test_backward_finite_differences():
     P = list(_params(E, H, I, r, rng, scale=0.5))
     dY = rng.normal(size=(T, H))
     _, ctx = O.block_forward(X, L, k, *P, s)
-    grads = O.block_backward(dY, ctx)
+    grads = O.block_backward(dY, ctx, base=True)
     route = (ctx["idx"], ctx["w"])
 
     def loss(X_, P_, w_=None):
@@ -284,8 +285,9 @@ def test_backward_finite_differences():
         Xm_[i, j] -= eps
         fd[i, j] = (loss(Xp_, P) - loss(Xm_, P)) / (2 * eps)
     np.testing.assert_allclose(grads["dX"], fd, rtol=1e-6, atol=1e-7)
-    # LoRA matrices: every entry
-    for pi, name in [(1, "dA1"), (2, "dB1"), (4, "dA2"), (5, "dB2")]:
+    # LoRA matrices and base weights: every entry
+    for pi, name in [(1, "dA1"), (2, "dB1"), (4, "dA2"), (5, "dB2"), (0, "dW1"),
+                     (3, "dW2")]:
         fd = np.zeros_like(P[pi])
         for ix in np.ndindex(P[pi].shape):
             Pp = [p.copy() for p in P]
@@ -313,8 +315,31 @@ def test_empty_expert_grads_are_exact_zero():
     L[:, 4:] = -30.0
     P = _params(E, H, I, r, rng)
     _, ctx = O.block_forward(X, L, k, *P, 2.0)
-    g = O.block_backward(rng.normal(size=(T, H)), ctx)
+    g = O.block_backward(rng.normal(size=(T, H)), ctx, base=True)
     assert (ctx["counts"][4:] == 0).all()
-    for n in ("dA1", "dB1", "dA2", "dB2"):
+    for n in ("dA1", "dB1", "dA2", "dB2", "dW1", "dW2"):
         assert np.all(g[n][4:] == 0.0)
         assert np.any(g[n][:4] != 0.0)
+
+
+def test_base_grads_dense_closed_form():
+    """E = 1, k = 1: dW2 = (w dY)^T h and dW1 = dZ1^T X over all tokens, with
+    h and dZ1 from the textbook SwiGLU chain written out here."""
+    rng = np.random.default_rng(31)
+    T, H, I, r, s = 9, 7, 5, 2, 1.5
+    X = rng.normal(size=(T, H))
+    L = np.zeros((T, 1), dtype=np.float32)
+    W1, A1, B1, W2, A2, B2 = _params(1, H, I, r, rng)
+    dY = rng.normal(size=(T, H))
+    _, ctx = O.block_forward(X, L, 1, W1, A1, B1, W2, A2, B2, s)
+    g = O.block_backward(dY, ctx, base=True)
+    M1 = W1[0] + s * B1[0] @ A1[0]
+    M2 = W2[0] + s * B2[0] @ A2[0]
+    Z = X @ M1.T
+    gate, up = Z[:, :I], Z[:, I:]
+    sig = 1.0 / (1.0 + np.exp(-gate))
+    h = gate * sig * up
+    dh = dY @ M2
+    dZ1 = np.concatenate([dh * up * (sig + gate * sig * (1 - sig)), dh * gate * sig], axis=1)
+    np.testing.assert_allclose(g["dW2"][0], dY.T @ h, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dW1"][0], dZ1.T @ X, rtol=1e-12, atol=1e-12)
