@@ -197,7 +197,7 @@ def run_ours(args, cfg):
     inp = S.make_inputs(cfg)
     W = [inp[n].to(dev) for n in ("W1", "A1", "B1", "W2", "A2", "B2")]
     X, logits, dY = (inp[n].to(dev) for n in ("X", "logits", "dY"))
-    blk = ops.MoeBlock(T, H, I, E, k, r, s, device=dev)
+    blk = ops.MoeBlock(T, H, I, E, k, r, s, device=dev, full_ft=args.full_ft)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -253,7 +253,7 @@ def run_ours(args, cfg):
     # (two block instances, double-buffered).
     e2e = None
     if not args.no_e2e:
-        blocks = [blk, ops.MoeBlock(T, H, I, E, k, r, s, device=dev)]
+        blocks = [blk, ops.MoeBlock(T, H, I, E, k, r, s, device=dev, full_ft=args.full_ft)]
         hin = [(X.cpu().pin_memory(), logits.cpu().pin_memory(), dY.cpu().pin_memory())
                for _ in range(2)]
         din = [(torch.empty_like(X), torch.empty_like(logits), torch.empty_like(dY))
@@ -310,7 +310,9 @@ def run_ours(args, cfg):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / K,
                "note": "pinned host buffers; copies on two streams overlap the "
-                       "neighbouring steps' compute (double-buffered)"}
+                       "neighbouring steps' compute (double-buffered)"
+                       + ("; dW1, dW2 stay on the device (an optimizer step would "
+                          "consume them there)" if args.full_ft else "")}
         st = ops.device_status()
         if st != 0:
             raise RuntimeError(f"device status {st} after end-to-end steps")
@@ -361,6 +363,8 @@ def main():
     ap.add_argument("--cpu-sample-tokens", type=int, default=128)
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (small cases for profiler captures)")
+    ap.add_argument("--full-ft", action="store_true",
+                    help="full fine-tuning: also the base-weight gradients dW1, dW2")
     ap.add_argument("--cta-pairs", type=int, default=-1,
                     help="1: grouped GEMMs on CTA pairs, 0: single CTAs, "
                          "-1: library default")
@@ -372,13 +376,15 @@ def main():
         cfg["T"] = args.tokens
     T, H, I, E, k, r = (cfg[x] for x in ("T", "H", "I", "E", "k", "r"))
     R = T * k
-    flops = WL.block_flops(T, H, I, E, k, r)["total"]
+    flops = WL.block_flops(T, H, I, E, k, r, full_ft=args.full_ft)["total"]
     pk = peaks()
     workload = {"gpt-oss-20b": "gpt-oss-20b-shaped MoE layer fwd+bwd",
                 "qwen3-30b-a3b": "Qwen3-30B-A3B-shaped MoE layer fwd+bwd",
                 "gpt-oss-20b-long": "long-context gpt-oss-20b-shaped MoE layer fwd+bwd",
                 "deepseek-v3": "DeepSeek-V3-shaped MoE layer fwd+bwd",
                 "tiny": "tiny MoE block fwd+bwd"}[args.config]
+    if args.full_ft:
+        workload += ", full fine-tuning (base-weight gradients too)"
     config = {"workload": workload, "T": T, "H": H, "I": I, "E": E, "top_k": k,
               "lora_r": r, "lora_s": cfg["s"], "logits": cfg["logits"],
               "parallelism": "replicas", "l2": "256 MiB memset before each step, "

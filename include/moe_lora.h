@@ -179,6 +179,27 @@ MOE_API moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
                               void* dB2, void* ws, size_t ws_bytes,
                               moe_stream_t stream);
 
+/* -------------------------- full fine-tuning: base-weight gradients as well
+ * The page lists full fine-tuning beside LoRA among what its MoE kernels
+ * support.  Everything moe_lora_mlp_bwd computes, plus, with W1 and W2
+ * trainable (dW = dy^T x for each projection y = x W^T), per expert e with
+ * rows [a, b):
+ *   dW1[e] = dZ1[a:b]^T Xp[a:b]   [2I, H]     dW2[e] = dZ2[a:b]^T h[a:b]   [H, I]
+ * Outputs dW1 [E, 2I, H] and dW2 [E, H, I] bf16 (the layouts of W1, W2),
+ * accumulated in fp32 over the expert's rows in a fixed order
+ * (deterministic); experts with no rows get exact zeros.  dW1 and dW2 must
+ * both be non-NULL (MOE_ERR_INVALID_ARG otherwise) and 16-byte aligned.  Same
+ * saved activations and workspace as moe_lora_mlp_bwd. */
+MOE_API moe_status_t moe_lora_mlp_bwd_full(const void* dZ2, const void* Xp,
+                                   const int32_t* expert_offsets,
+                                   int E, int H, int I, int r, float s,
+                                   const void* W1, const void* A1, const void* B1,
+                                   const void* W2, const void* A2, const void* B2,
+                                   const void* saved, size_t saved_bytes, int R,
+                                   void* dXp, void* dA1, void* dB1, void* dA2,
+                                   void* dB2, void* dW1, void* dW2, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- status
  * moe_get_device_status synchronises `stream`, returns the first device-side
  * error recorded since the last call (MOE_OK if none) and clears it.
@@ -230,7 +251,8 @@ MOE_API void moe_set_cta_pairs(int mode);
 #define MOE_PROF_GATE_UP_BWD 6
 #define MOE_PROF_LORA_GRAD 7
 #define MOE_PROF_TRANSPOSE 8
-#define MOE_PROF_KINDS 9
+#define MOE_PROF_BASE_GRAD 9
+#define MOE_PROF_KINDS 10
 MOE_API moe_status_t moe_profile_enable(int on);
 MOE_API int moe_profile_collect(int kind, float* ms, int max_n);
 

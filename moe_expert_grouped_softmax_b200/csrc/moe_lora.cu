@@ -18,6 +18,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "lora_grad.cuh"
+#include "base_grad.cuh"
 
 using namespace moe;
 
@@ -401,6 +402,63 @@ struct FactorPrep {
   }
 };
 
+template <int BN>
+moe_status_t launch_base_grad_t(const CUtensorMap* u, const CUtensorMap* v,
+                                BaseGradArgs args, cudaStream_t st) {
+  using C = BaseGradCfg<BN>;
+  int begin = 0;
+  for (int i = 0; i < 2; ++i) {
+    BaseGradProblem& p = args.prob[i];
+    p.p_tiles = (p.P + 127) / 128;
+    p.q_tiles = (p.Q + BN - 1) / BN;
+    p.tile_begin = begin;
+    begin += args.E * p.p_tiles * p.q_tiles;
+  }
+  args.total_tiles = begin;
+  auto kern = base_grad_kernel<BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_BYTES) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int grid = std::min(num_sms(), args.total_tiles);
+  if (grid <= 0) return MOE_OK;
+  ProfScope prof(MOE_PROF_BASE_GRAD, st);
+  kern<<<grid, 192, C::SMEM_BYTES, st>>>(u[0], u[1], v[0], v[1], args);
+  count_launch();
+  return launch_status();
+}
+
+// dW1 = per-expert dZ1^T Xp, dW2 = dZ2^T h (one launch for both).  The tile
+// width is the one of {256, 192} with the smaller estimated cost
+// tiles * (BN + 32) over both problems.
+moe_status_t base_grads(const void* dZ1, const void* Xp, const void* dZ2, const void* h,
+                        const int32_t* offsets, int E, int H, int I, int R, void* dW1,
+                        void* dW2, cudaStream_t st) {
+  const void* U[2] = {dZ1, dZ2};
+  const void* V[2] = {Xp, h};
+  const int P[2] = {2 * I, H}, Q[2] = {H, I};
+  CUtensorMap tu[2], tv[2];
+  for (int i = 0; i < 2; ++i) {
+    bool ok = tmap_2d(&tu[i], U[i], P[i], R, P[i] * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tv[i], V[i], Q[i], R, Q[i] * 2ull, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return MOE_ERR_CUDA;
+  }
+  BaseGradArgs g{};
+  g.offsets = offsets;
+  g.E = E;
+  g.R = R;
+  g.wait_ns = g_wait_limit_ns;
+  g.prob[0].P = P[0]; g.prob[0].Q = Q[0]; g.prob[0].out = static_cast<__nv_bfloat16*>(dW1);
+  g.prob[1].P = P[1]; g.prob[1].Q = Q[1]; g.prob[1].out = static_cast<__nv_bfloat16*>(dW2);
+  double cost[2] = {0, 0};
+  const int bns[2] = {256, 192};
+  for (int c = 0; c < 2; ++c)
+    for (int i = 0; i < 2; ++i)
+      cost[c] += static_cast<double>((P[i] + 127) / 128) * ((Q[i] + bns[c] - 1) / bns[c]) *
+                 (bns[c] + 32);
+  return cost[0] <= cost[1] ? launch_base_grad_t<256>(tu, tv, g, st)
+                            : launch_base_grad_t<192>(tu, tv, g, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -714,16 +772,22 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
 }
 
 // ------------------------------------------------------------------ backward
-moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
-                              const int32_t* expert_offsets, int E, int H, int I, int r,
-                              float s, const void* W1, const void* A1, const void* B1,
-                              const void* W2, const void* A2, const void* B2,
-                              const void* saved, size_t saved_bytes, int R, void* dXp,
-                              void* dA1, void* dB1, void* dA2, void* dB2, void* ws,
-                              size_t ws_bytes, moe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
+                               const int32_t* expert_offsets, int E, int H, int I, int r,
+                               float s, const void* W1, const void* A1, const void* B1,
+                               const void* W2, const void* A2, const void* B2,
+                               const void* saved, size_t saved_bytes, int R, void* dXp,
+                               void* dA1, void* dB1, void* dA2, void* dB2, void* dW1,
+                               void* dW2, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (!shape_ok(E, H, I, r) || R < 0) return MOE_ERR_UNSUPPORTED;
   if (!dA1 || !dB1 || !dA2 || !dB2) return MOE_ERR_INVALID_ARG;
-  cudaStream_t st = stream;
+  const bool full = dW1 != nullptr;
+  if (full && ((reinterpret_cast<uintptr_t>(dW1) | reinterpret_cast<uintptr_t>(dW2)) & 15u))
+    return MOE_ERR_INVALID_ARG;
   if (R == 0) {
     const size_t n = static_cast<size_t>(E) * r * 2;
     if (cudaMemsetAsync(dA1, 0, n * H, st) != cudaSuccess ||
@@ -731,6 +795,12 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
         cudaMemsetAsync(dA2, 0, n * I, st) != cudaSuccess ||
         cudaMemsetAsync(dB2, 0, n * H, st) != cudaSuccess)
       return MOE_ERR_CUDA;
+    if (full) {
+      const size_t w = static_cast<size_t>(E) * H * I * 2;
+      if (cudaMemsetAsync(dW1, 0, 2 * w, st) != cudaSuccess ||
+          cudaMemsetAsync(dW2, 0, w, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
     return MOE_OK;
   }
   if (!dZ2 || !Xp || !expert_offsets || !W1 || !A1 || !B1 || !W2 || !A2 || !B2 ||
@@ -863,7 +933,41 @@ moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
     else stt = launch_grad_t<64>(tu, tv, g, st);
     if (stt != MOE_OK) return stt;
   }
+  // base-weight gradients (full fine-tuning)
+  if (full &&
+      (stt = base_grads(dZ1, Xp, dZ2, h, expert_offsets, E, H, I, R, dW1, dW2, st)) != MOE_OK)
+    return stt;
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_lora_mlp_bwd(const void* dZ2, const void* Xp,
+                              const int32_t* expert_offsets, int E, int H, int I, int r,
+                              float s, const void* W1, const void* A1, const void* B1,
+                              const void* W2, const void* A2, const void* B2,
+                              const void* saved, size_t saved_bytes, int R, void* dXp,
+                              void* dA1, void* dB1, void* dA2, void* dB2, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+  return lora_mlp_bwd_impl(dZ2, Xp, expert_offsets, E, H, I, r, s, W1, A1, B1, W2, A2, B2,
+                           saved, saved_bytes, R, dXp, dA1, dB1, dA2, dB2, nullptr,
+                           nullptr, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_lora_mlp_bwd_full(const void* dZ2, const void* Xp,
+                                   const int32_t* expert_offsets, int E, int H, int I,
+                                   int r, float s, const void* W1, const void* A1,
+                                   const void* B1, const void* W2, const void* A2,
+                                   const void* B2, const void* saved, size_t saved_bytes,
+                                   int R, void* dXp, void* dA1, void* dB1, void* dA2,
+                                   void* dB2, void* dW1, void* dW2, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream) {
+  if (!dW1 || !dW2) return MOE_ERR_INVALID_ARG;
+  return lora_mlp_bwd_impl(dZ2, Xp, expert_offsets, E, H, I, r, s, W1, A1, B1, W2, A2, B2,
+                           saved, saved_bytes, R, dXp, dA1, dB1, dA2, dB2, dW1, dW2, ws,
+                           ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape",
 EXPORTS = [
     "moe_route_workspace_bytes", "moe_route_topk", "moe_permute", "moe_unpermute",
     "moe_saved_bytes", "moe_saved_part_offset", "moe_workspace_bytes",
-    "moe_lora_mlp_fwd", "moe_lora_mlp_bwd", "moe_get_device_status",
+    "moe_lora_mlp_fwd", "moe_lora_mlp_bwd", "moe_lora_mlp_bwd_full", "moe_get_device_status",
     "moe_status_string", "moe_set_wait_limit_ns", "moe_test_inject_stall",
     "moe_set_cta_pairs", "moe_kernel_launches", "moe_profile_enable",
     "moe_profile_collect",
@@ -31,7 +31,7 @@ EXPORTS = [
 
 PROF_KINDS = {"route": 0, "permute": 1, "gate_up_fwd": 2, "down_fwd": 3,
               "unpermute": 4, "down_bwd": 5, "gate_up_bwd": 6, "lora_grad": 7,
-              "transpose": 8}
+              "transpose": 8, "base_grad": 9}
 
 
 class MoeError(RuntimeError):
@@ -71,6 +71,9 @@ def lib():
         L.moe_lora_mlp_bwd.argtypes = [P, P, P, I, I, I, I, F, P, P, P, P, P, P, P,
                                        S, I, P, P, P, P, P, P, S, P]
         L.moe_lora_mlp_bwd.restype = I
+        L.moe_lora_mlp_bwd_full.argtypes = [P, P, P, I, I, I, I, F, P, P, P, P, P, P, P,
+                                            S, I, P, P, P, P, P, P, P, P, S, P]
+        L.moe_lora_mlp_bwd_full.restype = I
         L.moe_get_device_status.argtypes = [P]
         L.moe_get_device_status.restype = I
         L.moe_status_string.argtypes = [I]
@@ -275,8 +278,10 @@ def lora_mlp_fwd(Xp, offsets, W1, A1, B1, W2, A2, B2, s, out=None, saved=None):
 
 
 def lora_mlp_bwd(dZ2, Xp, offsets, W1, A1, B1, W2, A2, B2, s, saved, out=None,
-                 ws=None):
-    """a7 + a8 + a9: returns (dXp, dA1, dB1, dA2, dB2)."""
+                 ws=None, base_out=None):
+    """a7 + a8 + a9: returns (dXp, dA1, dB1, dA2, dB2).  With ``base_out`` =
+    (dW1 [E, 2I, H], dW2 [E, H, I]) the base-weight gradients of full
+    fine-tuning are written there too (``moe_lora_mlp_bwd_full``)."""
     E, H, I, r = _weights_check(W1, A1, B1, W2, A2, B2)
     R = Xp.shape[0]
     _need(dZ2, torch.bfloat16, (R, H), "dZ2")
@@ -293,12 +298,24 @@ def lora_mlp_bwd(dZ2, Xp, offsets, W1, A1, B1, W2, A2, B2, s, saved, out=None,
     nb = workspace_bytes(R, E, H, I, r)
     if ws is None or ws.numel() < nb:
         ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev)
-    _check(lib().moe_lora_mlp_bwd(_p(dZ2), _p(Xp), _p(offsets), E, H, I, r, float(s),
-                                  _p(W1), _p(A1), _p(B1), _p(W2), _p(A2), _p(B2),
-                                  _p(saved), saved.numel(), R, _p(dXp), _p(dA1),
-                                  _p(dB1), _p(dA2), _p(dB2), _p(ws), ws.numel(),
-                                  _stream()),
-           "moe_lora_mlp_bwd")
+    if base_out is None:
+        _check(lib().moe_lora_mlp_bwd(_p(dZ2), _p(Xp), _p(offsets), E, H, I, r, float(s),
+                                      _p(W1), _p(A1), _p(B1), _p(W2), _p(A2), _p(B2),
+                                      _p(saved), saved.numel(), R, _p(dXp), _p(dA1),
+                                      _p(dB1), _p(dA2), _p(dB2), _p(ws), ws.numel(),
+                                      _stream()),
+               "moe_lora_mlp_bwd")
+    else:
+        dW1, dW2 = base_out
+        _need(dW1, torch.bfloat16, (E, 2 * I, H), "dW1")
+        _need(dW2, torch.bfloat16, (E, H, I), "dW2")
+        _check(lib().moe_lora_mlp_bwd_full(_p(dZ2), _p(Xp), _p(offsets), E, H, I, r,
+                                           float(s), _p(W1), _p(A1), _p(B1), _p(W2),
+                                           _p(A2), _p(B2), _p(saved), saved.numel(), R,
+                                           _p(dXp), _p(dA1), _p(dB1), _p(dA2), _p(dB2),
+                                           _p(dW1), _p(dW2), _p(ws), ws.numel(),
+                                           _stream()),
+               "moe_lora_mlp_bwd_full")
     return dXp, dA1, dB1, dA2, dB2
 
 
@@ -308,9 +325,10 @@ class MoeBlock:
     buffers preallocated once for a fixed shape (used by the benchmark and the
     end-to-end tests).  ``step`` runs, on the current stream: route, permute,
     gate_up + SwiGLU, down, weighted unpermute, weighted dY gather, down /
-    gate_up backward, LoRA gradients and the dX combine."""
+    gate_up backward, LoRA gradients and the dX combine (with ``full_ft``, also
+    the base-weight gradients dW1, dW2 of full fine-tuning)."""
 
-    def __init__(self, T, H, I, E, k, r, s, device="cuda", with_dw=False):
+    def __init__(self, T, H, I, E, k, r, s, device="cuda", with_dw=False, full_ft=False):
         self.T, self.H, self.I, self.E, self.k, self.r, self.s = T, H, I, E, k, r, s
         self.R = R = T * k
         self.with_dw = with_dw
@@ -336,6 +354,9 @@ class MoeBlock:
         self.dB1 = torch.empty((E, 2 * I, r), dtype=bf, device=dev)
         self.dA2 = torch.empty((E, r, I), dtype=bf, device=dev)
         self.dB2 = torch.empty((E, H, r), dtype=bf, device=dev)
+        self.full_ft = full_ft
+        self.dW1 = torch.empty((E, 2 * I, H), dtype=bf, device=dev) if full_ft else None
+        self.dW2 = torch.empty((E, H, I), dtype=bf, device=dev) if full_ft else None
         self.ws = torch.empty(max(1, workspace_bytes(R, E, H, I, r)), dtype=torch.uint8,
                               device=dev)
 
@@ -353,7 +374,8 @@ class MoeBlock:
         else:
             permute(dY, self.dest, scale=self.w, out=self.dZ2)
         lora_mlp_bwd(self.dZ2, self.Xp, self.offsets, *W, self.s, self.saved,
-                     out=(self.dXp, self.dA1, self.dB1, self.dA2, self.dB2), ws=self.ws)
+                     out=(self.dXp, self.dA1, self.dB1, self.dA2, self.dB2), ws=self.ws,
+                     base_out=(self.dW1, self.dW2) if self.full_ft else None)
         unpermute(self.dXp, self.dest, None, out=self.dX)
         return self.dX
 

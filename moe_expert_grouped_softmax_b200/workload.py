@@ -32,8 +32,15 @@ def merged_lora_flops(E, rows, m, n, r):
     return E * (2 * m * n * r + m * n) + 2 * rows * m * n
 
 
-def block_flops(T, H, I, E, k, r):
-    """Forward + backward algorithmic FLOPs of the block (base frozen)."""
+def base_grad_flops(R, H, I):
+    """Base-weight gradients of full fine-tuning: dW1 = dZ1^T Xp [2I, H] and
+    dW2 = dZ2^T h [H, I] over all routed rows."""
+    return 2 * R * (2 * I * H + H * I)
+
+
+def block_flops(T, H, I, E, k, r, full_ft=False):
+    """Forward + backward algorithmic FLOPs of the block (base frozen, or with
+    the base-weight gradients when ``full_ft``)."""
     R = T * k
     fwd = (split_lora_proj_flops(R, H, 2 * I, r)
            + split_lora_proj_flops(R, I, H, r))
@@ -41,8 +48,9 @@ def block_flops(T, H, I, E, k, r):
     # dA 2rm, dB 2nr
     def bwd(m, n):
         return 2 * R * (m * n + n * r + r * m + r * m + n * r)
-    return dict(fwd=fwd, bwd=bwd(H, 2 * I) + bwd(I, H),
-                total=fwd + bwd(H, 2 * I) + bwd(I, H),
+    extra = base_grad_flops(R, H, I) if full_ft else 0
+    return dict(fwd=fwd, bwd=bwd(H, 2 * I) + bwd(I, H) + extra,
+                total=fwd + bwd(H, 2 * I) + bwd(I, H) + extra,
                 base_gemm=2 * R * (H * 2 * I + I * H) * 2)
 
 
@@ -54,6 +62,7 @@ def gemm_flops(R, H, I, r):
         down_bwd=2 * R * (H * I + H * r + r * I),     # dh, with LoRA path
         gate_up_bwd=2 * R * (2 * I * H + 2 * I * r + r * H),
         lora_grads=2 * R * r * (H + 2 * I + I + H),
+        base_grad=base_grad_flops(R, H, I),
     )
 
 

@@ -65,6 +65,7 @@ __all__ = [
     "expert_backward",
     "grouped_forward",
     "grouped_backward",
+    "expert_base_grads",
     "grouped_base_grads",
     "block_forward",
     "block_backward",

@@ -36,11 +36,12 @@ def f32(t):
     return t.detach().float().cpu().numpy()
 
 
-def oracle_block(inp, k):
-    """Full fp64 oracle forward + backward on the given (CPU) inputs."""
+def oracle_block(inp, k, base=False):
+    """Full fp64 oracle forward + backward on the given (CPU) inputs (with
+    ``base``, also the base-weight gradients dW1, dW2)."""
     W = [f32(inp[n]) for n in ("W1", "A1", "B1", "W2", "A2", "B2")]
     Y, ctx = O.block_forward(f32(inp["X"]), inp["logits"].numpy(), k, *W, inp["s"])
-    g = O.block_backward(f32(inp["dY"]), ctx)
+    g = O.block_backward(f32(inp["dY"]), ctx, base=base)
     return Y, ctx, g
 
 

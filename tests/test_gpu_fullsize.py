@@ -22,6 +22,7 @@ pytestmark = pytest.mark.gpu
 
 NAMES = ("W1", "A1", "B1", "W2", "A2", "B2")
 FULL = ["gpt-oss-20b", "qwen3-30b-a3b", "gpt-oss-20b-long", "deepseek-v3"]
+FULL_FT = ("gpt-oss-20b", "qwen3-30b-a3b")   # also run the full fine-tuning backward
 
 
 def _expert_weights(inp, e):
@@ -35,13 +36,14 @@ def run(request, cuda_ok):
     dev = torch.device("cuda")
     T, H, I, E, k, r, s = (cfg[x] for x in ("T", "H", "I", "E", "k", "r", "s"))
     W = [inp[n].to(dev) for n in NAMES]
-    blk = ops.MoeBlock(T, H, I, E, k, r, s, device=dev)
+    full_ft = request.param in FULL_FT
+    blk = ops.MoeBlock(T, H, I, E, k, r, s, device=dev, full_ft=full_ft)
     blk.step(inp["X"].to(dev), inp["logits"].to(dev), inp["dY"].to(dev), W)
     torch.cuda.synchronize()
     status = ops.device_status()
-    got = {n: getattr(blk, n).cpu() for n in
-           ("idx", "w", "counts", "offsets", "dest", "Y", "dX", "Z2",
-            "dA1", "dB1", "dA2", "dB2")}
+    names = ["idx", "w", "counts", "offsets", "dest", "Y", "dX", "Z2",
+             "dA1", "dB1", "dA2", "dB2"] + (["dW1", "dW2"] if full_ft else [])
+    got = {n: getattr(blk, n).cpu() for n in names}
     del W, blk
     torch.cuda.empty_cache()
     # oracle routing on the full logits (cheap) drives the sampling
@@ -112,11 +114,15 @@ def test_sampled_experts_lora_grads(run):
         _, dA1, dB1, dA2, dB2 = O.expert_backward(dz2, cache, *W, s)
         for name, ref in (("dA1", dA1), ("dB1", dB1), ("dA2", dA2), ("dB2", dB2)):
             assert_bf16_close(g[name][e], ref, f"{name}[expert {e}, {len(f)} rows]")
+        if "dW1" in g:
+            dW1, dW2 = O.expert_base_grads(dz2, cache)
+            assert_bf16_close(g["dW1"][e], dW1, f"dW1[expert {e}, {len(f)} rows]")
+            assert_bf16_close(g["dW2"][e], dW2, f"dW2[expert {e}, {len(f)} rows]")
 
 
 def test_empty_experts_exact_zero(run):
     g = run["got"]
     empty = np.nonzero(run["rc"] == 0)[0]
-    for name in ("dA1", "dB1", "dA2", "dB2"):
-        if len(empty):
+    for name in ("dA1", "dB1", "dA2", "dB2", "dW1", "dW2"):
+        if len(empty) and name in g:
             assert torch.all(g[name][torch.as_tensor(empty)] == 0), name

@@ -137,10 +137,12 @@ def block_run(request, cuda_ok):
     name, pairs = request.param
     cfg = BLOCK_CASES[name]
     inp = S.make_inputs(cfg)
-    Y, ctx, grads = oracle_block(inp, cfg["k"])
+    Y, ctx, grads = oracle_block(inp, cfg["k"], base=True)
     g = _cuda(inp)
+    # the full fine-tuning backward: the LoRA outputs plus dW1, dW2 (the
+    # LoRA-only entry point is checked against it bit for bit below)
     blk = ops.MoeBlock(cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"], cfg["r"], cfg["s"],
-                       with_dw=True)
+                       with_dw=True, full_ft=True)
     W = _weights(g)
     ops.set_cta_pairs(pairs)
     try:
@@ -206,15 +208,44 @@ def test_block_lora_grads(block_run, name):
         assert torch.all(got[torch.as_tensor(empty, device=got.device)] == 0)
 
 
+@pytest.mark.parametrize("name", ["dW1", "dW2"])
+def test_block_base_grads(block_run, name):
+    """Full fine-tuning: dW1 = dZ1^T Xp and dW2 = dZ2^T h per expert."""
+    b, g, ctx = block_run["blk"], block_run["grads"], block_run["ctx"]
+    got = getattr(b, name)
+    assert_bf16_close(got, g[name], name)
+    empty = np.nonzero(ctx["counts"] == 0)[0]
+    if len(empty):
+        assert torch.all(got[torch.as_tensor(empty, device=got.device)] == 0)
+
+
+def test_block_lora_only_entry_point_matches(block_run):
+    """moe_lora_mlp_bwd (base weights frozen) gives bit-identical LoRA
+    gradients and dX to the full fine-tuning entry point."""
+    cfg, b = block_run["cfg"], block_run["blk"]
+    g = _cuda(block_run["inp"])
+    W = _weights(g)
+    lo = ops.MoeBlock(cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"], cfg["r"], cfg["s"])
+    ops.set_cta_pairs(block_run["pairs"])
+    try:
+        lo.step(g["X"], g["logits"], g["dY"], W)
+        torch.cuda.synchronize()
+    finally:
+        ops.set_cta_pairs(None)
+    assert ops.device_status() == 0
+    for n in ("Y", "dX", "dA1", "dB1", "dA2", "dB2"):
+        assert torch.equal(getattr(lo, n), getattr(b, n)), n
+
+
 def test_block_deterministic(block_run):
     b = block_run["blk"]
     g = _cuda(block_run["inp"])
     W = _weights(g)
-    first = [t.clone() for t in (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2)]
+    first = [t.clone() for t in (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2, b.dW1, b.dW2)]
     ops.set_cta_pairs(block_run["pairs"])
     try:
         b.step(g["X"], g["logits"], g["dY"], W)
     finally:
         ops.set_cta_pairs(None)
-    for x, y in zip(first, (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2)):
+    for x, y in zip(first, (b.Y, b.dX, b.dA1, b.dB1, b.dA2, b.dB2, b.dW1, b.dW2)):
         assert torch.equal(x, y)
