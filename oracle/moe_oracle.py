@@ -69,11 +69,44 @@ __all__ = [
     "grouped_base_grads",
     "block_forward",
     "block_backward",
+    "router_logits",
+    "router_backward",
 ]
 
 
 def _f64(a):
     return np.asarray(a, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------
+# router (trainable variant; the pages keep it frozen by default)
+# --------------------------------------------------------------------------
+def router_logits(X, Wr):
+    """The router's linear layer: ``logits = X Wr^T`` [T, E] for Wr [E, H]
+    ([P1] "What is torch._grouped_mm?": the gate scores each token against
+    every expert before the top-k choice)."""
+    return _f64(X) @ _f64(Wr).T
+
+
+def router_backward(w, dw, idx, X, Wr, E):
+    """Gradients through a trained router, from the routing-weight gradient
+    ``dw`` [T, k] (of ``<dY, Y>``, see :func:`block_backward`).
+
+    The k kept weights are a softmax over the k kept logits (the selection
+    itself is piecewise constant), so for kept slot j of token t
+    ``dlogit[t, idx[t, j]] = w_j (dw_j - sum_i w_i dw_i)`` and 0 for the
+    experts not kept.  Then ``dWr = dlogit^T X`` [E, H] and the router's part
+    of dX is ``dlogit Wr`` [T, H].
+    Returns (dlogits [T, E], dWr [E, H], dX_router [T, H]).
+    """
+    w, dw = _f64(w), _f64(dw)
+    T, k = w.shape
+    dl = np.zeros((T, E))
+    for t in range(T):
+        mean = float(w[t] @ dw[t])
+        for j in range(k):
+            dl[t, int(idx[t, j])] += w[t, j] * (dw[t, j] - mean)
+    return dl, dl.T @ _f64(X), dl @ _f64(Wr)
 
 
 # --------------------------------------------------------------------------

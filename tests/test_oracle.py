@@ -343,3 +343,89 @@ def test_base_grads_dense_closed_form():
     dZ1 = np.concatenate([dh * up * (sig + gate * sig * (1 - sig)), dh * gate * sig], axis=1)
     np.testing.assert_allclose(g["dW2"][0], dY.T @ h, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(g["dW1"][0], dZ1.T @ X, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- trained router
+def _router_case(seed=41):
+    rng = np.random.default_rng(seed)
+    T, H, I, E, k, r, s = 10, 7, 5, 5, 2, 2, 1.4
+    X = rng.normal(size=(T, H))
+    Wr = rng.normal(size=(E, H))
+    P = list(_params(E, H, I, r, rng, scale=0.5))
+    dY = rng.normal(size=(T, H))
+    return X, Wr, P, dY, k, s
+
+
+def _router_loss(X, Wr, P, dY, k, s, route=None):
+    L = O.router_logits(X, Wr)
+    Y, ctx = O.block_forward(X, L, k, *P, s, route=route)
+    return float((Y * dY).sum()), ctx, L
+
+
+def test_router_backward_matches_torch_autograd():
+    """logits = X Wr^T, top-k by torch.topk (no gradient through the choice),
+    softmax over the kept logits, merged-weight experts; autograd gives dX
+    (expert + router paths) and dWr."""
+    X, Wr, P, dY, k, s = _router_case()
+    E = Wr.shape[0]
+    _, ctx, L = _router_loss(X, Wr, P, dY, k, s)
+    g = O.block_backward(dY, ctx)
+    dl, dWr, dXr = O.router_backward(ctx["w"], g["dw"], ctx["idx"], X, Wr, E)
+    tX = torch.tensor(X, requires_grad=True)
+    tWr = torch.tensor(Wr, requires_grad=True)
+    tP = [torch.tensor(p) for p in P]
+    logits = tX @ tWr.T
+    idx = torch.topk(logits.detach(), k, dim=1).indices
+    assert np.array_equal(np.sort(idx.numpy(), 1), np.sort(ctx["idx"], 1))
+    tw = torch.softmax(torch.gather(logits, 1, idx), dim=1)
+    loss = _torch_merged_loss(tX, tw, idx.numpy(), tP, s, torch.tensor(dY))
+    gX, gWr = torch.autograd.grad(loss, [tX, tWr])
+    np.testing.assert_allclose(g["dX"] + dXr, gX.numpy(), rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(dWr, gWr.numpy(), rtol=1e-10, atol=1e-10)
+
+
+def test_router_backward_finite_differences():
+    """Central differences of <dY, Y> in every logit (top-k set unchanged by
+    the step) and every router weight."""
+    X, Wr, P, dY, k, s = _router_case(43)
+    E = Wr.shape[0]
+    _, ctx, L = _router_loss(X, Wr, P, dY, k, s)
+    g = O.block_backward(dY, ctx)
+    dl, dWr, _ = O.router_backward(ctx["w"], g["dw"], ctx["idx"], X, Wr, E)
+    eps = 1e-6
+
+    def loss_L(L_):
+        Y, c = O.block_forward(X, L_, k, *P, s)
+        assert np.array_equal(c["idx"], ctx["idx"])
+        return float((Y * dY).sum())
+
+    fd = np.zeros_like(L)
+    for ix in np.ndindex(L.shape):
+        Lp, Lm = L.copy(), L.copy()
+        Lp[ix] += eps
+        Lm[ix] -= eps
+        fd[ix] = (loss_L(Lp) - loss_L(Lm)) / (2 * eps)
+    np.testing.assert_allclose(dl, fd, rtol=1e-6, atol=1e-7)
+    fd = np.zeros_like(Wr)
+    for ix in np.ndindex(Wr.shape):
+        Wp, Wm = Wr.copy(), Wr.copy()
+        Wp[ix] += eps
+        Wm[ix] -= eps
+        fd[ix] = (_router_loss(X, Wp, P, dY, k, s)[0] - _router_loss(X, Wm, P, dY, k, s)[0]) / (2 * eps)
+    np.testing.assert_allclose(dWr, fd, rtol=1e-6, atol=1e-7)
+
+
+def test_router_gradient_zero_for_unselected_and_sums_to_zero():
+    """Unselected experts get no logit gradient; a shift of all kept logits
+    of a token leaves its weights unchanged, so each row of dlogits sums to 0."""
+    X, Wr, P, dY, k, s = _router_case(47)
+    E = Wr.shape[0]
+    _, ctx, _ = _router_loss(X, Wr, P, dY, k, s)
+    g = O.block_backward(dY, ctx)
+    dl, _, _ = O.router_backward(ctx["w"], g["dw"], ctx["idx"], X, Wr, E)
+    for t in range(X.shape[0]):
+        kept = set(int(e) for e in ctx["idx"][t])
+        for e in range(E):
+            if e not in kept:
+                assert dl[t, e] == 0.0
+    np.testing.assert_allclose(dl.sum(1), 0.0, atol=1e-12)
