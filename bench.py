@@ -197,7 +197,12 @@ def run_ours(args, cfg):
     inp = S.make_inputs(cfg)
     W = [inp[n].to(dev) for n in ("W1", "A1", "B1", "W2", "A2", "B2")]
     X, logits, dY = (inp[n].to(dev) for n in ("X", "logits", "dY"))
-    blk = ops.MoeBlock(T, H, I, E, k, r, s, device=dev, full_ft=args.full_ft)
+    blk = ops.MoeBlock(T, H, I, E, k, r, s, device=dev, full_ft=args.full_ft,
+                       train_router=args.train_router)
+    Wr = None
+    if args.train_router:   # router weights of the trained-router variant
+        g = torch.Generator().manual_seed(cfg["seed"] + 77)
+        Wr = (torch.randn(E, H, generator=g) * 0.05).to(torch.bfloat16).to(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -206,7 +211,7 @@ def run_ours(args, cfg):
             dist.barrier()
 
     for _ in range(args.warmup):
-        blk.step(X, logits, dY, W)
+        blk.step(X, logits, dY, W, Wr)
     torch.cuda.synchronize()
     st = ops.device_status()
     if st != 0:
@@ -225,7 +230,7 @@ def run_ours(args, cfg):
     for i in range(K):
         flush.zero_()                      # L2 flush, outside the timed span
         ev0[i].record(stream)
-        blk.step(X, logits, dY, W)
+        blk.step(X, logits, dY, W, Wr)
         ev1[i].record(stream)
     launches = ops.kernel_launches() - launches0
     torch.cuda.synchronize()
@@ -253,7 +258,8 @@ def run_ours(args, cfg):
     # (two block instances, double-buffered).
     e2e = None
     if not args.no_e2e:
-        blocks = [blk, ops.MoeBlock(T, H, I, E, k, r, s, device=dev, full_ft=args.full_ft)]
+        blocks = [blk, ops.MoeBlock(T, H, I, E, k, r, s, device=dev, full_ft=args.full_ft,
+                                    train_router=args.train_router)]
         hin = [(X.cpu().pin_memory(), logits.cpu().pin_memory(), dY.cpu().pin_memory())
                for _ in range(2)]
         din = [(torch.empty_like(X), torch.empty_like(logits), torch.empty_like(dY))
@@ -281,7 +287,7 @@ def run_ours(args, cfg):
                 comp.wait_event(ev["in_ready"][b])
                 if i >= 2:
                     comp.wait_event(ev["out_free"][b])
-                blocks[b].step(din[b][0], din[b][1], din[b][2], W)
+                blocks[b].step(din[b][0], din[b][1], din[b][2], W, Wr)
                 ev["in_free"][b].record(comp)
                 ev["done"][b].record(comp)
                 with torch.cuda.stream(s_out):
@@ -365,6 +371,8 @@ def main():
                     help="override T (small cases for profiler captures)")
     ap.add_argument("--full-ft", action="store_true",
                     help="full fine-tuning: also the base-weight gradients dW1, dW2")
+    ap.add_argument("--train-router", action="store_true",
+                    help="trained router: logits = X Wr^T and its backward in the step")
     ap.add_argument("--cta-pairs", type=int, default=-1,
                     help="1: grouped GEMMs on CTA pairs, 0: single CTAs, "
                          "-1: library default")
@@ -376,7 +384,8 @@ def main():
         cfg["T"] = args.tokens
     T, H, I, E, k, r = (cfg[x] for x in ("T", "H", "I", "E", "k", "r"))
     R = T * k
-    flops = WL.block_flops(T, H, I, E, k, r, full_ft=args.full_ft)["total"]
+    flops = WL.block_flops(T, H, I, E, k, r, full_ft=args.full_ft,
+                           train_router=args.train_router)["total"]
     pk = peaks()
     workload = {"gpt-oss-20b": "gpt-oss-20b-shaped MoE layer fwd+bwd",
                 "qwen3-30b-a3b": "Qwen3-30B-A3B-shaped MoE layer fwd+bwd",
@@ -385,6 +394,8 @@ def main():
                 "tiny": "tiny MoE block fwd+bwd"}[args.config]
     if args.full_ft:
         workload += ", full fine-tuning (base-weight gradients too)"
+    if args.train_router:
+        workload += ", trained router (logits GEMM and router backward in the step)"
     config = {"workload": workload, "T": T, "H": H, "I": I, "E": E, "top_k": k,
               "lora_r": r, "lora_s": cfg["s"], "logits": cfg["logits"],
               "parallelism": "replicas", "l2": "256 MiB memset before each step, "

@@ -200,6 +200,32 @@ MOE_API moe_status_t moe_lora_mlp_bwd_full(const void* dZ2, const void* Xp,
                                    void* dB2, void* dW1, void* dW2, void* ws,
                                    size_t ws_bytes, moe_stream_t stream);
 
+/* ------------------------------------------ trained router (optional)
+ * The pages keep the router frozen by default; these two calls make it
+ * trainable.  moe_router_fwd: logits [T, E] fp32 = X [T, H] bf16 times
+ * Wr [E, H] bf16 transposed (the router's linear layer; fp32 accumulation
+ * on the tensor cores), to feed moe_route_topk.
+ * moe_router_bwd, from the routing-weight gradient dw [T, k] (moe_permute's
+ * optional output) and the routing of the step (topk_w, topk_idx, dest,
+ * expert_offsets): with the kept weights a softmax over the kept logits,
+ *   g[t, j] = w[t, j] (dw[t, j] - sum_i w[t, i] dw[t, i])   (dlogits)
+ *   dWr[e]  = sum over the rows of expert e of g * Xp[row]     [E, H] fp32
+ *   dX[t]   = sum_j dXp[dest[t, j]] + sum_j g[t, j] Wr[topk_idx[t, j]]
+ * dX replaces the plain dX combine (moe_unpermute of dXp with w = NULL): both
+ * sums are accumulated in fp32 and rounded once to bf16.  dWr sums each
+ * expert's rows in order (deterministic).  ws: at least
+ * moe_router_bwd_workspace_bytes(T, k) device bytes.  H a multiple of 16
+ * (>= 64), 1 <= k <= E <= 512; bf16 pointers 16-byte aligned. */
+MOE_API moe_status_t moe_router_fwd(const void* X, const void* Wr, int T, int H, int E,
+                                    float* logits, moe_stream_t stream);
+MOE_API size_t moe_router_bwd_workspace_bytes(int T, int k);
+MOE_API moe_status_t moe_router_bwd(const float* topk_w, const float* dw,
+                                    const int32_t* topk_idx, const int32_t* dest,
+                                    const int32_t* expert_offsets, const void* Xp,
+                                    const void* Wr, const void* dXp, int T, int H, int E,
+                                    int k, void* dX, float* dWr, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
 /* ---------------------------------------------------------------- status
  * moe_get_device_status synchronises `stream`, returns the first device-side
  * error recorded since the last call (MOE_OK if none) and clears it.
@@ -252,7 +278,9 @@ MOE_API void moe_set_cta_pairs(int mode);
 #define MOE_PROF_LORA_GRAD 7
 #define MOE_PROF_TRANSPOSE 8
 #define MOE_PROF_BASE_GRAD 9
-#define MOE_PROF_KINDS 10
+#define MOE_PROF_ROUTER_FWD 10
+#define MOE_PROF_ROUTER_BWD 11
+#define MOE_PROF_KINDS 12
 MOE_API moe_status_t moe_profile_enable(int on);
 MOE_API int moe_profile_collect(int kind, float* ms, int max_n);
 

@@ -19,6 +19,7 @@
 #include "gemm_pair.cuh"
 #include "lora_grad.cuh"
 #include "base_grad.cuh"
+#include "router.cuh"
 
 using namespace moe;
 
@@ -459,6 +460,25 @@ moe_status_t base_grads(const void* dZ1, const void* Xp, const void* dZ2, const 
                             : launch_base_grad_t<192>(tu, tv, g, st);
 }
 
+template <int BN>
+moe_status_t launch_router_logits_t(const void* X, const void* Wr, int T, int H, int E,
+                                    float* logits, cudaStream_t st) {
+  using C = RouterCfg<BN>;
+  CUtensorMap tx, tw;
+  bool ok = tmap_2d(&tx, X, H, T, H * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && tmap_2d(&tw, Wr, H, E, H * 2ull, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return MOE_ERR_CUDA;
+  auto kern = router_logits_kernel<BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_BYTES) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  dim3 grid((T + 127) / 128, (E + BN - 1) / BN);
+  ProfScope prof(MOE_PROF_ROUTER_FWD, st);
+  kern<<<grid, 192, C::SMEM_BYTES, st>>>(tx, tw, T, H, E, logits, g_wait_limit_ns);
+  count_launch();
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -659,6 +679,68 @@ moe_status_t moe_unpermute(const void* Yp, const int32_t* dest, const float* w, 
   unpermute_kernel<<<grid, warps * 32, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(Yp), dest, w, T, H, k,
       static_cast<__nv_bfloat16*>(Y));
+  count_launch();
+  return launch_status();
+}
+
+// ------------------------------------------------------------- trained router
+moe_status_t moe_router_fwd(const void* X, const void* Wr, int T, int H, int E,
+                            float* logits, moe_stream_t stream) {
+  if (T < 0 || H < 64 || (H % 16) || E < 1 || E > 512) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!X || !Wr || !logits) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Wr)) & 15u)
+    return MOE_ERR_INVALID_ARG;
+  if (E <= 16) return launch_router_logits_t<16>(X, Wr, T, H, E, logits, stream);
+  if (E <= 32) return launch_router_logits_t<32>(X, Wr, T, H, E, logits, stream);
+  if (E <= 64) return launch_router_logits_t<64>(X, Wr, T, H, E, logits, stream);
+  if (E <= 128) return launch_router_logits_t<128>(X, Wr, T, H, E, logits, stream);
+  return launch_router_logits_t<256>(X, Wr, T, H, E, logits, stream);
+}
+
+size_t moe_router_bwd_workspace_bytes(int T, int k) {
+  if (T < 0 || k < 1) return 0;
+  return 2 * align256(static_cast<size_t>(T) * k * 4);
+}
+
+moe_status_t moe_router_bwd(const float* w, const float* dw, const int32_t* topk_idx,
+                            const int32_t* dest, const int32_t* expert_offsets,
+                            const void* Xp, const void* Wr, const void* dXp, int T, int H,
+                            int E, int k, void* dX, float* dWr, void* ws, size_t ws_bytes,
+                            moe_stream_t stream) {
+  if (T < 0 || H < 64 || (H % 16) || E < 1 || E > 512 || k < 1 || k > E)
+    return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(T) * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (!dWr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = stream;
+  if (T == 0)
+    return cudaMemsetAsync(dWr, 0, static_cast<size_t>(E) * H * 4, st) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+  if (!w || !dw || !topk_idx || !dest || !expert_offsets || !Xp || !Wr || !dXp || !dX || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(Xp) | reinterpret_cast<uintptr_t>(Wr) |
+       reinterpret_cast<uintptr_t>(dXp) | reinterpret_cast<uintptr_t>(dX)) & 15u)
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_router_bwd_workspace_bytes(T, k)) return MOE_ERR_INVALID_ARG;
+  const int R = T * k;
+  float* g = static_cast<float*>(ws);
+  float* g_row = at<float>(ws, align256(static_cast<size_t>(R) * 4));
+  ProfScope prof(MOE_PROF_ROUTER_BWD, st);
+  const int grid0 = std::min((T + 255) / 256, std::max(1, num_sms()) * 4);
+  router_dlogit_kernel<<<grid0, 256, 0, st>>>(w, dw, dest, T, k, g, g_row);
+  count_launch();
+  moe_status_t s;
+  if ((s = launch_status()) != MOE_OK) return s;
+  router_wgrad_kernel<<<dim3(E, (H + kRouterWCols - 1) / kRouterWCols), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(Xp), g_row, expert_offsets, E, H, R, dWr);
+  count_launch();
+  if ((s = launch_status()) != MOE_OK) return s;
+  const int warps = 8;
+  const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
+  unpermute_kernel<<<grid, warps * 32, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(dXp), dest, nullptr, T, H, k,
+      static_cast<__nv_bfloat16*>(dX), static_cast<const __nv_bfloat16*>(Wr), topk_idx, g, E);
   count_launch();
   return launch_status();
 }

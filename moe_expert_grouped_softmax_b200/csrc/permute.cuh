@@ -167,12 +167,17 @@ __global__ void __launch_bounds__(256)
 constexpr int kCombVec = 4;  // 16-byte vectors per lane per source row
 
 // Y[t] = sum_j (w ? w[t,j] : 1) * Yp[dest[t,j]], fp32 in j order -> bf16.
+// With a trained router (Wr != nullptr) the router's part of dX is added
+// before the one rounding: + sum_j g[t,j] * Wr[idx[t,j]] (Wr [E, H] bf16).
 // One warp per token; kCombVec x k loads in flight per lane.
 __global__ void __launch_bounds__(256)
     unpermute_kernel(const __nv_bfloat16* __restrict__ Yp,
                      const int32_t* __restrict__ dest,
                      const float* __restrict__ w, int T, int H, int k,
-                     __nv_bfloat16* __restrict__ Y) {
+                     __nv_bfloat16* __restrict__ Y,
+                     const __nv_bfloat16* __restrict__ Wr = nullptr,
+                     const int32_t* __restrict__ idx = nullptr,
+                     const float* __restrict__ g = nullptr, int E = 0) {
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const int nvec = H >> 3;
@@ -206,6 +211,32 @@ __global__ void __launch_bounds__(256)
             acc[u][5] = fmaf(c, bf16_hi(z.z), acc[u][5]);
             acc[u][6] = fmaf(c, bf16_lo(z.w), acc[u][6]);
             acc[u][7] = fmaf(c, bf16_hi(z.w), acc[u][7]);
+          }
+        }
+      }
+      if (Wr != nullptr) {
+        for (int j = 0; j < k; ++j) {
+          const int e = idx[static_cast<size_t>(t) * k + j];
+          if (e < 0 || e >= E) {
+            if (lane == 0) set_status(5);
+            continue;
+          }
+          const float c = g[static_cast<size_t>(t) * k + j];
+          const char* wrow = reinterpret_cast<const char*>(Wr + static_cast<size_t>(e) * H);
+#pragma unroll
+          for (int u = 0; u < kCombVec; ++u) {
+            const int v = v0 + 32 * u;
+            if (v < nvec) {
+              const uint4 z = *reinterpret_cast<const uint4*>(wrow + 16 * static_cast<size_t>(v));
+              acc[u][0] = fmaf(c, bf16_lo(z.x), acc[u][0]);
+              acc[u][1] = fmaf(c, bf16_hi(z.x), acc[u][1]);
+              acc[u][2] = fmaf(c, bf16_lo(z.y), acc[u][2]);
+              acc[u][3] = fmaf(c, bf16_hi(z.y), acc[u][3]);
+              acc[u][4] = fmaf(c, bf16_lo(z.z), acc[u][4]);
+              acc[u][5] = fmaf(c, bf16_hi(z.z), acc[u][5]);
+              acc[u][6] = fmaf(c, bf16_lo(z.w), acc[u][6]);
+              acc[u][7] = fmaf(c, bf16_hi(z.w), acc[u][7]);
+            }
           }
         }
       }

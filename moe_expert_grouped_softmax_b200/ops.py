@@ -26,12 +26,13 @@ EXPORTS = [
     "moe_lora_mlp_fwd", "moe_lora_mlp_bwd", "moe_lora_mlp_bwd_full", "moe_get_device_status",
     "moe_status_string", "moe_set_wait_limit_ns", "moe_test_inject_stall",
     "moe_set_cta_pairs", "moe_kernel_launches", "moe_profile_enable",
+    "moe_router_fwd", "moe_router_bwd_workspace_bytes", "moe_router_bwd",
     "moe_profile_collect",
 ]
 
 PROF_KINDS = {"route": 0, "permute": 1, "gate_up_fwd": 2, "down_fwd": 3,
               "unpermute": 4, "down_bwd": 5, "gate_up_bwd": 6, "lora_grad": 7,
-              "transpose": 8, "base_grad": 9}
+              "transpose": 8, "base_grad": 9, "router_fwd": 10, "router_bwd": 11}
 
 
 class MoeError(RuntimeError):
@@ -59,6 +60,12 @@ def lib():
         L.moe_permute.restype = I
         L.moe_unpermute.argtypes = [P, P, P, I, I, I, P, P]
         L.moe_unpermute.restype = I
+        L.moe_router_fwd.argtypes = [P, P, I, I, I, P, P]
+        L.moe_router_fwd.restype = I
+        L.moe_router_bwd_workspace_bytes.argtypes = [I, I]
+        L.moe_router_bwd_workspace_bytes.restype = S
+        L.moe_router_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, P, P, P, S, P]
+        L.moe_router_bwd.restype = I
         L.moe_saved_bytes.argtypes = [I, I, I, I]
         L.moe_saved_bytes.restype = S
         L.moe_saved_part_offset.argtypes = [I, I, I, I, I]
@@ -233,6 +240,44 @@ def permute(X, dest, scale=None, Zp=None, out=None, dw=None):
     return (out, dw) if Zp is not None else out
 
 
+def router_fwd(X, Wr, out=None):
+    """Trained router: logits [T, E] fp32 = X Wr^T."""
+    T, H = X.shape
+    E = Wr.shape[0]
+    _need(X, torch.bfloat16, (T, H), "X")
+    _need(Wr, torch.bfloat16, (E, H), "Wr")
+    if out is None:
+        out = torch.empty((T, E), dtype=torch.float32, device=X.device)
+    _need(out, torch.float32, (T, E), "logits")
+    _check(lib().moe_router_fwd(_p(X), _p(Wr), T, H, E, _p(out), _stream()), "moe_router_fwd")
+    return out
+
+
+def router_bwd(w, dw, idx, dest, offsets, Xp, Wr, dXp, out=None, ws=None):
+    """Trained router backward: returns (dX with the router's part, dWr fp32)."""
+    T, k = w.shape
+    E, H = Wr.shape
+    for t, dt, sh, n in ((w, torch.float32, (T, k), "w"), (dw, torch.float32, (T, k), "dw"),
+                         (idx, torch.int32, (T, k), "idx"), (dest, torch.int32, (T, k), "dest"),
+                         (offsets, torch.int32, (E + 1,), "offsets"),
+                         (Xp, torch.bfloat16, (T * k, H), "Xp"), (Wr, torch.bfloat16, (E, H), "Wr"),
+                         (dXp, torch.bfloat16, (T * k, H), "dXp")):
+        _need(t, dt, sh, n)
+    dev = Xp.device
+    if out is None:
+        out = (torch.empty((T, H), dtype=torch.bfloat16, device=dev),
+               torch.empty((E, H), dtype=torch.float32, device=dev))
+    dX, dWr = out
+    nb = int(lib().moe_router_bwd_workspace_bytes(T, k))
+    if ws is None or ws.numel() < nb:
+        ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev)
+    _check(lib().moe_router_bwd(_p(w), _p(dw), _p(idx), _p(dest), _p(offsets), _p(Xp), _p(Wr),
+                                _p(dXp), T, H, E, k, _p(dX), _p(dWr), _p(ws), ws.numel(),
+                                _stream()),
+           "moe_router_bwd")
+    return dX, dWr
+
+
 def unpermute(Yp, dest, w=None, out=None):
     """a5 / a10: Y[t] = sum_j w[t, j] Yp[dest[t, j]]."""
     T, k = dest.shape
@@ -328,7 +373,8 @@ class MoeBlock:
     gate_up backward, LoRA gradients and the dX combine (with ``full_ft``, also
     the base-weight gradients dW1, dW2 of full fine-tuning)."""
 
-    def __init__(self, T, H, I, E, k, r, s, device="cuda", with_dw=False, full_ft=False):
+    def __init__(self, T, H, I, E, k, r, s, device="cuda", with_dw=False, full_ft=False,
+                 train_router=False):
         self.T, self.H, self.I, self.E, self.k, self.r, self.s = T, H, I, E, k, r, s
         self.R = R = T * k
         self.with_dw = with_dw
@@ -355,12 +401,24 @@ class MoeBlock:
         self.dA2 = torch.empty((E, r, I), dtype=bf, device=dev)
         self.dB2 = torch.empty((E, H, r), dtype=bf, device=dev)
         self.full_ft = full_ft
+        # trained router: logits = X Wr^T on the device; dw, dlogits -> dWr and
+        # the router's part of dX (needs the routing-weight gradient)
+        self.train_router = train_router
+        if train_router:
+            self.with_dw = True
+            self.dw = torch.empty((T, k), dtype=f32, device=dev)
+            self.logits = torch.empty((T, E), dtype=f32, device=dev)
+            self.dWr = torch.empty((E, H), dtype=f32, device=dev)
+            self.router_ws = torch.empty(max(1, int(lib().moe_router_bwd_workspace_bytes(T, k))),
+                                         dtype=torch.uint8, device=dev)
         self.dW1 = torch.empty((E, 2 * I, H), dtype=bf, device=dev) if full_ft else None
         self.dW2 = torch.empty((E, H, I), dtype=bf, device=dev) if full_ft else None
         self.ws = torch.empty(max(1, workspace_bytes(R, E, H, I, r)), dtype=torch.uint8,
                               device=dev)
 
-    def forward(self, X, logits, W):
+    def forward(self, X, logits, W, Wr=None):
+        if self.train_router:
+            logits = router_fwd(X, Wr, out=self.logits)
         route_topk(logits, self.k, out=(self.idx, self.w, self.counts, self.offsets,
                                         self.dest), ws=self.route_ws)
         permute(X, self.dest, out=self.Xp)
@@ -368,7 +426,7 @@ class MoeBlock:
         unpermute(self.Z2, self.dest, self.w, out=self.Y)
         return self.Y
 
-    def backward(self, dY, W):
+    def backward(self, dY, W, Wr=None):
         if self.with_dw:
             permute(dY, self.dest, scale=self.w, Zp=self.Z2, out=self.dZ2, dw=self.dw)
         else:
@@ -376,9 +434,15 @@ class MoeBlock:
         lora_mlp_bwd(self.dZ2, self.Xp, self.offsets, *W, self.s, self.saved,
                      out=(self.dXp, self.dA1, self.dB1, self.dA2, self.dB2), ws=self.ws,
                      base_out=(self.dW1, self.dW2) if self.full_ft else None)
-        unpermute(self.dXp, self.dest, None, out=self.dX)
+        if self.train_router:
+            router_bwd(self.w, self.dw, self.idx, self.dest, self.offsets, self.Xp, Wr,
+                       self.dXp, out=(self.dX, self.dWr), ws=self.router_ws)
+        else:
+            unpermute(self.dXp, self.dest, None, out=self.dX)
         return self.dX
 
-    def step(self, X, logits, dY, W):
-        self.forward(X, logits, W)
-        self.backward(dY, W)
+    def step(self, X, logits, dY, W, Wr=None):
+        """One fwd+bwd; with a trained router, ``Wr`` [E, H] bf16 replaces
+        ``logits`` (which may then be None)."""
+        self.forward(X, logits, W, Wr)
+        self.backward(dY, W, Wr)

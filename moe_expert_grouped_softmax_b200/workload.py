@@ -38,9 +38,16 @@ def base_grad_flops(R, H, I):
     return 2 * R * (2 * I * H + H * I)
 
 
-def block_flops(T, H, I, E, k, r, full_ft=False):
+def router_flops(T, H, E, k):
+    """Trained router: logits X Wr^T (2 T E H), and from the k kept logits per
+    token dWr (2 T k H) and the router's part of dX (2 T k H)."""
+    return 2 * T * E * H + 4 * T * k * H
+
+
+def block_flops(T, H, I, E, k, r, full_ft=False, train_router=False):
     """Forward + backward algorithmic FLOPs of the block (base frozen, or with
-    the base-weight gradients when ``full_ft``)."""
+    the base-weight gradients when ``full_ft``; with the router's when
+    ``train_router``)."""
     R = T * k
     fwd = (split_lora_proj_flops(R, H, 2 * I, r)
            + split_lora_proj_flops(R, I, H, r))
@@ -48,7 +55,8 @@ def block_flops(T, H, I, E, k, r, full_ft=False):
     # dA 2rm, dB 2nr
     def bwd(m, n):
         return 2 * R * (m * n + n * r + r * m + r * m + n * r)
-    extra = base_grad_flops(R, H, I) if full_ft else 0
+    extra = (base_grad_flops(R, H, I) if full_ft else 0) + (
+        router_flops(T, H, E, k) if train_router else 0)
     return dict(fwd=fwd, bwd=bwd(H, 2 * I) + bwd(I, H) + extra,
                 total=fwd + bwd(H, 2 * I) + bwd(I, H) + extra,
                 base_gemm=2 * R * (H * 2 * I + I * H) * 2)
