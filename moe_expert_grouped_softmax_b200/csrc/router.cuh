@@ -10,6 +10,7 @@
 #pragma once
 
 #include "gemm.cuh"
+#include "permute.cuh"
 
 namespace moe {
 
@@ -182,33 +183,54 @@ __global__ void router_dlogit_kernel(const float* __restrict__ w, const float* _
 }
 
 // ----------------------------------------------------------- weight gradient
-// dWr[e, c] = sum over the rows of expert e (in order) of g_row * Xp[row, c],
-// fp32.  One CTA per (expert, 512-column chunk); each thread owns two
-// adjacent columns, so every row is read as one coalesced 1 KB segment.
-constexpr int kRouterWCols = 512;
+// dWr[e, c] = sum over the rows of expert e of g_row * Xp[row, c], fp32.
+// One CTA per (expert, 256-column chunk), 8 warps: warp w takes rows
+// a + w, a + w + 8, ... with each lane owning 8 adjacent columns (one 16-byte
+// load per row), and the 8 partial sums are added in warp order at the end,
+// so the result does not depend on timing.
+constexpr int kRouterWCols = 256;
 __global__ void __launch_bounds__(256)
     router_wgrad_kernel(const __nv_bfloat16* __restrict__ Xp, const float* __restrict__ g_row,
                         const int32_t* __restrict__ offsets, int E, int H, int R,
                         float* __restrict__ dWr) {
+  __shared__ float part[8][kRouterWCols];
   const int e = blockIdx.x;
-  const int c = blockIdx.y * kRouterWCols + 2 * threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c0 = blockIdx.y * kRouterWCols + 8 * lane;
   int a = offsets[e], b = offsets[e + 1];
   if (a < 0 || b > R || a > b) {
     if (threadIdx.x == 0) set_status(5);
     a = b = 0;
   }
-  if (c >= H) return;
-  float acc0 = 0.f, acc1 = 0.f;
-  const __nv_bfloat16* col = Xp + c;
-#pragma unroll 8
-  for (int row = a; row < b; ++row) {
-    const float gr = g_row[row];
-    const uint32_t x = *reinterpret_cast<const uint32_t*>(col + static_cast<size_t>(row) * H);
-    acc0 = fmaf(gr, bf16_lo(x), acc0);
-    acc1 = fmaf(gr, bf16_hi(x), acc1);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  if (c0 < H) {  // H is a multiple of 16: the 8 columns are all in range
+    const __nv_bfloat16* col = Xp + c0;
+#pragma unroll 4
+    for (int row = a + warp; row < b; row += 8) {
+      const float gr = g_row[row];
+      const uint4 x = ld_nc_v4(col + static_cast<size_t>(row) * H);
+      acc[0] = fmaf(gr, bf16_lo(x.x), acc[0]);
+      acc[1] = fmaf(gr, bf16_hi(x.x), acc[1]);
+      acc[2] = fmaf(gr, bf16_lo(x.y), acc[2]);
+      acc[3] = fmaf(gr, bf16_hi(x.y), acc[3]);
+      acc[4] = fmaf(gr, bf16_lo(x.z), acc[4]);
+      acc[5] = fmaf(gr, bf16_hi(x.z), acc[5]);
+      acc[6] = fmaf(gr, bf16_lo(x.w), acc[6]);
+      acc[7] = fmaf(gr, bf16_hi(x.w), acc[7]);
+    }
   }
-  dWr[static_cast<size_t>(e) * H + c] = acc0;
-  if (c + 1 < H) dWr[static_cast<size_t>(e) * H + c + 1] = acc1;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[warp][8 * lane + i] = acc[i];
+  __syncthreads();
+  const int c = blockIdx.y * kRouterWCols + threadIdx.x;
+  if (c < H) {
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += part[w][threadIdx.x];
+    dWr[static_cast<size_t>(e) * H + c] = sum;
+  }
 }
 
 }  // namespace moe
