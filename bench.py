@@ -463,8 +463,10 @@ def main():
                                  "traffic": traffic.get(kk)}
     hb = WL.hbm_bytes(T, H, E, k)
     hb["lora_grad"] = R * (H + 2 * I + I + H) * 2 + 4 * r * R * 2 + E * r * (3 * H + 3 * I) * 2
+    # rank-r passes of the pair backward: dZ2 (K = H) and dZ1 (K = 2I), mean per launch
+    hb["rank_down"] = (R * (H + 2 * I) * 2 + E * r * (H + 2 * I) * 2 + 2 * 2 * R * r * 2) // 2
     mem = {}
-    for kk in ("permute", "unpermute", "route", "lora_grad"):
+    for kk in ("permute", "unpermute", "route", "lora_grad", "rank_down"):
         if kk in kern:
             # permute / unpermute run twice per step with the same bytes
             gbs = hb[kk] / (kern[kk]["avg_ms"] / 1e3) / 1e9

@@ -253,10 +253,12 @@ MOE_API unsigned long long moe_kernel_launches(void);
  * the next moe_lora_mlp_fwd / moe_lora_mlp_bwd call): mode > 0 runs them on
  * CTA pairs (256-row tiles on the 2-SM tensor-core instruction), mode == 0
  * on single CTAs (128-row tiles), mode < 0 (the default) chooses per GEMM:
- * a forward GEMM runs on pairs when the mean rows per expert R / E is at
- * least 768 (little padding on each expert's ragged last 256-row tile) and
- * its K is at least 1024 (H for gate_up, I for down); the backward GEMMs run
- * on single CTAs.  All compute the same result. */
+ * pairs when the mean rows per expert R / E is at least 768 (little padding
+ * on each expert's ragged last 256-row tile) and the GEMM's K is at least
+ * 1024 (H for gate_up forward and down backward, I for down forward, 2I for
+ * gate_up backward).  A backward GEMM on pairs takes its rank-r product
+ * (s dZ2 B2 or s dZ1 B1) from a separate memory-bound pass.  All compute the
+ * same result. */
 MOE_API void moe_set_cta_pairs(int mode);
 
 /* Benchmark hook (not thread-safe; for measurement only).
@@ -276,11 +278,12 @@ MOE_API void moe_set_cta_pairs(int mode);
 #define MOE_PROF_DOWN_BWD 5
 #define MOE_PROF_GATE_UP_BWD 6
 #define MOE_PROF_LORA_GRAD 7
-#define MOE_PROF_TRANSPOSE 8
+#define MOE_PROF_TRANSPOSE 8   /* the factor operand copies (one launch) */
 #define MOE_PROF_BASE_GRAD 9
 #define MOE_PROF_ROUTER_FWD 10
 #define MOE_PROF_ROUTER_BWD 11
-#define MOE_PROF_KINDS 12
+#define MOE_PROF_RANK_DOWN 12
+#define MOE_PROF_KINDS 13
 MOE_API moe_status_t moe_profile_enable(int on);
 MOE_API int moe_profile_collect(int kind, float* ms, int max_n);
 

@@ -7,10 +7,12 @@
 // halves of N/2), so every SM moves a third less operand data per FLOP
 // than the single-CTA 128-row tile, through shared memory as well as from L2.
 // Forward (K-major B): the halves are row blocks of W and of the factor.
-// Backward (MN-major B, W read in place as [K, N]): 32-column atoms with the
-// 64-byte swizzle, one TMA box of 32 columns x 64 K-rows each; the r factor
-// columns (B2 or B1, zero-padded to a multiple of 32 columns when r = 16) fill
-// whole atoms next to the weight columns, so BN = 256 - round_up(r, 32).  The even CTA ("leader") issues the
+// Backward (MN-major B, W read in place as [K, N]): the rank-r
+// down-products (s dZ2 B2, s dZ1 B1) come from their own pass, so the B
+// operand is weight columns only, BN = 256 as four 64-column atoms (128-byte
+// swizzle, 64 x 64 TMA boxes, two per CTA); each tile's up-projection
+// operands (its 256 rows of the rank-r product and the BN rows of the
+// K-major up factor) are loaded by TMA and accumulated after the mainloop.  The even CTA ("leader") issues the
 // MMAs, which read both CTAs' shared memory and write both CTAs' TMEM (each
 // holds its 128 rows x N columns).  The split-LoRA schedule is the one of the
 // single-CTA kernel: rank-r down-projection inside the mainloop MMA,
@@ -62,9 +64,9 @@ struct PairCfg {
   static constexpr bool kSwiGLU = (MODE == kGateUpFwd);
   static constexpr bool kBMN = (MODE == kDownBwd || MODE == kGateUpBwd);
   static constexpr int BM = 128, BK = 64;           // rows per CTA
-  // factor columns in the fused B operand (MN-major: whole 32-column atoms)
-  static constexpr int FPAD = kBMN ? (RK + 31) / 32 * 32 : RK;
-  static constexpr int NMMA = BN + FPAD;            // N of the fused MMA
+  // forward: the down factor's r rows ride in the B operand (N = BN + r);
+  // backward: weight columns only
+  static constexpr int NMMA = kBMN ? BN : BN + RK;  // N of the mainloop MMA
   static constexpr int NH = NMMA / 2;               // B rows per CTA
   static constexpr int HALF = BN / 2;
   // B segments of each CTA (rows of N): SwiGLU: CTA0 = gate HALF + up U0,
@@ -79,6 +81,9 @@ struct PairCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int LB_BYTES = HALF * RK * 2;    // this CTA's half of LB
   static constexpr int XA_BYTES = BM * RK * 2;
+  // up-projection operands one CTA loads per tile (backward: the rank-r
+  // product rows too)
+  static constexpr int UP_BYTES = kBMN ? LB_BYTES + XA_BYTES : LB_BYTES;
   static constexpr int MISC_BYTES = 512 + 8 * 520;  // barriers, counts, tables
   static constexpr int FIXED = 2 * LB_BYTES + 2 * XA_BYTES + MISC_BYTES;
   static constexpr int NS_FIT = (kSmemOptin - 1024 - FIXED) / STAGE_BYTES;
@@ -91,17 +96,17 @@ struct PairCfg {
   static constexpr int ACC_STRIDE = 256;
   static constexpr int EPI_WARPS = gemm_epi_warps(MODE);
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  // MN-major B: one 32-column x BK-row box (64-byte swizzle) per atom
-  static constexpr int MN_COLS = 32;
+  // MN-major B: one 64-column x BK-row box (128-byte swizzle) per atom
+  static constexpr int MN_COLS = 64;
   static constexpr int MN_BOX = MN_COLS * BK * 2;
-  static_assert(!kBMN || (W0 % MN_COLS == 0 && W1 % MN_COLS == 0 && NMMA == 256),
-                "MN-major halves in whole 32-column atoms");
+  static_assert(!kBMN || (NH % MN_COLS == 0 && NMMA == 256),
+                "MN-major halves in whole 64-column atoms");
   static_assert(NS >= 3, "not enough shared memory for three stages");
   static_assert(SMEM_BYTES <= kSmemOptin, "shared memory over the opt-in limit");
   static_assert(NMMA <= ACC_STRIDE && NMMA % 16 == 0, "MMA N = BN + r");
   static_assert(BN % 16 == 0 && NH % 8 == 0, "8-row operand atoms");
   static_assert(!kSwiGLU || (U0 % 8 == 0 && U1 % 8 == 0 && U1 > 0), "SwiGLU segments");
-  static_assert(W1 % 8 == 0 && W1 > 0, "plain segments");
+  static_assert(kBMN || (W1 % 8 == 0 && W1 > 0), "plain segments");
 };
 
 // Host-visible box heights of the weight segments (rows), for the maps.
@@ -217,12 +222,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         if (!mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
-        if (leader) mbar_arrive_expect_tx(&lb_full[b], 2 * C::LB_BYTES);
+        if (leader) mbar_arrive_expect_tx(&lb_full[b], 2 * C::UP_BYTES);
         // this CTA's half of the up-projection factor: output columns
         // [rank * BN/2, (rank + 1) * BN/2) of the tile
         const int lb_row = kSwiGLU ? e * args.lb_rows + (rank ? args.I : 0) + nt * HALF
                                    : e * args.lb_rows + nt * BN + static_cast<int>(rank) * HALF;
         tma_load_2d_pair(sLB + b * C::LB_BYTES, &tmLB, lead(&lb_full[b]), 0, lb_row);
+        // backward: this CTA's 128 rows of the rank-r product (K-major)
+        if constexpr (kBMN)
+          tma_load_2d_pair(sXA + b * C::XA_BYTES, &tmLA, lead(&lb_full[b]), 0, row0);
         ++n_lb;
         for (int kt = 0; kt < k_iters; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, wait_ns)) { ok = false; break; }
@@ -233,19 +241,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           tma_load_2d_pair(st, &tmA, fb, kx, row0);
           if constexpr (kBMN) {
-            // W [K, N] in place: this CTA's weight columns, then (CTA1) the
-            // factor's columns, one 32-column atom per box
+            // W [K, N] in place: this CTA's half of the tile's weight
+            // columns, one 64-column atom per box
             constexpr int A = C::MN_COLS;
-            const int nw = rank ? C::W1 : C::W0;
-            const int n0 = nt * BN + (rank ? C::W0 : 0);
+            const int n0 = nt * BN + static_cast<int>(rank) * C::NH;
             const int krow = e * args.b_rows + kx;
-            for (int i = 0; i < nw / A; ++i)
-              tma_load_2d_pair(sb + i * C::MN_BOX, &tmW0, fb, n0 + A * i, krow);
-            if (rank) {
 #pragma unroll
-              for (int i = 0; i < C::FPAD / A; ++i)
-                tma_load_2d_pair(sb + (nw / A + i) * C::MN_BOX, &tmLA, fb, A * i, krow);
-            }
+            for (int i = 0; i < C::NH / A; ++i)
+              tma_load_2d_pair(sb + i * C::MN_BOX, &tmW0, fb, n0 + A * i, krow);
           } else if (kSwiGLU) {
             const int gate = e * args.b_rows + nt * HALF;
             const int up = e * args.b_rows + args.I + nt * HALF;
@@ -301,12 +304,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         __syncwarp();
       };
       const uint64_t a_desc0 = smem_desc(smem_u32(sStage), 16, 1024, kLayoutSW128);
-      // MN-major: LBO = next 32-column atom, SBO = next 8 K-rows (8 x 64 B)
+      // MN-major: LBO = next 64-column atom, SBO = next 8 K-rows (8 x 128 B)
       const uint64_t b_desc0 =
-          kBMN ? smem_desc(smem_u32(sStage) + C::A_BYTES, C::MN_BOX, 512, kLayoutSW64)
+          kBMN ? smem_desc(smem_u32(sStage) + C::A_BYTES, C::MN_BOX, 1024, kLayoutSW128)
                : smem_desc(smem_u32(sStage) + C::A_BYTES, 16, 1024, kLayoutSW128);
       constexpr uint64_t kStageInc = C::STAGE_BYTES >> 4;
-      constexpr uint64_t kBStep = kBMN ? (1024 >> 4) : (32 >> 4);  // 16 K
+      constexpr uint64_t kBStep = kBMN ? (2048 >> 4) : (32 >> 4);  // 16 K
       int stage = 0;
       uint64_t soff = 0;
       uint32_t phase = 0;
@@ -351,6 +354,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           }
         }
         if (!ok) break;
+        if constexpr (kBMN) {
+          // backward: the tile's up-projection operands came by TMA
+          if (!warp_wait(&lb_full[b], use, s_abort, wait_ns)) { ok = false; break; }
+          up_when_ready(b);
+          continue;
+        }
         if (elect_one()) umma_commit_pair_mc(&lora_full[b], kBoth);
         __syncwarp();
         if (pending >= 0) {
@@ -394,7 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       const int grow = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * C::BM + row_in_tile;
       const bool rvalid = grow < s_off[e + 1];
       const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
-      if (ehalf == 0) {  // rank-r hand-off: the first four epilogue warps
+      if (!kBMN && ehalf == 0) {  // rank-r hand-off: the first four epilogue warps
         if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
         tc_fence_after();
         epi_rank_handoff<RK>(args, t_acc + BN, sXA + b * C::XA_BYTES, row_in_tile, nt,
@@ -430,7 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
     } else {
       drain_wait_cluster(peer_done, 0, wait_ns);
       drain_pair_copies(full, C::NS, C::STAGE_BYTES, s_issued[0], s_issued[2], wait_ns);
-      drain_pair_copies(lb_full, 2, C::LB_BYTES, s_issued[1], s_issued[3], wait_ns);
+      drain_pair_copies(lb_full, 2, C::UP_BYTES, s_issued[1], s_issued[3], wait_ns);
       mbar_arrive_cluster(mapa_shared(smem_u32(drained), 1));
     }
   }

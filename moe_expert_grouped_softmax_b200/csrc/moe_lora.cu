@@ -20,6 +20,7 @@
 #include "lora_grad.cuh"
 #include "base_grad.cuh"
 #include "router.cuh"
+#include "rank_down.cuh"
 
 using namespace moe;
 
@@ -61,19 +62,16 @@ std::atomic<unsigned long long> g_launches{0};  // kernels launched by the libra
 inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 int g_stall_test = 0;                      // testing hook, see moe_test_inject_stall
 int g_cta_pairs = -1;                      // grouped GEMMs on CTA pairs: <0 auto
-// Automatic choice (measured): the forward GEMMs run on CTA pairs when the
-// mean rows per expert fill at least three 256-row tiles (little padding on
-// each expert's ragged last tile) and K is long enough (16 k-steps) for the
-// per-tile hand-offs to stay hidden.  The backward GEMMs stay on single CTAs:
-// their MN-major weight operand needs 32-column atoms in the pair kernel,
-// which pads the fused factor columns, and with the 256-row padding that
-// costs more than the pair saves.
+// Automatic choice (measured): a GEMM runs on CTA pairs when the mean rows
+// per expert fill at least three 256-row tiles (little padding on each
+// expert's ragged last tile) and K is long enough (16 k-steps) for the
+// per-tile work around the mainloop to stay hidden.
 constexpr int kPairMinRowsPerExpert = 768;
 constexpr int kPairMinK = 1024;
 bool use_pairs(int R, int E, int K, bool backward) {
+  (void)backward;
   if (g_cta_pairs >= 0) return g_cta_pairs > 0;
-  return !backward &&
-         static_cast<int64_t>(R) >= static_cast<int64_t>(kPairMinRowsPerExpert) * E &&
+  return static_cast<int64_t>(R) >= static_cast<int64_t>(kPairMinRowsPerExpert) * E &&
          K >= kPairMinK;
 }
 
@@ -248,14 +246,12 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* LA, const v
   CUtensorMap ta, tw0, tw1, tw2, tla, tlb;
   bool ok = tmap_2d(&ta, A, K, args.R, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if constexpr (C::kBMN) {
-    // W [E * K, N] in place and the down-projection factor [E * K, FPAD]
-    // (zero-padded copy when r < FPAD), 32-column x 64-row boxes (64-byte
-    // swizzle)
+    // W [E * K, N] in place, 64-column x 64-row boxes (128-byte swizzle); LA
+    // is the rank-r product [R, r] (row-major), one box per CTA and tile
     const uint64_t N = static_cast<uint64_t>(args.N);
     ok = ok && tmap_2d(&tw0, W, N, EU * args.b_rows, N * 2, C::MN_COLS, 64,
-                       CU_TENSOR_MAP_SWIZZLE_64B);
-    ok = ok && tmap_2d(&tla, LA, C::FPAD, EU * args.b_rows, C::FPAD * 2ull, C::MN_COLS, 64,
-                       CU_TENSOR_MAP_SWIZZLE_64B);
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, LA, RK, args.R, RK * 2ull, RK, C::BM, lora_swizzle(RK));
     tw1 = tw0;
     tw2 = tw0;
   } else {
@@ -288,11 +284,9 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* LA, const v
 }
 
 // Tile width of the CTA-pair kernels: N = BN + r fills the 256-column MMA
-// (forward, K-major factor rows); backward: BN + round_up(r, 32) = 256.
+// (forward, K-major factor rows); backward: weight columns only, BN = 256.
 constexpr bool pair_backward(int mode) { return mode == kDownBwd || mode == kGateUpBwd; }
-constexpr int pair_bn(int mode, int r) {
-  return 256 - (pair_backward(mode) ? (r + 31) / 32 * 32 : r);
-}
+constexpr int pair_bn(int mode, int r) { return pair_backward(mode) ? 256 : 256 - r; }
 
 template <int MODE>
 moe_status_t launch_pair(int r, const void* A, const void* W, const void* LA,
@@ -334,7 +328,7 @@ void saved_layout(int R, int H, int I, int r, size_t off[5]) {
 }
 
 // Backward scratch parts.
-void bwd_layout(int R, int E, int H, int I, int r, size_t off[8]) {
+void bwd_layout(int R, int E, int H, int I, int r, size_t off[10]) {
   const size_t dz1 = static_cast<size_t>(R) * 2 * I * 2;
   const size_t vt = static_cast<size_t>(r) * ld_rank(R) * 2;
   off[0] = 0;                                                  // dZ1 [R, 2I]
@@ -344,7 +338,9 @@ void bwd_layout(int R, int E, int H, int I, int r, size_t off[8]) {
   off[4] = off[3] + align256(static_cast<size_t>(E) * H * 64 * 2);     // A2t [E, I, r]
   off[5] = off[4] + align256(static_cast<size_t>(E) * I * r * 2);      // B1p [E*2I, <= 64]
   off[6] = off[5] + align256(static_cast<size_t>(E) * 2 * I * 64 * 2);  // A1t [E, H, r]
-  off[7] = off[6] + align256(static_cast<size_t>(E) * H * r * 2);
+  off[7] = off[6] + align256(static_cast<size_t>(E) * H * r * 2);     // s dZ2 B2 [R, r]
+  off[8] = off[7] + align256(static_cast<size_t>(R) * r * 2);          // s dZ1 B1 [R, r]
+  off[9] = off[8] + align256(static_cast<size_t>(R) * r * 2);
 }
 
 template <typename T>
@@ -477,6 +473,44 @@ moe_status_t launch_router_logits_t(const void* X, const void* Wr, int T, int H,
   kern<<<grid, 192, C::SMEM_BYTES, st>>>(tx, tw, T, H, E, logits, g_wait_limit_ns);
   count_launch();
   return launch_status();
+}
+
+template <int RK>
+moe_status_t launch_rank_down_t(const void* U, const void* F, int K, const int32_t* offsets,
+                                int E, int R, float s, void* out_rm, void* out_t,
+                                cudaStream_t st) {
+  using C = RankDownCfg<RK>;
+  CUtensorMap tu, tf;
+  const uint64_t EU = static_cast<uint64_t>(E);
+  bool ok = tmap_2d(&tu, U, K, R, K * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && tmap_2d(&tf, F, RK, EU * K, RK * 2ull, RK, 64, lora_swizzle(RK));
+  if (!ok) return MOE_ERR_CUDA;
+  RankDownArgs a{};
+  a.offsets = offsets;
+  a.E = E; a.R = R; a.K = K; a.k_rows = K; a.s = s;
+  a.out_rm = static_cast<__nv_bfloat16*>(out_rm);
+  a.out_t = static_cast<__nv_bfloat16*>(out_t);
+  a.ld_t = ld_rank(R);
+  a.wait_ns = g_wait_limit_ns;
+  auto kern = rank_down_kernel<RK>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_BYTES) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int grid = static_cast<int>(std::min<long long>(num_sms(), R / 128 + E));
+  if (grid <= 0) return MOE_OK;
+  ProfScope prof(MOE_PROF_RANK_DOWN, st);
+  kern<<<grid, 192, C::SMEM_BYTES, st>>>(tu, tf, a);
+  count_launch();
+  return launch_status();
+}
+
+// s U_e F[e] per expert, row-major [R, r] and transposed [r, ldR].
+moe_status_t rank_down(int r, const void* U, const void* F, int K, const int32_t* offsets,
+                       int E, int R, float s, void* out_rm, void* out_t, cudaStream_t st) {
+  if (r == 16) return launch_rank_down_t<16>(U, F, K, offsets, E, R, s, out_rm, out_t, st);
+  if (r == 32) return launch_rank_down_t<32>(U, F, K, offsets, E, R, s, out_rm, out_t, st);
+  if (r == 64) return launch_rank_down_t<64>(U, F, K, offsets, E, R, s, out_rm, out_t, st);
+  return MOE_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -762,9 +796,9 @@ size_t moe_saved_part_offset(int R, int H, int I, int r, int part) {
 
 size_t moe_workspace_bytes(int R, int E, int H, int I, int r) {
   if (R < 0 || E <= 0 || H <= 0 || I <= 0 || r <= 0) return 0;
-  size_t off[8];
+  size_t off[10];
   bwd_layout(R, E, H, I, r, off);
-  return off[7];
+  return off[9];
 }
 
 // ------------------------------------------------------------------ forward
@@ -890,7 +924,7 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     return MOE_ERR_INVALID_ARG;
   if (saved_bytes < moe_saved_bytes(R, H, I, r)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_workspace_bytes(R, E, H, I, r)) return MOE_ERR_INVALID_ARG;
-  size_t so[5], wo[8];
+  size_t so[5], wo[10];
   saved_layout(R, H, I, r, so);
   bwd_layout(R, E, H, I, r, wo);
   const __nv_bfloat16* Z1 = at<__nv_bfloat16>(saved, so[0]);
@@ -913,16 +947,18 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
   // up-projection factors A2, A1 transposed to K-major (both kernels).
   const bool pair_down = use_pairs(R, E, H, true);
   const bool pair_gate_up = use_pairs(R, E, 2 * I, true);
-  const int wdown = pair_down ? 32 : 64, wgate = pair_gate_up ? 32 : 64;
+  // (the CTA-pair backward reads B2, B1 in place in its rank-r pass)
   FactorPrep prep;
-  if (r < wdown) {
+  if (r < 64 && !pair_down) {
     B2p = at<__nv_bfloat16>(ws, wo[3]);
-    prep.pad(B2, const_cast<void*>(B2p), 1ll * E * H, r, wdown);
+    prep.pad(B2, const_cast<void*>(B2p), 1ll * E * H, r, 64);
   }
-  if (r < wgate) {
+  if (r < 64 && !pair_gate_up) {
     B1p = at<__nv_bfloat16>(ws, wo[5]);
-    prep.pad(B1, const_cast<void*>(B1p), 2ll * E * I, r, wgate);
+    prep.pad(B1, const_cast<void*>(B1p), 2ll * E * I, r, 64);
   }
+  __nv_bfloat16* dzb2_rm = at<__nv_bfloat16>(ws, wo[7]);
+  __nv_bfloat16* dzb1_rm = at<__nv_bfloat16>(ws, wo[8]);
   prep.transpose(A2, A2t, E, r, I);
   prep.transpose(A1, A1t, E, r, H);
   if ((stt = prep.launch(st)) != MOE_OK) return stt;
@@ -937,9 +973,12 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + bn - 1) / bn; g.I = I;
     g.b_rows = H; g.lb_rows = I; g.s = s;
     g.out = dZ1; g.ld_out = 2 * I; g.aux = Z1; g.ld_aux = 2 * I;
-    g.lora_t = dzb2; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
     g.stall_test = g_stall_test;
-    if ((stt = launch_pair<kDownBwd>(r, dZ2, W2, B2p, A2t, g, st)) != MOE_OK) return stt;
+    // s dZ2 B2 (both layouts) on its own pass, then the GEMM
+    if ((stt = rank_down(r, dZ2, B2, H, expert_offsets, E, R, s, dzb2_rm, dzb2, st)) != MOE_OK)
+      return stt;
+    if ((stt = launch_pair<kDownBwd>(r, dZ2, W2, dzb2_rm, A2t, g, st)) != MOE_OK) return stt;
   } else {
     const int bn = pick_bn(I, false, r, true);
     CUtensorMap ta, tb, tla, tlb;
@@ -965,9 +1004,12 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
     g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
     g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
-    g.lora_t = dzb1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
     g.stall_test = g_stall_test;
-    if ((stt = launch_pair<kGateUpBwd>(r, dZ1, W1, B1p, A1t, g, st)) != MOE_OK) return stt;
+    if ((stt = rank_down(r, dZ1, B1, 2 * I, expert_offsets, E, R, s, dzb1_rm, dzb1, st)) !=
+        MOE_OK)
+      return stt;
+    if ((stt = launch_pair<kGateUpBwd>(r, dZ1, W1, dzb1_rm, A1t, g, st)) != MOE_OK) return stt;
   } else {
     const int bn = pick_bn(H, false, r, true);
     CUtensorMap ta, tb, tla, tlb;

@@ -32,7 +32,8 @@ EXPORTS = [
 
 PROF_KINDS = {"route": 0, "permute": 1, "gate_up_fwd": 2, "down_fwd": 3,
               "unpermute": 4, "down_bwd": 5, "gate_up_bwd": 6, "lora_grad": 7,
-              "transpose": 8, "base_grad": 9, "router_fwd": 10, "router_bwd": 11}
+              "transpose": 8, "base_grad": 9, "router_fwd": 10, "router_bwd": 11,
+              "rank_down": 12}
 
 
 class MoeError(RuntimeError):
