@@ -412,13 +412,28 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
     for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
       constexpr int W = decltype(w)::value;
       uint4 gv[W / 8], uv[W / 8];
+      // loads first (in flight during the TMEM read), 32 bytes at a time
+      // where the address allows
+      const bool a32 = ((reinterpret_cast<uintptr_t>(grow_p + col0 + c) |
+                         reinterpret_cast<uintptr_t>(grow_p + args.I + col0 + c)) & 31u) == 0;
 #pragma unroll
-      for (int q = 0; q < W / 8; ++q) {  // loads first: in flight during the TMEM read
+      for (int q = 0; q < W / 8; q += 2) {
         const int col = col0 + c + 8 * q;
         gv[q] = uv[q] = make_uint4(0, 0, 0, 0);
-        if (rvalid && col < args.N) {
-          gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
-          uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
+        if (q + 1 < W / 8) gv[q + 1] = uv[q + 1] = make_uint4(0, 0, 0, 0);
+        if (!rvalid) continue;
+        if (q + 1 < W / 8 && a32 && col + 16 <= args.N) {
+          ld_global_nc_v8(grow_p + col, gv[q], gv[q + 1]);
+          ld_global_nc_v8(grow_p + args.I + col, uv[q], uv[q + 1]);
+        } else {
+          if (col < args.N) {
+            gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
+            uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
+          }
+          if (q + 1 < W / 8 && col + 8 < args.N) {
+            gv[q + 1] = *reinterpret_cast<const uint4*>(grow_p + col + 8);
+            uv[q + 1] = *reinterpret_cast<const uint4*>(grow_p + args.I + col + 8);
+          }
         }
       }
       float dh[W];

@@ -263,6 +263,15 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// 32-byte global load (8 x 32 bits) through the non-coherent path; p must
+// be 32-byte aligned.
+__device__ __forceinline__ void ld_global_nc_v8(const void* p, uint4& a, uint4& b) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y),
+                 "=r"(b.z), "=r"(b.w)
+               : "l"(p));
+}
+
 // 32-byte global store (8 x 32 bits) with an L2 cache policy; p must be
 // 32-byte aligned.
 __device__ __forceinline__ void st_global_v8_hint(void* p, uint4 a, uint4 b, uint64_t policy) {
