@@ -59,6 +59,12 @@ __device__ __forceinline__ void drain_pair_copies(uint64_t* bars, int n, uint32_
   }
 }
 
+// L2 policies of the pair kernels' operand loads: 0 = default for both,
+// 1 = weights evict-last, 2 = activations evict-last.
+#ifndef MOE_PAIR_HINTS
+#define MOE_PAIR_HINTS 1
+#endif
+
 template <int MODE, int BN, int RK>
 struct PairCfg {
   static constexpr bool kSwiGLU = (MODE == kGateUpFwd);
@@ -215,6 +221,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       int n_st = 0, n_lb = 0;
       bool ok = true;
       int local = 0;
+      // L2 residency: activations (A, reused by the tile's n-tiles) and
+      // weights (reused by the expert's m-tiles), see MOE_PAIR_HINTS
+#if MOE_PAIR_HINTS == 1
+      const uint64_t pol_a = policy_evict_normal(), pol_w = policy_evict_last();
+#elif MOE_PAIR_HINTS == 2
+      const uint64_t pol_a = policy_evict_last(), pol_w = policy_evict_normal();
+#else
+      const uint64_t pol_a = policy_evict_normal(), pol_w = policy_evict_normal();
+#endif
       for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++local) {
         int e, mt, nt;
         decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
@@ -239,7 +254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           const int kx = kt * C::BK;
           const uint32_t fb = lead(&full[stage]);
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
-          tma_load_2d_pair(st, &tmA, fb, kx, row0);
+          tma_load_2d_pair_hint(st, &tmA, fb, kx, row0, pol_a);
           if constexpr (kBMN) {
             // W [K, N] in place: this CTA's half of the tile's weight
             // columns, one 64-column atom per box
@@ -248,23 +263,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
             const int krow = e * args.b_rows + kx;
 #pragma unroll
             for (int i = 0; i < C::NH / A; ++i)
-              tma_load_2d_pair(sb + i * C::MN_BOX, &tmW0, fb, n0 + A * i, krow);
+              tma_load_2d_pair_hint(sb + i * C::MN_BOX, &tmW0, fb, n0 + A * i, krow, pol_w);
           } else if (kSwiGLU) {
             const int gate = e * args.b_rows + nt * HALF;
             const int up = e * args.b_rows + args.I + nt * HALF;
             if (rank == 0) {
-              tma_load_2d_pair(sb, &tmW0, fb, kx, gate);
-              tma_load_2d_pair(sb + HALF * 128, &tmW1, fb, kx, up);
+              tma_load_2d_pair_hint(sb, &tmW0, fb, kx, gate, pol_w);
+              tma_load_2d_pair_hint(sb + HALF * 128, &tmW1, fb, kx, up, pol_w);
             } else {
-              tma_load_2d_pair(sb, &tmW2, fb, kx, up + C::U0);
+              tma_load_2d_pair_hint(sb, &tmW2, fb, kx, up + C::U0, pol_w);
               tma_load_2d_pair(sb + C::U1 * 128, &tmLA, fb, kx, e * RK);
             }
           } else {
             const int w = e * args.b_rows + nt * BN;
             if (rank == 0) {
-              tma_load_2d_pair(sb, &tmW0, fb, kx, w);
+              tma_load_2d_pair_hint(sb, &tmW0, fb, kx, w, pol_w);
             } else {
-              tma_load_2d_pair(sb, &tmW2, fb, kx, w + C::W0);
+              tma_load_2d_pair_hint(sb, &tmW2, fb, kx, w + C::W0, pol_w);
               tma_load_2d_pair(sb + C::W1 * 128, &tmLA, fb, kx, e * RK);
             }
           }

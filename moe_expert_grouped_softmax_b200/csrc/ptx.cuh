@@ -217,6 +217,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// The same with an L2 cache policy for the copied lines.
+__device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const CUtensorMap* m,
+                                                      uint32_t bar_cluster, int x, int y,
+                                                      uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes.L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
 // Marks `bytes` of the current phase's expected transaction count as done
 // without a copy (balances copies that were expected but never issued).
 __device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
