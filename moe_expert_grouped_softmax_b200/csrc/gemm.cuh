@@ -378,9 +378,11 @@ __device__ __forceinline__ void epi_prefetch_saved(const GemmArgs& args, int gro
 
 // Epilogue step 2: drain the accumulator of this thread's row with the
 // mode's math (SwiGLU; plain store; SwiGLU backward).
-template <int MODE, int BN, bool kSplit>
+// Non-SwiGLU modes can drain a part of the tile: NC columns starting at
+// tile column cbase (TMEM column t_acc holds tile column cbase).
+template <int MODE, int BN, bool kSplit, int NC = BN>
 __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, int grow,
-                                          bool rvalid, int nt, int ehalf) {
+                                          bool rvalid, int nt, int ehalf, int cbase = 0) {
   constexpr bool kSwiGLU = (MODE == kGateUpFwd);
   constexpr int HALF = BN / 2;
   const uint64_t pol = policy_evict_first();  // outputs stream out of L2
@@ -406,10 +408,10 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
       }
     });
   } else if constexpr (MODE == kDownBwd) {
-    const int col0 = nt * BN;
+    const int col0 = nt * BN + cbase;
     const __nv_bfloat16* grow_p = args.aux + static_cast<size_t>(grow) * args.ld_aux;
     __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
-    for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
+    for_my_chunks<NC, kSplit>(ehalf, [&](int c, auto w) {
       constexpr int W = decltype(w)::value;
       uint4 gv[W / 8], uv[W / 8];
       // loads first (in flight during the TMEM read), 32 bytes at a time
@@ -464,9 +466,9 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
       }
     });
   } else {
-    const int col0 = nt * BN;
+    const int col0 = nt * BN + cbase;
     __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
-    for_my_chunks<BN, kSplit>(ehalf, [&](int c, auto w) {
+    for_my_chunks<NC, kSplit>(ehalf, [&](int c, auto w) {
       constexpr int W = decltype(w)::value;
       float v[W];
       tmem_ld<W>(t_acc + c, v);

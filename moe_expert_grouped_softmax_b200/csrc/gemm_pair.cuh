@@ -59,6 +59,14 @@ __device__ __forceinline__ void drain_pair_copies(uint64_t* bars, int n, uint32_
   }
 }
 
+// Backward tiles: an expert's last 256-row tile with at most 128 rows of the
+// expert runs as a half tile on the M = 128 pair instruction (64 rows per
+// CTA).  Its accumulator sits in TMEM as lanes 0-63 = the CTA's 64 rows for
+// tile columns [0, N/2) and lanes 64-127 = the same rows for [N/2, N).
+__device__ __forceinline__ bool pair_half_tile(const int* s_off, int e, int mt) {
+  return s_off[e + 1] - (s_off[e] + mt * 256) <= 128;
+}
+
 // L2 policies of the pair kernels' operand loads: 0 = default for both,
 // 1 = weights evict-last, 2 = activations evict-last.
 #ifndef MOE_PAIR_HINTS
@@ -233,7 +241,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++local) {
         int e, mt, nt;
         decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
-        const int row0 = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * C::BM;
+        const int rows_per_cta = (kBMN && pair_half_tile(s_off, e, mt)) ? C::BM / 2 : C::BM;
+        const int row0 = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * rows_per_cta;
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         if (!mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
@@ -301,6 +310,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       // elected lane issues the tensor-core instructions.
       constexpr uint32_t kIdesc = idesc_bf16_f32(256, C::NMMA, false, kBMN);
       constexpr uint32_t kIdescUp = idesc_bf16_f32(256, BN, false, false);
+      constexpr uint32_t kIdescH = idesc_bf16_f32(128, C::NMMA, false, kBMN);
+      constexpr uint32_t kIdescUpH = idesc_bf16_f32(128, BN, false, false);
+      uint32_t idesc = kIdesc, idesc_up = kIdescUp;
       constexpr uint16_t kBoth = 0x3;
       auto issue_up = [&](int b) {
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
@@ -309,7 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
 #pragma unroll
         for (int kk = 0; kk < RK / 16; ++kk)
           umma_bf16_pair(t_acc, smem_desc(xa0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
-                         smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), kIdescUp, 1u);
+                         smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), idesc_up, 1u);
         umma_commit_pair_mc(&lb_empty[b], kBoth);
         umma_commit_pair_mc(&acc_full[b], kBoth);
       };
@@ -339,16 +351,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
+        if constexpr (kBMN) {
+          int e, mt, nt;
+          decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+          const bool half = pair_half_tile(s_off, e, mt);
+          idesc = half ? kIdescH : kIdesc;
+          idesc_up = half ? kIdescUpH : kIdescUp;
+        }
         if (!MOE_TIMED(MODE, 14, warp_wait_cluster(&acc_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < k_iters; ++kt) {
           if (!MOE_TIMED(MODE, 11, warp_wait(&full[stage], phase, s_abort, wait_ns))) { ok = false; break; }
           const uint64_t da = a_desc0 + soff, db = b_desc0 + soff;
           if (elect_one()) {
-            umma_bf16_pair(t_acc, da, db, kIdesc, kt > 0 ? 1u : 0u);
+            umma_bf16_pair(t_acc, da, db, idesc, kt > 0 ? 1u : 0u);
 #pragma unroll
             for (int kk = 1; kk < C::BK / 16; ++kk)
-              umma_bf16_pair(t_acc, da + 2 * kk, db + kk * kBStep, kIdesc, 1u);
+              umma_bf16_pair(t_acc, da + 2 * kk, db + kk * kBStep, idesc, 1u);
             umma_commit_pair_mc(&empty[stage], kBoth);
           }
           __syncwarp();
@@ -415,7 +434,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
       const int b = local & 1;
       const uint32_t use = (local >> 1) & 1;
-      const int grow = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * C::BM + row_in_tile;
+      const bool half = kBMN && pair_half_tile(s_off, e, mt);
+      // half tile: lane quarters 0-1 hold rows 0-63 for columns [0, BN/2),
+      // quarters 2-3 the same rows for [BN/2, BN)
+      const int row_local = half ? (ew & 1) * 32 + lane : row_in_tile;
+      const int grow = s_off[e] + mt * 2 * C::BM +
+                       static_cast<int>(rank) * (half ? C::BM / 2 : C::BM) + row_local;
       const bool rvalid = grow < s_off[e + 1];
       const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
       if (!kBMN && ehalf == 0) {  // rank-r hand-off: the first four epilogue warps
@@ -428,10 +452,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(lead(&xa_ready[b]));
       }
-      if constexpr (MODE == kDownBwd) epi_prefetch_saved<BN>(args, grow, rvalid, nt, ehalf);
+      if constexpr (MODE == kDownBwd) {
+        if (!half) epi_prefetch_saved<BN>(args, grow, rvalid, nt, ehalf);
+      }
       if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
       tc_fence_after();
-      epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
+      if constexpr (kBMN) {
+        if (half)
+          epi_drain<MODE, BN, kSplit, BN / 2>(args, t_acc, grow, rvalid, nt, ehalf,
+                                              (ew >> 1) * (BN / 2));
+        else
+          epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
+      } else {
+        epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead(&acc_empty[b]));
