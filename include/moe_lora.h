@@ -132,7 +132,11 @@ MOE_API moe_status_t moe_unpermute(const void* Yp, const int32_t* dest, const fl
  *   part 2: XA1 bf16 [r, R]   s * (Xp A1^T), transposed, row pitch
  *                             round_up(R, 64) elements (padding zeroed)
  *   part 3: HA2 bf16 [r, R]   s * (h A2^T), transposed, same pitch
- * moe_saved_part_offset(R, H, I, r, part) gives each part's byte offset. */
+ *   part 4: XA1 bf16 [R, r]   s * (Xp A1^T), row-major (written when the
+ *                             gate_up GEMM runs on CTA pairs)
+ *   part 5: HA2 bf16 [R, r]   s * (h A2^T), row-major (likewise, down GEMM)
+ * moe_saved_part_offset(R, H, I, r, part) gives each part's byte offset;
+ * part 6 is the end (= moe_saved_bytes). */
 MOE_API size_t moe_saved_bytes(int R, int H, int I, int r);
 MOE_API size_t moe_saved_part_offset(int R, int H, int I, int r, int part);
 /* Scratch needed by moe_lora_mlp_fwd / moe_lora_mlp_bwd (device bytes). */
@@ -256,9 +260,9 @@ MOE_API unsigned long long moe_kernel_launches(void);
  * pairs when the mean rows per expert R / E is at least 768 (little padding
  * on each expert's ragged last 256-row tile) and the GEMM's K is at least
  * 1024 (H for gate_up forward and down backward, I for down forward, 2I for
- * gate_up backward).  A backward GEMM on pairs takes its rank-r product
- * (s dZ2 B2 or s dZ1 B1) from a separate memory-bound pass.  All compute the
- * same result. */
+ * gate_up backward).  A GEMM on pairs takes its rank-r product (s Xp A1^T,
+ * s h A2^T, s dZ2 B2 or s dZ1 B1) from a separate memory-bound pass.  All
+ * compute the same result to the tolerance of bf16 rounding. */
 MOE_API void moe_set_cta_pairs(int mode);
 
 /* Benchmark hook (not thread-safe; for measurement only).

@@ -1,32 +1,40 @@
-// a3, a4, a7, a8 on CTA pairs: the grouped GEMMs with 256-row tiles on the
+// a3, a4, a7, a8 on CTA pairs: the grouped GEMMs with 256 x 256 tiles on the
 // 2-SM tensor-core instruction (tcgen05.mma.cta_group::2).
 //
-// A cluster of two CTAs on two SMs computes one 256 x BN tile of one expert.
-// Each CTA stages its own 128 rows of A and half of the B operand
-// [W (BN columns) ; LoRA-down factor (r columns)] (N = BN + r, split into two
-// halves of N/2), so every SM moves a third less operand data per FLOP
-// than the single-CTA 128-row tile, through shared memory as well as from L2.
-// Forward (K-major B): the halves are row blocks of W and of the factor.
-// Backward (MN-major B, W read in place as [K, N]): the rank-r
-// down-products (s dZ2 B2, s dZ1 B1) come from their own pass, so the B
-// operand is weight columns only, BN = 256 as four 64-column atoms (128-byte
-// swizzle, 64 x 64 TMA boxes, two per CTA); each tile's up-projection
-// operands (its 256 rows of the rank-r product and the BN rows of the
-// K-major up factor) are loaded by TMA and accumulated after the mainloop.  The even CTA ("leader") issues the
-// MMAs, which read both CTAs' shared memory and write both CTAs' TMEM (each
-// holds its 128 rows x N columns).  The split-LoRA schedule is the one of the
-// single-CTA kernel: rank-r down-projection inside the mainloop MMA,
-// hand-off through shared memory, up-projection (M = 256, K = r) into the
-// same accumulator during the next tile's mainloop.
+// A cluster of two CTAs on two SMs computes one 256-row x 256-column tile of
+// one expert.  Each CTA stages its own 128 rows of A and half (128 columns)
+// of the weight operand, so every SM moves a third less operand data per
+// FLOP than the single-CTA 128-row tile, through shared memory as well as
+// from L2.  The even CTA ("leader") issues the MMAs, which read both CTAs'
+// shared memory and write both CTAs' TMEM.
+//
+// Split LoRA: the rank-r down-products (s Xp A1^T, s h A2^T, s dZ2 B2,
+// s dZ1 B1) come from their own pass (rank_down_kernel), so the B operand is
+// weight columns only.  Each tile's up-projection operands -- its rows of the
+// rank-r product and the up factor rows of its columns, both K-major with
+// K = r -- are loaded by TMA beside the tile and accumulated into the same
+// TMEM tile right after the mainloop: W + s B A is never formed.
+//
+// B operand of each CTA (128 of the tile's 256 columns):
+//   gate_up fwd: [gate j..j+63 | up j..j+63] with j = 128 nt + 64 rank, so
+//                every 128 tile columns hold gate and up of the same 64
+//                output columns (the SwiGLU epilogue needs both in one
+//                thread, also for half tiles);
+//   down fwd:    W2 rows 256 nt + 128 rank .. +127 (K-major);
+//   backward:    W read in place as [K, N], MN-major atoms of 64 columns.
+// Half tiles: an expert's last tile with at most 128 rows of the expert runs
+// on the M = 128 pair instruction (64 rows per CTA); its accumulator sits in
+// TMEM as lanes 0-63 = the CTA's 64 rows for tile columns [0, 128) and lanes
+// 64-127 = the same rows for [128, 256) (measured).
 //
 // Synchronisation (every wait bounded):
 //  * both CTAs' TMA loads of a stage complete on the leader's barrier (the
 //    pair form of the tensor copy signals a barrier of either CTA); only the
 //    leader arms it, for the bytes of both halves;
 //  * the leader's MMA commits are multicast to both CTAs' barriers
-//    (stage free, rank-r product ready, accumulator ready);
-//  * both CTAs' epilogues arrive on the leader's barriers (hand-off written,
-//    accumulator drained);
+//    (stage free, up-projection operands free, accumulator ready);
+//  * both CTAs' epilogues arrive on the leader's barriers (accumulator
+//    drained);
 //  * at exit, each CTA waits for the leader's last MMAs (which touch its
 //    shared memory and TMEM); the peer then tells the leader how many copies
 //    it issued, the leader balances and waits out every copy either CTA has
@@ -59,10 +67,7 @@ __device__ __forceinline__ void drain_pair_copies(uint64_t* bars, int n, uint32_
   }
 }
 
-// Backward tiles: an expert's last 256-row tile with at most 128 rows of the
-// expert runs as a half tile on the M = 128 pair instruction (64 rows per
-// CTA).  Its accumulator sits in TMEM as lanes 0-63 = the CTA's 64 rows for
-// tile columns [0, N/2) and lanes 64-127 = the same rows for [N/2, N).
+// An expert's last 256-row tile with at most 128 rows of the expert.
 __device__ __forceinline__ bool pair_half_tile(const int* s_off, int e, int mt) {
   return s_off[e + 1] - (s_off[e] + mt * 256) <= 128;
 }
@@ -73,78 +78,82 @@ __device__ __forceinline__ bool pair_half_tile(const int* s_off, int e, int mt) 
 #define MOE_PAIR_HINTS 1
 #endif
 
-template <int MODE, int BN, int RK>
+template <int MODE, int RK>
 struct PairCfg {
   static constexpr bool kSwiGLU = (MODE == kGateUpFwd);
   static constexpr bool kBMN = (MODE == kDownBwd || MODE == kGateUpBwd);
-  static constexpr int BM = 128, BK = 64;           // rows per CTA
-  // forward: the down factor's r rows ride in the B operand (N = BN + r);
-  // backward: weight columns only
-  static constexpr int NMMA = kBMN ? BN : BN + RK;  // N of the mainloop MMA
-  static constexpr int NH = NMMA / 2;               // B rows per CTA
-  static constexpr int HALF = BN / 2;
-  // B segments of each CTA (rows of N): SwiGLU: CTA0 = gate HALF + up U0,
-  // CTA1 = up U1 + factor RK.  Plain and backward: CTA0 = W0 weight
-  // columns, CTA1 = W1 weight columns + factor RK.
-  static constexpr int U0 = NH - HALF;              // = RK / 2
-  static constexpr int U1 = HALF - U0;
-  static constexpr int W0 = NH;
-  static constexpr int W1 = BN - NH;
+  static constexpr int BM = 128, BK = 64;           // rows per CTA, K per stage
+  static constexpr int BN = 256;                    // tile columns (MMA N)
+  static constexpr int NH = BN / 2;                 // B columns per CTA
+  // output columns per tile (gate_up: 128 gate + 128 up columns)
+  static constexpr int OUT_COLS = kSwiGLU ? BN / 2 : BN;
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = NH * 128;
+  static constexpr int B_BYTES = NH * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int LB_BYTES = HALF * RK * 2;    // this CTA's half of LB
-  static constexpr int XA_BYTES = BM * RK * 2;
-  // up-projection operands one CTA loads per tile (backward: the rank-r
-  // product rows too)
-  static constexpr int UP_BYTES = kBMN ? LB_BYTES + XA_BYTES : LB_BYTES;
+  static constexpr int LSPAN = RK * 2;              // bytes per K-major rank-r row
+  static constexpr int LB_BYTES = NH * LSPAN;       // this CTA's up-factor rows
+  static constexpr int XA_BYTES = BM * LSPAN;       // this CTA's rank-r rows
+  static constexpr int UP_BYTES = LB_BYTES + XA_BYTES;
   static constexpr int MISC_BYTES = 512 + 8 * 520;  // barriers, counts, tables
-  static constexpr int FIXED = 2 * LB_BYTES + 2 * XA_BYTES + MISC_BYTES;
+  static constexpr int FIXED = 2 * UP_BYTES + MISC_BYTES;
   static constexpr int NS_FIT = (kSmemOptin - 1024 - FIXED) / STAGE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + FIXED;
-  static constexpr int LSPAN = RK * 2;
   static constexpr uint32_t LLAYOUT =
       RK == 16 ? kLayoutSW32 : (RK == 32 ? kLayoutSW64 : kLayoutSW128);
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_STRIDE = 256;
   static constexpr int EPI_WARPS = gemm_epi_warps(MODE);
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  // MN-major B: one 64-column x BK-row box (128-byte swizzle) per atom
-  static constexpr int MN_COLS = 64;
-  static constexpr int MN_BOX = MN_COLS * BK * 2;
-  static_assert(!kBMN || (NH % MN_COLS == 0 && NMMA == 256),
-                "MN-major halves in whole 64-column atoms");
+  // weight rows per TMA box: gate_up fwd loads gate and up blocks of 64
+  static constexpr int W_BOX_ROWS = kSwiGLU ? 64 : NH;
+  static constexpr int LB_BOX_ROWS = kSwiGLU ? 64 : NH;
+  static constexpr int MN_BOX = 64 * BK * 2;        // one 64-column MN-major atom
   static_assert(NS >= 3, "not enough shared memory for three stages");
   static_assert(SMEM_BYTES <= kSmemOptin, "shared memory over the opt-in limit");
-  static_assert(NMMA <= ACC_STRIDE && NMMA % 16 == 0, "MMA N = BN + r");
-  static_assert(BN % 16 == 0 && NH % 8 == 0, "8-row operand atoms");
-  static_assert(!kSwiGLU || (U0 % 8 == 0 && U1 % 8 == 0 && U1 > 0), "SwiGLU segments");
-  static_assert(kBMN || (W1 % 8 == 0 && W1 > 0), "plain segments");
+  static_assert(LB_BYTES % 1024 == 0 && XA_BYTES % 1024 == 0, "swizzle atoms");
 };
 
-// Host-visible box heights of the weight segments (rows), for the maps.
-template <int MODE, int BN, int RK>
-struct PairBoxes {
-  using C = PairCfg<MODE, BN, RK>;
-  static constexpr int seg0 = C::kSwiGLU ? C::HALF : C::W0;  // CTA0, first
-  static constexpr int seg1 = C::kSwiGLU ? C::U0 : 0;        // CTA0, second
-  static constexpr int seg2 = C::kSwiGLU ? C::U1 : C::W1;    // CTA1, first
-};
+// SwiGLU epilogue of one 64-column gate / up segment of a row: gate at TMEM
+// column t_gate, up at t_gate + 64; output columns col .. col + 63.
+__device__ __forceinline__ void epi_swiglu_seg64(const GemmArgs& args, uint32_t t_gate,
+                                                 int grow, bool rvalid, int col,
+                                                 uint64_t pol) {
+  __nv_bfloat16* hrow = args.out + static_cast<size_t>(grow) * args.ld_out;
+  __nv_bfloat16* zrow = args.out2 + static_cast<size_t>(grow) * args.ld_out2;
+  for_chunks<64>([&](int c, auto w) {
+    constexpr int W = decltype(w)::value;
+    float g[W], u[W];
+    tmem_ld<W>(t_gate + c, g);
+    tmem_ld<W>(t_gate + 64 + c, u);
+    tmem_ld_wait();
+    if (rvalid) {
+      float h[W];
+#pragma unroll
+      for (int i = 0; i < W; ++i) h[i] = g[i] * sigmoidf_(g[i]) * u[i];
+      const int cc = col + c, nv = args.N - cc;
+      store_row_bf16<W>(hrow + cc, h, nv, pol);
+      store_row_bf16<W>(zrow + cc, g, nv, pol);
+      store_row_bf16<W>(zrow + args.I + cc, u, nv, pol);
+    }
+  });
+}
 
-template <int MODE, int BN, int RK>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK>::THREADS, 1)
+// Operand maps: tmA = A [R, K] (128-row boxes); tmW = the weight (K-major
+// [E * b_rows, K] in W_BOX_ROWS-row boxes, or MN-major [E * b_rows, N] in
+// 64 x 64 atoms); tmXA = the rank-r product [R, r] (128-row boxes);
+// tmLB = the up factor [E * lb_rows, r] (LB_BOX_ROWS-row boxes).
+template <int MODE, int RK>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::THREADS, 1)
     grouped_lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                                  const __grid_constant__ CUtensorMap tmW0,
-                                  const __grid_constant__ CUtensorMap tmW1,
-                                  const __grid_constant__ CUtensorMap tmW2,
-                                  const __grid_constant__ CUtensorMap tmLA,
+                                  const __grid_constant__ CUtensorMap tmW,
+                                  const __grid_constant__ CUtensorMap tmXA,
                                   const __grid_constant__ CUtensorMap tmLB,
                                   const GemmArgs args) {
-  using C = PairCfg<MODE, BN, RK>;
+  using C = PairCfg<MODE, RK>;
   constexpr bool kSwiGLU = C::kSwiGLU;
   constexpr bool kBMN = C::kBMN;
-  constexpr int HALF = C::HALF;
+  constexpr int BN = C::BN;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -156,16 +165,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
   uint64_t* empty = full + C::NS;
   uint64_t* lb_full = empty + C::NS;
   uint64_t* lb_empty = lb_full + 2;
-  uint64_t* lora_full = lb_empty + 2;
-  uint64_t* xa_ready = lora_full + 2;
-  uint64_t* acc_full = xa_ready + 2;
+  uint64_t* acc_full = lb_empty + 2;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* final_bar = acc_empty + 2;
   uint64_t* peer_done = final_bar + 1;       // leader: the peer is done
   uint64_t* drained = peer_done + 1;         // peer: its copies have landed
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  // copies issued by this CTA's producer: [0] stages, [1] up-factor halves;
+  // copies issued by this CTA's producer: [0] stages, [1] up-operand sets;
   // [2], [3]: the same counts of the peer (written into the leader)
   int* s_issued = reinterpret_cast<int*>(s_tmem + 4);
   int* s_off = s_issued + 4;
@@ -186,8 +193,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
     for (int i = 0; i < 2; ++i) {
       mbar_init(&lb_full[i], 1);
       mbar_init(&lb_empty[i], 1);
-      mbar_init(&lora_full[i], 1);
-      mbar_init(&xa_ready[i], 2 * 4);
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 2 * C::EPI_WARPS);
     }
@@ -200,10 +205,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
-    prefetch_tmap(&tmW0);
-    prefetch_tmap(&tmW1);
-    prefetch_tmap(&tmW2);
-    prefetch_tmap(&tmLA);
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmXA);
     prefetch_tmap(&tmLB);
   }
   if (warp == 1) {
@@ -241,20 +244,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++local) {
         int e, mt, nt;
         decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
-        const int rows_per_cta = (kBMN && pair_half_tile(s_off, e, mt)) ? C::BM / 2 : C::BM;
+        const int rows_per_cta = pair_half_tile(s_off, e, mt) ? C::BM / 2 : C::BM;
         const int row0 = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * rows_per_cta;
+        // first weight / up-factor row of this CTA's tile columns
+        const int n0 = kSwiGLU ? nt * (BN / 2) + static_cast<int>(rank) * 64
+                               : nt * BN + static_cast<int>(rank) * C::NH;
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         if (!mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
         if (leader) mbar_arrive_expect_tx(&lb_full[b], 2 * C::UP_BYTES);
-        // this CTA's half of the up-projection factor: output columns
-        // [rank * BN/2, (rank + 1) * BN/2) of the tile
-        const int lb_row = kSwiGLU ? e * args.lb_rows + (rank ? args.I : 0) + nt * HALF
-                                   : e * args.lb_rows + nt * BN + static_cast<int>(rank) * HALF;
-        tma_load_2d_pair(sLB + b * C::LB_BYTES, &tmLB, lead(&lb_full[b]), 0, lb_row);
-        // backward: this CTA's 128 rows of the rank-r product (K-major)
-        if constexpr (kBMN)
-          tma_load_2d_pair(sXA + b * C::XA_BYTES, &tmLA, lead(&lb_full[b]), 0, row0);
+        {
+          // up-projection operands: this CTA's rows of the rank-r product and
+          // the up factor rows of its tile columns
+          const uint32_t lbb = lead(&lb_full[b]);
+          uint8_t* lb = sLB + b * C::LB_BYTES;
+          const int lrow = e * args.lb_rows + n0;
+          tma_load_2d_pair(lb, &tmLB, lbb, 0, lrow);
+          if constexpr (kSwiGLU)
+            tma_load_2d_pair(lb + 64 * C::LSPAN, &tmLB, lbb, 0, lrow + args.I);
+          tma_load_2d_pair(sXA + b * C::XA_BYTES, &tmXA, lbb, 0, row0);
+        }
         ++n_lb;
         for (int kt = 0; kt < k_iters; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, wait_ns)) { ok = false; break; }
@@ -265,32 +274,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           tma_load_2d_pair_hint(st, &tmA, fb, kx, row0, pol_a);
           if constexpr (kBMN) {
-            // W [K, N] in place: this CTA's half of the tile's weight
-            // columns, one 64-column atom per box
-            constexpr int A = C::MN_COLS;
-            const int n0 = nt * BN + static_cast<int>(rank) * C::NH;
+            // W [K, N] in place: this CTA's 128 tile columns as two 64-column
+            // atoms
             const int krow = e * args.b_rows + kx;
-#pragma unroll
-            for (int i = 0; i < C::NH / A; ++i)
-              tma_load_2d_pair_hint(sb + i * C::MN_BOX, &tmW0, fb, n0 + A * i, krow, pol_w);
-          } else if (kSwiGLU) {
-            const int gate = e * args.b_rows + nt * HALF;
-            const int up = e * args.b_rows + args.I + nt * HALF;
-            if (rank == 0) {
-              tma_load_2d_pair_hint(sb, &tmW0, fb, kx, gate, pol_w);
-              tma_load_2d_pair_hint(sb + HALF * 128, &tmW1, fb, kx, up, pol_w);
-            } else {
-              tma_load_2d_pair_hint(sb, &tmW2, fb, kx, up + C::U0, pol_w);
-              tma_load_2d_pair(sb + C::U1 * 128, &tmLA, fb, kx, e * RK);
-            }
+            tma_load_2d_pair_hint(sb, &tmW, fb, n0, krow, pol_w);
+            tma_load_2d_pair_hint(sb + C::MN_BOX, &tmW, fb, n0 + 64, krow, pol_w);
+          } else if constexpr (kSwiGLU) {
+            const int wrow = e * args.b_rows + n0;
+            tma_load_2d_pair_hint(sb, &tmW, fb, kx, wrow, pol_w);                 // gate
+            tma_load_2d_pair_hint(sb + 64 * 128, &tmW, fb, kx, wrow + args.I, pol_w);  // up
           } else {
-            const int w = e * args.b_rows + nt * BN;
-            if (rank == 0) {
-              tma_load_2d_pair_hint(sb, &tmW0, fb, kx, w, pol_w);
-            } else {
-              tma_load_2d_pair_hint(sb, &tmW2, fb, kx, w + C::W0, pol_w);
-              tma_load_2d_pair(sb + C::W1 * 128, &tmLA, fb, kx, e * RK);
-            }
+            tma_load_2d_pair_hint(sb, &tmW, fb, kx, e * args.b_rows + n0, pol_w);
           }
           ++n_st;
           if (++stage == C::NS) {
@@ -308,28 +302,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       // ---------------------------------------------------------- MMA (leader)
       // The whole warp runs the loop (its state stays warp-uniform); one
       // elected lane issues the tensor-core instructions.
-      constexpr uint32_t kIdesc = idesc_bf16_f32(256, C::NMMA, false, kBMN);
+      constexpr uint32_t kIdesc = idesc_bf16_f32(256, BN, false, kBMN);
+      constexpr uint32_t kIdescH = idesc_bf16_f32(128, BN, false, kBMN);
       constexpr uint32_t kIdescUp = idesc_bf16_f32(256, BN, false, false);
-      constexpr uint32_t kIdescH = idesc_bf16_f32(128, C::NMMA, false, kBMN);
       constexpr uint32_t kIdescUpH = idesc_bf16_f32(128, BN, false, false);
-      uint32_t idesc = kIdesc, idesc_up = kIdescUp;
       constexpr uint16_t kBoth = 0x3;
-      auto issue_up = [&](int b) {
-        const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
-        const uint32_t xa0 = smem_u32(sXA + b * C::XA_BYTES);
-        const uint32_t lb0 = smem_u32(sLB + b * C::LB_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < RK / 16; ++kk)
-          umma_bf16_pair(t_acc, smem_desc(xa0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
-                         smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), idesc_up, 1u);
-        umma_commit_pair_mc(&lb_empty[b], kBoth);
-        umma_commit_pair_mc(&acc_full[b], kBoth);
-      };
-      auto up_when_ready = [&](int b) {
-        tc_fence_after();
-        if (elect_one()) issue_up(b);
-        __syncwarp();
-      };
       const uint64_t a_desc0 = smem_desc(smem_u32(sStage), 16, 1024, kLayoutSW128);
       // MN-major: LBO = next 64-column atom, SBO = next 8 K-rows (8 x 128 B)
       const uint64_t b_desc0 =
@@ -341,7 +318,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
       uint64_t soff = 0;
       uint32_t phase = 0;
       int local = 0;
-      int pending = -1;
       bool ok = true;
       if (args.stall_test) ok = warp_wait(final_bar, 0, s_abort, wait_ns);
 #ifdef MOE_GEMM_TRACE
@@ -351,13 +327,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
-        if constexpr (kBMN) {
-          int e, mt, nt;
-          decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
-          const bool half = pair_half_tile(s_off, e, mt);
-          idesc = half ? kIdescH : kIdesc;
-          idesc_up = half ? kIdescUpH : kIdescUp;
-        }
+        int e, mt, nt;
+        decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+        const bool half = pair_half_tile(s_off, e, mt);
+        const uint32_t idesc = half ? kIdescH : kIdesc;
+        const uint32_t idesc_up = half ? kIdescUpH : kIdescUp;
         if (!MOE_TIMED(MODE, 14, warp_wait_cluster(&acc_empty[b], use ^ 1, s_abort, wait_ns))) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < k_iters; ++kt) {
@@ -377,40 +351,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
             soff = 0;
             phase ^= 1;
           }
-          if (pending >= 0) {
-            const int pb = pending & 1;
-            const uint32_t pu = (pending >> 1) & 1;
-            if (warp_uniform(mbar_test_wait_cluster(&xa_ready[pb], pu) &&
-                             mbar_test_wait(&lb_full[pb], pu))) {
-              up_when_ready(pb);
-              pending = -1;
-            }
-          }
         }
         if (!ok) break;
-        if constexpr (kBMN) {
-          // backward: the tile's up-projection operands came by TMA
-          if (!warp_wait(&lb_full[b], use, s_abort, wait_ns)) { ok = false; break; }
-          up_when_ready(b);
-          continue;
+        // up-projection (K = r) into the same accumulator
+        if (!warp_wait(&lb_full[b], use, s_abort, wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t xa0 = smem_u32(sXA + b * C::XA_BYTES);
+          const uint32_t lb0 = smem_u32(sLB + b * C::LB_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < RK / 16; ++kk)
+            umma_bf16_pair(t_acc, smem_desc(xa0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
+                           smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), idesc_up,
+                           1u);
+          umma_commit_pair_mc(&lb_empty[b], kBoth);
+          umma_commit_pair_mc(&acc_full[b], kBoth);
         }
-        if (elect_one()) umma_commit_pair_mc(&lora_full[b], kBoth);
         __syncwarp();
-        if (pending >= 0) {
-          const int pb = pending & 1;
-          const uint32_t pu = (pending >> 1) & 1;
-          if (!warp_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) ||
-              !warp_wait(&lb_full[pb], pu, s_abort, wait_ns)) { ok = false; break; }
-          up_when_ready(pb);
-        }
-        pending = local;
-      }
-      if (ok && pending >= 0) {
-        const int pb = pending & 1;
-        const uint32_t pu = (pending >> 1) & 1;
-        if (warp_wait_cluster(&xa_ready[pb], pu, s_abort, wait_ns) &&
-            warp_wait(&lb_full[pb], pu, s_abort, wait_ns))
-          up_when_ready(pb);
       }
 #ifdef MOE_GEMM_TRACE
       if (lane == 0)
@@ -426,45 +383,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, BN, RK
     const int ew = warp & 3;              // TMEM lane quarter
     constexpr bool kSplit = C::EPI_WARPS == 8;
     const int ehalf = (warp - 2) >> 2;    // which share of the columns
-    const int row_in_tile = ew * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(ew * 32) << 16;
+    const uint64_t pol = policy_evict_first();  // outputs stream out of L2
     int local = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++local) {
       int e, mt, nt;
       decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
       const int b = local & 1;
       const uint32_t use = (local >> 1) & 1;
-      const bool half = kBMN && pair_half_tile(s_off, e, mt);
-      // half tile: lane quarters 0-1 hold rows 0-63 for columns [0, BN/2),
-      // quarters 2-3 the same rows for [BN/2, BN)
-      const int row_local = half ? (ew & 1) * 32 + lane : row_in_tile;
+      const bool half = pair_half_tile(s_off, e, mt);
+      // half tile: lane quarters 0-1 hold rows 0-63 for tile columns
+      // [0, 128), quarters 2-3 the same rows for [128, 256)
+      const int row_local = half ? (ew & 1) * 32 + lane : ew * 32 + lane;
       const int grow = s_off[e] + mt * 2 * C::BM +
                        static_cast<int>(rank) * (half ? C::BM / 2 : C::BM) + row_local;
       const bool rvalid = grow < s_off[e + 1];
       const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
-      if (!kBMN && ehalf == 0) {  // rank-r hand-off: the first four epilogue warps
-        if (!warp_wait(&lora_full[b], use, s_abort, wait_ns)) break;
-        tc_fence_after();
-        epi_rank_handoff<RK>(args, t_acc + BN, sXA + b * C::XA_BYTES, row_in_tile, nt,
-                             rvalid, grow);
-        fence_proxy_async_all();  // the leader's MMA reads this tile
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead(&xa_ready[b]));
-      }
       if constexpr (MODE == kDownBwd) {
         if (!half) epi_prefetch_saved<BN>(args, grow, rvalid, nt, ehalf);
       }
       if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
       tc_fence_after();
-      if constexpr (kBMN) {
+      if constexpr (kSwiGLU) {
+        // 128-column blocks [gate 64 | up 64] of output columns
+        // 128 nt + 64 q .. +63, q = the block
+        const int col0 = nt * (BN / 2);
+        if (half) {
+          epi_swiglu_seg64(args, t_acc, grow, rvalid, col0 + (ew >> 1) * 64, pol);
+        } else {
+          epi_swiglu_seg64(args, t_acc, grow, rvalid, col0, pol);
+          epi_swiglu_seg64(args, t_acc + 128, grow, rvalid, col0 + 64, pol);
+        }
+      } else {
         if (half)
           epi_drain<MODE, BN, kSplit, BN / 2>(args, t_acc, grow, rvalid, nt, ehalf,
                                               (ew >> 1) * (BN / 2));
         else
           epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
-      } else {
-        epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
       }
       tc_fence_before();
       __syncwarp();

@@ -233,39 +233,31 @@ moe_status_t launch_gemm(int bn, int r, const CUtensorMap& a, const CUtensorMap&
   return MOE_ERR_UNSUPPORTED;
 }
 
-// Forward GEMM on CTA pairs (256-row tiles, BN = 256 - r).  A: [R, K]
-// activations; W: the base weight as [E * b_rows, K]; LA: the down factor as
-// [E * r, K]; LB: the up factor as [E * lb_rows, r].
-template <int MODE, int BN, int RK>
-moe_status_t launch_pair_t(const void* A, const void* W, const void* LA, const void* LB,
+// Grouped GEMM on CTA pairs (256 x 256 tiles, weight-only B operand).
+// A: [R, K] activations; W: the base weight as [E * b_rows, K] (forward) or
+// read in place as [E * b_rows, N] (backward); XA: the s-scaled rank-r
+// product [R, r] from the rank pass; LB: the up factor as [E * lb_rows, r].
+template <int MODE, int RK>
+moe_status_t launch_pair_t(const void* A, const void* W, const void* XA, const void* LB,
                            const GemmArgs& args, cudaStream_t st) {
-  using C = PairCfg<MODE, BN, RK>;
-  using Bx = PairBoxes<MODE, BN, RK>;
+  using C = PairCfg<MODE, RK>;
   const uint64_t K = static_cast<uint64_t>(args.K);
   const uint64_t EU = static_cast<uint64_t>(args.E);
-  CUtensorMap ta, tw0, tw1, tw2, tla, tlb;
+  CUtensorMap ta, tw, txa, tlb;
   bool ok = tmap_2d(&ta, A, K, args.R, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if constexpr (C::kBMN) {
-    // W [E * K, N] in place, 64-column x 64-row boxes (128-byte swizzle); LA
-    // is the rank-r product [R, r] (row-major), one box per CTA and tile
+    // W [E * K, N] in place, 64-column x 64-row boxes (128-byte swizzle)
     const uint64_t N = static_cast<uint64_t>(args.N);
-    ok = ok && tmap_2d(&tw0, W, N, EU * args.b_rows, N * 2, C::MN_COLS, 64,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, LA, RK, args.R, RK * 2ull, RK, C::BM, lora_swizzle(RK));
-    tw1 = tw0;
-    tw2 = tw0;
+    ok = ok && tmap_2d(&tw, W, N, EU * args.b_rows, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   } else {
-    ok = ok && tmap_2d(&tw0, W, K, EU * args.b_rows, K * 2, 64, Bx::seg0,
+    ok = ok && tmap_2d(&tw, W, K, EU * args.b_rows, K * 2, 64, C::W_BOX_ROWS,
                        CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tw1, W, K, EU * args.b_rows, K * 2, 64, Bx::seg1 > 0 ? Bx::seg1 : 8,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tw2, W, K, EU * args.b_rows, K * 2, 64, Bx::seg2,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, LA, K, EU * RK, K * 2, 64, RK, CU_TENSOR_MAP_SWIZZLE_128B);
   }
-  ok = ok && tmap_2d(&tlb, LB, RK, EU * args.lb_rows, RK * 2ull, RK, C::HALF, lora_swizzle(RK));
+  ok = ok && tmap_2d(&txa, XA, RK, args.R, RK * 2ull, RK, C::BM, lora_swizzle(RK));
+  ok = ok && tmap_2d(&tlb, LB, RK, EU * args.lb_rows, RK * 2ull, RK, C::LB_BOX_ROWS,
+                     lora_swizzle(RK));
   if (!ok) return MOE_ERR_CUDA;
-  auto kern = grouped_lora_gemm_pair_kernel<MODE, BN, RK>;
+  auto kern = grouped_lora_gemm_pair_kernel<MODE, RK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM_BYTES) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -278,22 +270,21 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* LA, const v
                  : MODE == kDownBwd   ? MOE_PROF_DOWN_BWD
                                       : MOE_PROF_GATE_UP_BWD,
                  st);
-  kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tw0, tw1, tw2, tla, tlb, args);
+  kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tw, txa, tlb, args);
   count_launch();
   return launch_status();
 }
 
-// Tile width of the CTA-pair kernels: N = BN + r fills the 256-column MMA
-// (forward, K-major factor rows); backward: weight columns only, BN = 256.
-constexpr bool pair_backward(int mode) { return mode == kDownBwd || mode == kGateUpBwd; }
-constexpr int pair_bn(int mode, int r) { return pair_backward(mode) ? 256 : 256 - r; }
+// Output columns per CTA-pair tile: 128 (gate_up forward: 128 gate + 128 up
+// columns) or 256.
+constexpr int pair_out_cols(int mode) { return mode == kGateUpFwd ? 128 : 256; }
 
 template <int MODE>
-moe_status_t launch_pair(int r, const void* A, const void* W, const void* LA,
+moe_status_t launch_pair(int r, const void* A, const void* W, const void* XA,
                          const void* LB, const GemmArgs& args, cudaStream_t st) {
-  if (r == 16) return launch_pair_t<MODE, pair_bn(MODE, 16), 16>(A, W, LA, LB, args, st);
-  if (r == 32) return launch_pair_t<MODE, pair_bn(MODE, 32), 32>(A, W, LA, LB, args, st);
-  if (r == 64) return launch_pair_t<MODE, pair_bn(MODE, 64), 64>(A, W, LA, LB, args, st);
+  if (r == 16) return launch_pair_t<MODE, 16>(A, W, XA, LB, args, st);
+  if (r == 32) return launch_pair_t<MODE, 32>(A, W, XA, LB, args, st);
+  if (r == 64) return launch_pair_t<MODE, 64>(A, W, XA, LB, args, st);
   return MOE_ERR_UNSUPPORTED;
 }
 
@@ -315,16 +306,20 @@ moe_status_t launch_grad_t(const CUtensorMap* u, const CUtensorMap* v,
 }
 
 // Saved-activation parts (bytes from the start of `saved`).
-void saved_layout(int R, int H, int I, int r, size_t off[5]) {
+constexpr int kSavedParts = 6;
+void saved_layout(int R, int H, int I, int r, size_t off[kSavedParts + 1]) {
   (void)H;
   const size_t z1 = static_cast<size_t>(R) * 2 * I * 2;
   const size_t h = static_cast<size_t>(R) * I * 2;
   const size_t xa = static_cast<size_t>(r) * ld_rank(R) * 2;
-  off[0] = 0;
-  off[1] = off[0] + align256(z1);
-  off[2] = off[1] + align256(h);
-  off[3] = off[2] + align256(xa);
-  off[4] = off[3] + align256(xa);
+  const size_t xa_rm = static_cast<size_t>(R) * r * 2;
+  off[0] = 0;                          // Z1 [R, 2I]
+  off[1] = off[0] + align256(z1);      // h [R, I]
+  off[2] = off[1] + align256(h);       // XA1t [r, ldR]
+  off[3] = off[2] + align256(xa);      // HA2t [r, ldR]
+  off[4] = off[3] + align256(xa);      // XA1 [R, r]
+  off[5] = off[4] + align256(xa_rm);   // HA2 [R, r]
+  off[6] = off[5] + align256(xa_rm);
 }
 
 // Backward scratch parts.
@@ -475,15 +470,18 @@ moe_status_t launch_router_logits_t(const void* X, const void* Wr, int T, int H,
   return launch_status();
 }
 
-template <int RK>
+template <int RK, bool KMAJ_F>
 moe_status_t launch_rank_down_t(const void* U, const void* F, int K, const int32_t* offsets,
                                 int E, int R, float s, void* out_rm, void* out_t,
                                 cudaStream_t st) {
-  using C = RankDownCfg<RK>;
+  using C = RankDownCfg<RK, KMAJ_F>;
   CUtensorMap tu, tf;
   const uint64_t EU = static_cast<uint64_t>(E);
   bool ok = tmap_2d(&tu, U, K, R, K * 2ull, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok = ok && tmap_2d(&tf, F, RK, EU * K, RK * 2ull, RK, 64, lora_swizzle(RK));
+  if constexpr (KMAJ_F)  // F^T = A [E * r, K]
+    ok = ok && tmap_2d(&tf, F, K, EU * RK, K * 2ull, 64, RK, CU_TENSOR_MAP_SWIZZLE_128B);
+  else                   // F = B [E * K, r]
+    ok = ok && tmap_2d(&tf, F, RK, EU * K, RK * 2ull, RK, 64, lora_swizzle(RK));
   if (!ok) return MOE_ERR_CUDA;
   RankDownArgs a{};
   a.offsets = offsets;
@@ -492,7 +490,7 @@ moe_status_t launch_rank_down_t(const void* U, const void* F, int K, const int32
   a.out_t = static_cast<__nv_bfloat16*>(out_t);
   a.ld_t = ld_rank(R);
   a.wait_ns = g_wait_limit_ns;
-  auto kern = rank_down_kernel<RK>;
+  auto kern = rank_down_kernel<RK, KMAJ_F>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM_BYTES) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -504,12 +502,18 @@ moe_status_t launch_rank_down_t(const void* U, const void* F, int K, const int32
   return launch_status();
 }
 
-// s U_e F[e] per expert, row-major [R, r] and transposed [r, ldR].
-moe_status_t rank_down(int r, const void* U, const void* F, int K, const int32_t* offsets,
-                       int E, int R, float s, void* out_rm, void* out_t, cudaStream_t st) {
-  if (r == 16) return launch_rank_down_t<16>(U, F, K, offsets, E, R, s, out_rm, out_t, st);
-  if (r == 32) return launch_rank_down_t<32>(U, F, K, offsets, E, R, s, out_rm, out_t, st);
-  if (r == 64) return launch_rank_down_t<64>(U, F, K, offsets, E, R, s, out_rm, out_t, st);
+// s U_e F[e] per expert, row-major [R, r] and transposed [r, ldR]; F is
+// B [E, K, r] (backward) or, with kmaj_f, A [E, r, K] (forward: s U A^T).
+moe_status_t rank_down(int r, bool kmaj_f, const void* U, const void* F, int K,
+                       const int32_t* offsets, int E, int R, float s, void* out_rm,
+                       void* out_t, cudaStream_t st) {
+#define MOE_RANK_DOWN(RK_)                                                                   \
+  return kmaj_f ? launch_rank_down_t<RK_, true>(U, F, K, offsets, E, R, s, out_rm, out_t, st) \
+                : launch_rank_down_t<RK_, false>(U, F, K, offsets, E, R, s, out_rm, out_t, st)
+  if (r == 16) MOE_RANK_DOWN(16);
+  if (r == 32) MOE_RANK_DOWN(32);
+  if (r == 64) MOE_RANK_DOWN(64);
+#undef MOE_RANK_DOWN
   return MOE_ERR_UNSUPPORTED;
 }
 
@@ -782,14 +786,14 @@ moe_status_t moe_router_bwd(const float* w, const float* dw, const int32_t* topk
 // ------------------------------------------------------------------ sizes
 size_t moe_saved_bytes(int R, int H, int I, int r) {
   if (R < 0 || H <= 0 || I <= 0 || r <= 0) return 0;
-  size_t off[5];
+  size_t off[kSavedParts + 1];
   saved_layout(R, H, I, r, off);
-  return off[4];
+  return off[kSavedParts];
 }
 
 size_t moe_saved_part_offset(int R, int H, int I, int r, int part) {
-  if (part < 0 || part > 4 || R < 0) return 0;
-  size_t off[5];
+  if (part < 0 || part > kSavedParts || R < 0) return 0;
+  size_t off[kSavedParts + 1];
   saved_layout(R, H, I, r, off);
   return off[part];
 }
@@ -816,12 +820,14 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     return MOE_ERR_INVALID_ARG;
   if (saved_bytes < moe_saved_bytes(R, H, I, r)) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = stream;
-  size_t off[5];
+  size_t off[kSavedParts + 1];
   saved_layout(R, H, I, r, off);
   __nv_bfloat16* Z1 = at<__nv_bfloat16>(saved, off[0]);
   __nv_bfloat16* h = at<__nv_bfloat16>(saved, off[1]);
   __nv_bfloat16* xa1 = at<__nv_bfloat16>(saved, off[2]);
   __nv_bfloat16* ha2 = at<__nv_bfloat16>(saved, off[3]);
+  __nv_bfloat16* xa1_rm = at<__nv_bfloat16>(saved, off[4]);
+  __nv_bfloat16* ha2_rm = at<__nv_bfloat16>(saved, off[5]);
   moe_status_t stt;
   if ((stt = zero_rank_padding(xa1, R, r, st)) != MOE_OK) return stt;
   if ((stt = zero_rank_padding(ha2, R, r, st)) != MOE_OK) return stt;
@@ -830,15 +836,19 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
 
   // gate_up + SwiGLU
   if (use_pairs(R, E, H, false)) {
-    const int bn = pair_bn(kGateUpFwd, r), half = bn / 2;
+    // s Xp A1^T (both layouts) on its own pass, then the GEMM
+    if ((stt = rank_down(r, true, Xp, A1, H, expert_offsets, E, R, s, xa1_rm, xa1, st)) !=
+        MOE_OK)
+      return stt;
+    const int oc = pair_out_cols(kGateUpFwd);
     GemmArgs g{};
     g.offsets = expert_offsets;
-    g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + half - 1) / half; g.I = I;
+    g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + oc - 1) / oc; g.I = I;
     g.b_rows = 2 * I; g.lb_rows = 2 * I; g.s = s;
     g.out = h; g.ld_out = I; g.out2 = Z1; g.ld_out2 = 2 * I;
-    g.lora_t = xa1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
     g.stall_test = g_stall_test;
-    if ((stt = launch_pair<kGateUpFwd>(r, Xp, W1, A1, B1, g, st)) != MOE_OK) return stt;
+    if ((stt = launch_pair<kGateUpFwd>(r, Xp, W1, xa1_rm, B1, g, st)) != MOE_OK) return stt;
   } else {
     const int bn = pick_bn(I, true, r, false), half = bn / 2;
     CUtensorMap ta, tb, tla, tlb;
@@ -858,15 +868,18 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
   }
   // down
   if (use_pairs(R, E, I, false)) {
-    const int bn = pair_bn(kDownFwd, r);
+    if ((stt = rank_down(r, true, h, A2, I, expert_offsets, E, R, s, ha2_rm, ha2, st)) !=
+        MOE_OK)
+      return stt;
+    const int oc = pair_out_cols(kDownFwd);
     GemmArgs g{};
     g.offsets = expert_offsets;
-    g.E = E; g.R = R; g.K = I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
+    g.E = E; g.R = R; g.K = I; g.N = H; g.n_tiles = (H + oc - 1) / oc; g.I = I;
     g.b_rows = H; g.lb_rows = H; g.s = s;
     g.out = static_cast<__nv_bfloat16*>(Z2); g.ld_out = H;
-    g.lora_t = ha2; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
     g.stall_test = g_stall_test;
-    if ((stt = launch_pair<kDownFwd>(r, h, W2, A2, B2, g, st)) != MOE_OK) return stt;
+    if ((stt = launch_pair<kDownFwd>(r, h, W2, ha2_rm, B2, g, st)) != MOE_OK) return stt;
   } else {
     const int bn = pick_bn(H, false, r, false);
     CUtensorMap ta, tb, tla, tlb;
@@ -924,7 +937,7 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     return MOE_ERR_INVALID_ARG;
   if (saved_bytes < moe_saved_bytes(R, H, I, r)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_workspace_bytes(R, E, H, I, r)) return MOE_ERR_INVALID_ARG;
-  size_t so[5], wo[10];
+  size_t so[kSavedParts + 1], wo[10];
   saved_layout(R, H, I, r, so);
   bwd_layout(R, E, H, I, r, wo);
   const __nv_bfloat16* Z1 = at<__nv_bfloat16>(saved, so[0]);
@@ -967,7 +980,7 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
 
   // down backward: dh = dZ2 W2 + s (dZ2 B2) A2, SwiGLU backward -> dZ1
   if (pair_down) {
-    const int bn = pair_bn(kDownBwd, r);
+    const int bn = pair_out_cols(kDownBwd);
     GemmArgs g{};
     g.offsets = expert_offsets;
     g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + bn - 1) / bn; g.I = I;
@@ -976,7 +989,8 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
     g.stall_test = g_stall_test;
     // s dZ2 B2 (both layouts) on its own pass, then the GEMM
-    if ((stt = rank_down(r, dZ2, B2, H, expert_offsets, E, R, s, dzb2_rm, dzb2, st)) != MOE_OK)
+    if ((stt = rank_down(r, false, dZ2, B2, H, expert_offsets, E, R, s, dzb2_rm, dzb2, st)) !=
+        MOE_OK)
       return stt;
     if ((stt = launch_pair<kDownBwd>(r, dZ2, W2, dzb2_rm, A2t, g, st)) != MOE_OK) return stt;
   } else {
@@ -998,7 +1012,7 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
   }
   // gate_up backward: dXp = dZ1 W1 + s (dZ1 B1) A1
   if (pair_gate_up) {
-    const int bn = pair_bn(kGateUpBwd, r);
+    const int bn = pair_out_cols(kGateUpBwd);
     GemmArgs g{};
     g.offsets = expert_offsets;
     g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
@@ -1006,7 +1020,7 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
     g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
     g.stall_test = g_stall_test;
-    if ((stt = rank_down(r, dZ1, B1, 2 * I, expert_offsets, E, R, s, dzb1_rm, dzb1, st)) !=
+    if ((stt = rank_down(r, false, dZ1, B1, 2 * I, expert_offsets, E, R, s, dzb1_rm, dzb1, st)) !=
         MOE_OK)
       return stt;
     if ((stt = launch_pair<kGateUpBwd>(r, dZ1, W1, dzb1_rm, A1t, g, st)) != MOE_OK) return stt;

@@ -1,11 +1,13 @@
-// Rank-r down-projection of the backward on its own pass (used with the
-// CTA-pair backward GEMMs, whose weight operand then holds whole weight atoms
-// only): per expert e with rows [a, b)
+// Rank-r down-projections on their own pass (used with the CTA-pair GEMMs,
+// whose weight operand then holds whole weight atoms only): per expert e
+// with rows [a, b)
 //   V[a:b] = s * U[a:b] F[e]       [M_e, r]
-// with (U, F) = (dZ2, B2) -> s dZ2 B2 and (dZ1, B1) -> s dZ1 B1.  U [R, K] is
-// a K-major operand, F[e] [K, r] is read in place as an MN-major operand
-// (one r-column atom).  Written twice: row-major [R, r] (the A operand of the
-// up-projection MMA) and transposed [r, ldR] (the LoRA-gradient kernel's
+// Backward: (U, F) = (dZ2, B2) -> s dZ2 B2 and (dZ1, B1) -> s dZ1 B1, with
+// F[e] [K, r] read in place as an MN-major operand (one r-column atom).
+// Forward: (U, F) = (Xp, A1^T) -> s Xp A1^T and (h, A2^T) -> s h A2^T, with
+// F[e]^T = A[e] [r, K] read in place as a K-major operand.  U [R, K] is a
+// K-major operand.  Written twice: row-major [R, r] (the A operand of the
+// up-projection MMA) and transposed [r, ldR] (the saved / LoRA-gradient
 // operand).  Memory-bound: U is streamed once.
 #pragma once
 
@@ -13,7 +15,7 @@
 
 namespace moe {
 
-template <int RK>
+template <int RK, bool KMAJ_F>
 struct RankDownCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr int A_BYTES = BM * BK * 2;
@@ -42,11 +44,11 @@ struct RankDownArgs {
   uint64_t wait_ns;
 };
 
-template <int RK>
+template <int RK, bool KMAJ_F>
 __global__ void __launch_bounds__(192, 1)
     rank_down_kernel(const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmF, const RankDownArgs args) {
-  using C = RankDownCfg<RK>;
+  using C = RankDownCfg<RK, KMAJ_F>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -112,7 +114,10 @@ __global__ void __launch_bounds__(192, 1)
           uint8_t* st = sStage + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
           tma_load_2d_hint(st, &tmU, &full[stage], kt * C::BK, row0, pol_u);
-          tma_load_2d(st + C::A_BYTES, &tmF, &full[stage], 0, e * args.k_rows + kt * C::BK);
+          if constexpr (KMAJ_F)  // A[e] rows: r rows x 64 K-columns
+            tma_load_2d(st + C::A_BYTES, &tmF, &full[stage], kt * C::BK, e * RK);
+          else                   // B[e] rows: 64 K-rows x r columns
+            tma_load_2d(st + C::A_BYTES, &tmF, &full[stage], 0, e * args.k_rows + kt * C::BK);
           if (armed < C::NS) ++armed;
           if (++stage == C::NS) {
             stage = 0;
@@ -132,7 +137,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t kIdesc = idesc_bf16_f32(128, RK, false, true);
+    constexpr uint32_t kIdesc = idesc_bf16_f32(128, RK, false, !KMAJ_F);
     int stage = 0;
     uint32_t phase = 0;
     int local = 0;
@@ -151,8 +156,9 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk)
             umma_bf16(t_acc, smem_desc(a0 + kk * 32, 16, 1024, kLayoutSW128),
-                      smem_desc(b0 + kk * 16 * RK * 2, 16, C::FSBO, C::FLAYOUT), kIdesc,
-                      (kt | kk) ? 1u : 0u);
+                      KMAJ_F ? smem_desc(b0 + kk * 32, 16, 1024, kLayoutSW128)
+                             : smem_desc(b0 + kk * 16 * RK * 2, 16, C::FSBO, C::FLAYOUT),
+                      kIdesc, (kt | kk) ? 1u : 0u);
           umma_commit(&empty[stage]);
         }
         __syncwarp();

@@ -47,8 +47,9 @@ def test_sizes(L):
     R, H, I, r = 1000, 256, 512, 16
     sb = L.moe_saved_bytes(R, H, I, r)
     assert sb >= R * 2 * I * 2 + R * I * 2 + 2 * r * 1024 * 2
-    offs = [L.moe_saved_part_offset(R, H, I, r, p) for p in range(5)]
-    assert offs == sorted(offs) and offs[0] == 0 and offs[4] == sb
+    offs = [L.moe_saved_part_offset(R, H, I, r, p) for p in range(7)]
+    assert offs == sorted(offs) and offs[0] == 0 and offs[6] == sb
+    assert offs[5] - offs[4] >= R * r * 2 and sb - offs[5] >= R * r * 2
     assert all(o % 256 == 0 for o in offs)
     assert L.moe_workspace_bytes(R, 8, H, I, r) >= R * 2 * I * 2
     assert L.moe_route_workspace_bytes(512, 8, 2) >= 512 * 2 * 4
