@@ -40,6 +40,7 @@ struct GemmArgs {
   int E, R, K;
   int N;                   // output columns (I for gate_up fwd / down bwd)
   int n_tiles;             // tiles along N
+  int tile_n;              // CTA-pair kernels: columns per tile (MMA N)
   int I;                   // gate/up split
   int b_rows;              // rows per expert in B's 2-D view
   int lb_rows;             // rows per expert in LB's 2-D view
@@ -362,12 +363,13 @@ __device__ __forceinline__ void epi_rank_handoff(const GemmArgs& args, uint32_t 
 // SwiGLU backward: pull this row's saved gate / up segments (this warp's
 // share of the columns) into L2 while the up-projection and the next tile's
 // mainloop run.
+// The tile's columns start at output column col0.
 template <int BN>
 __device__ __forceinline__ void epi_prefetch_saved(const GemmArgs& args, int grow,
-                                                   bool rvalid, int nt, int ehalf) {
+                                                   bool rvalid, int col0, int ehalf) {
   if (!rvalid) return;
   using S = ColSplit<BN>;
-  const int c0 = nt * BN + (ehalf ? S::C0 : 0);
+  const int c0 = col0 + (ehalf ? S::C0 : 0);
   const int ncol = min(ehalf ? S::C1 : S::C0, args.N - c0);
   if (ncol > 0) {
     const __nv_bfloat16* gp = args.aux + static_cast<size_t>(grow) * args.ld_aux + c0;
@@ -379,10 +381,13 @@ __device__ __forceinline__ void epi_prefetch_saved(const GemmArgs& args, int gro
 // Epilogue step 2: drain the accumulator of this thread's row with the
 // mode's math (SwiGLU; plain store; SwiGLU backward).
 // Non-SwiGLU modes can drain a part of the tile: NC columns starting at
-// tile column cbase (TMEM column t_acc holds tile column cbase).
+// tile column cbase (TMEM column t_acc holds tile column cbase), writing no
+// output column at or beyond nlim.
 template <int MODE, int BN, bool kSplit, int NC = BN>
 __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, int grow,
-                                          bool rvalid, int nt, int ehalf, int cbase = 0) {
+                                          bool rvalid, int nt, int ehalf, int cbase = 0,
+                                          int nlim = 0x7fffffff) {
+  const int nmax = min(args.N, nlim);
   constexpr bool kSwiGLU = (MODE == kGateUpFwd);
   constexpr int HALF = BN / 2;
   const uint64_t pol = policy_evict_first();  // outputs stream out of L2
@@ -424,15 +429,15 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
         gv[q] = uv[q] = make_uint4(0, 0, 0, 0);
         if (q + 1 < W / 8) gv[q + 1] = uv[q + 1] = make_uint4(0, 0, 0, 0);
         if (!rvalid) continue;
-        if (q + 1 < W / 8 && a32 && col + 16 <= args.N) {
+        if (q + 1 < W / 8 && a32 && col + 16 <= nmax) {
           ld_global_nc_v8(grow_p + col, gv[q], gv[q + 1]);
           ld_global_nc_v8(grow_p + args.I + col, uv[q], uv[q + 1]);
         } else {
-          if (col < args.N) {
+          if (col < nmax) {
             gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
             uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
           }
-          if (q + 1 < W / 8 && col + 8 < args.N) {
+          if (q + 1 < W / 8 && col + 8 < nmax) {
             gv[q + 1] = *reinterpret_cast<const uint4*>(grow_p + col + 8);
             uv[q + 1] = *reinterpret_cast<const uint4*>(grow_p + args.I + col + 8);
           }
@@ -460,7 +465,7 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
             }
           }
         }
-        const int col = col0 + c, nv = args.N - col;
+        const int col = col0 + c, nv = nmax - col;
         store_row_bf16<W>(orow + col, dg, nv, pol);
         store_row_bf16<W>(orow + args.I + col, du, nv, pol);
       }
@@ -473,7 +478,7 @@ __device__ __forceinline__ void epi_drain(const GemmArgs& args, uint32_t t_acc, 
       float v[W];
       tmem_ld<W>(t_acc + c, v);
       tmem_ld_wait();
-      if (rvalid) store_row_bf16<W>(orow + c + col0, v, args.N - col0 - c, pol);
+      if (rvalid) store_row_bf16<W>(orow + c + col0, v, nmax - col0 - c, pol);
     });
   }
 }
@@ -778,7 +783,7 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&xa_ready[b]);
       }
-      if constexpr (MODE == kDownBwd) epi_prefetch_saved<BN>(args, grow, rvalid, nt, ehalf);
+      if constexpr (MODE == kDownBwd) epi_prefetch_saved<BN>(args, grow, rvalid, nt * BN, ehalf);
 
       if (!MOE_TIMED(MODE, 9, warp_wait(&acc_full[b], use, s_abort, wait_ns))) break;
       tc_fence_after();

@@ -15,17 +15,23 @@
 // K = r -- are loaded by TMA beside the tile and accumulated into the same
 // TMEM tile right after the mainloop: W + s B A is never formed.
 //
-// B operand of each CTA (128 of the tile's 256 columns):
+// Tile width Nt (the MMA's N), per launch: 256 for gate_up forward; down
+// forward: the narrowest multiple of 16 that covers N in as many tiles as
+// 256 would (N = 2880: 12 tiles of 240, no padded columns); backward: 128 or
+// 256 (whole MN-major atoms; any multiple of 16 computes correctly, but
+// partial atoms run slower).  B operand of each CTA (Nt / 2 columns):
 //   gate_up fwd: [gate j..j+63 | up j..j+63] with j = 128 nt + 64 rank, so
 //                every 128 tile columns hold gate and up of the same 64
 //                output columns (the SwiGLU epilogue needs both in one
 //                thread, also for half tiles);
-//   down fwd:    W2 rows 256 nt + 128 rank .. +127 (K-major);
-//   backward:    W read in place as [K, N], MN-major atoms of 64 columns.
+//   down fwd:    W2 rows Nt nt + Nt/2 rank .. (K-major);
+//   backward:    W read in place as [K, N], two MN-major atoms of 64
+//                columns from column Nt nt + Nt/2 rank (the MMA reads the
+//                first Nt/2).
 // Half tiles: an expert's last tile with at most 128 rows of the expert runs
 // on the M = 128 pair instruction (64 rows per CTA); its accumulator sits in
-// TMEM as lanes 0-63 = the CTA's 64 rows for tile columns [0, 128) and lanes
-// 64-127 = the same rows for [128, 256) (measured).
+// TMEM as lanes 0-63 = the CTA's 64 rows for tile columns [0, Nt/2) and
+// lanes 64-127 = the same rows for [Nt/2, Nt) (measured).
 //
 // Synchronisation (every wait bounded):
 //  * both CTAs' TMA loads of a stage complete on the leader's barrier (the
@@ -221,6 +227,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
   const uint32_t tmem_base = *s_tmem;
   const int total_tiles = s_mstart[E] * args.n_tiles;
   const int k_iters = (args.K + C::BK - 1) / C::BK;
+  // tile width (MMA N) and this CTA's share of it
+  const int Nt = kSwiGLU ? BN : args.tile_n;
+  const int NHt = Nt >> 1;
+  // bytes of one CTA's half of a stage (down fwd: Nt/2 weight rows)
+  const uint32_t stage_bytes = (kSwiGLU || kBMN)
+                                   ? static_cast<uint32_t>(C::STAGE_BYTES)
+                                   : static_cast<uint32_t>(C::A_BYTES + NHt * C::BK * 2);
   // cluster addresses of the leader's copies of the barriers
   auto lead = [&](const void* p) { return mapa_shared(smem_u32(p), 0); };
 
@@ -248,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
         const int row0 = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * rows_per_cta;
         // first weight / up-factor row of this CTA's tile columns
         const int n0 = kSwiGLU ? nt * (BN / 2) + static_cast<int>(rank) * 64
-                               : nt * BN + static_cast<int>(rank) * C::NH;
+                               : nt * Nt + static_cast<int>(rank) * NHt;
         const int b = local & 1;
         const uint32_t use = (local >> 1) & 1;
         if (!mbar_wait(&lb_empty[b], use ^ 1, s_abort, wait_ns)) { ok = false; break; }
@@ -271,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
           uint8_t* sb = st + C::A_BYTES;
           const int kx = kt * C::BK;
           const uint32_t fb = lead(&full[stage]);
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
           tma_load_2d_pair_hint(st, &tmA, fb, kx, row0, pol_a);
           if constexpr (kBMN) {
             // W [K, N] in place: this CTA's 128 tile columns as two 64-column
@@ -302,10 +315,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
       // ---------------------------------------------------------- MMA (leader)
       // The whole warp runs the loop (its state stays warp-uniform); one
       // elected lane issues the tensor-core instructions.
-      constexpr uint32_t kIdesc = idesc_bf16_f32(256, BN, false, kBMN);
-      constexpr uint32_t kIdescH = idesc_bf16_f32(128, BN, false, kBMN);
-      constexpr uint32_t kIdescUp = idesc_bf16_f32(256, BN, false, false);
-      constexpr uint32_t kIdescUpH = idesc_bf16_f32(128, BN, false, false);
+      const uint32_t kIdesc = idesc_bf16_f32(256, Nt, false, kBMN);
+      const uint32_t kIdescH = idesc_bf16_f32(128, Nt, false, kBMN);
+      const uint32_t kIdescUp = idesc_bf16_f32(256, Nt, false, false);
+      const uint32_t kIdescUpH = idesc_bf16_f32(128, Nt, false, false);
       constexpr uint16_t kBoth = 0x3;
       const uint64_t a_desc0 = smem_desc(smem_u32(sStage), 16, 1024, kLayoutSW128);
       // MN-major: LBO = next 64-column atom, SBO = next 8 K-rows (8 x 128 B)
@@ -399,27 +412,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
                        static_cast<int>(rank) * (half ? C::BM / 2 : C::BM) + row_local;
       const bool rvalid = grow < s_off[e + 1];
       const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
+      const int col0 = nt * Nt;             // first output column of the tile
+      const int cend = min(args.N, col0 + Nt);
       if constexpr (MODE == kDownBwd) {
-        if (!half) epi_prefetch_saved<BN>(args, grow, rvalid, nt, ehalf);
+        if (!half) epi_prefetch_saved<BN>(args, grow, rvalid, col0, ehalf);
       }
       if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
       tc_fence_after();
       if constexpr (kSwiGLU) {
         // 128-column blocks [gate 64 | up 64] of output columns
         // 128 nt + 64 q .. +63, q = the block
-        const int col0 = nt * (BN / 2);
+        const int oc0 = nt * (BN / 2);
         if (half) {
-          epi_swiglu_seg64(args, t_acc, grow, rvalid, col0 + (ew >> 1) * 64, pol);
+          epi_swiglu_seg64(args, t_acc, grow, rvalid, oc0 + (ew >> 1) * 64, pol);
         } else {
-          epi_swiglu_seg64(args, t_acc, grow, rvalid, col0, pol);
-          epi_swiglu_seg64(args, t_acc + 128, grow, rvalid, col0 + 64, pol);
+          epi_swiglu_seg64(args, t_acc, grow, rvalid, oc0, pol);
+          epi_swiglu_seg64(args, t_acc + 128, grow, rvalid, oc0 + 64, pol);
         }
       } else {
-        if (half)
-          epi_drain<MODE, BN, kSplit, BN / 2>(args, t_acc, grow, rvalid, nt, ehalf,
-                                              (ew >> 1) * (BN / 2));
-        else
-          epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, nt, ehalf);
+        // tile columns [0, Nt) = output columns col0 + c; TMEM columns past
+        // Nt (or past N) hold nothing of this tile and are not stored
+        if (half) {
+          const int q = ew >> 1;
+          epi_drain<MODE, BN, kSplit, BN / 2>(args, t_acc, grow, rvalid, 0, ehalf,
+                                              col0 + q * NHt,
+                                              min(cend, col0 + (q + 1) * NHt));
+        } else {
+          epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, 0, ehalf, col0, cend);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -442,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
       drain_wait(drained, 0, wait_ns);        // the leader saw every copy land
     } else {
       drain_wait_cluster(peer_done, 0, wait_ns);
-      drain_pair_copies(full, C::NS, C::STAGE_BYTES, s_issued[0], s_issued[2], wait_ns);
+      drain_pair_copies(full, C::NS, stage_bytes, s_issued[0], s_issued[2], wait_ns);
       drain_pair_copies(lb_full, 2, C::UP_BYTES, s_issued[1], s_issued[3], wait_ns);
       mbar_arrive_cluster(mapa_shared(smem_u32(drained), 1));
     }

@@ -250,7 +250,10 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* XA, const v
     const uint64_t N = static_cast<uint64_t>(args.N);
     ok = ok && tmap_2d(&tw, W, N, EU * args.b_rows, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   } else {
-    ok = ok && tmap_2d(&tw, W, K, EU * args.b_rows, K * 2, 64, C::W_BOX_ROWS,
+    // K-major: gate_up fwd loads 64-row gate / up blocks, down fwd the
+    // tile's Nt / 2 rows per CTA
+    const int wbox = C::kSwiGLU ? C::W_BOX_ROWS : args.tile_n / 2;
+    ok = ok && tmap_2d(&tw, W, K, EU * args.b_rows, K * 2, 64, wbox,
                        CU_TENSOR_MAP_SWIZZLE_128B);
   }
   ok = ok && tmap_2d(&txa, XA, RK, args.R, RK * 2ull, RK, C::BM, lora_swizzle(RK));
@@ -275,9 +278,17 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* XA, const v
   return launch_status();
 }
 
-// Output columns per CTA-pair tile: 128 (gate_up forward: 128 gate + 128 up
-// columns) or 256.
-constexpr int pair_out_cols(int mode) { return mode == kGateUpFwd ? 128 : 256; }
+// Columns per CTA-pair tile (the MMA's N) for N output columns.  K-major
+// weight (down forward): the narrowest multiple of 16 that covers N in as
+// many tiles as 256 would (2880 -> 12 tiles of 240; 2048 -> 256).  MN-major
+// weight (backward): whole 64-column atoms per CTA, 128 or 256 (measured:
+// 240 -- 120-column halves -- slows both backward GEMMs by about 20%).
+// Gate_up forward always uses 256 (128 gate + 128 up columns per tile).
+constexpr int pair_tile_n(int N, bool mn_major) {
+  if (mn_major) return N <= 128 ? 128 : 256;
+  const int tiles = (N + 255) / 256;
+  return 16 * ((N + 16 * tiles - 1) / (16 * tiles));
+}
 
 template <int MODE>
 moe_status_t launch_pair(int r, const void* A, const void* W, const void* XA,
@@ -840,10 +851,10 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     if ((stt = rank_down(r, true, Xp, A1, H, expert_offsets, E, R, s, xa1_rm, xa1, st)) !=
         MOE_OK)
       return stt;
-    const int oc = pair_out_cols(kGateUpFwd);
     GemmArgs g{};
     g.offsets = expert_offsets;
-    g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + oc - 1) / oc; g.I = I;
+    g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + 127) / 128; g.I = I;
+    g.tile_n = 256;
     g.b_rows = 2 * I; g.lb_rows = 2 * I; g.s = s;
     g.out = h; g.ld_out = I; g.out2 = Z1; g.ld_out2 = 2 * I;
     g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
@@ -871,10 +882,11 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     if ((stt = rank_down(r, true, h, A2, I, expert_offsets, E, R, s, ha2_rm, ha2, st)) !=
         MOE_OK)
       return stt;
-    const int oc = pair_out_cols(kDownFwd);
+    const int tn = pair_tile_n(H, false);
     GemmArgs g{};
     g.offsets = expert_offsets;
-    g.E = E; g.R = R; g.K = I; g.N = H; g.n_tiles = (H + oc - 1) / oc; g.I = I;
+    g.E = E; g.R = R; g.K = I; g.N = H; g.n_tiles = (H + tn - 1) / tn; g.I = I;
+    g.tile_n = tn;
     g.b_rows = H; g.lb_rows = H; g.s = s;
     g.out = static_cast<__nv_bfloat16*>(Z2); g.ld_out = H;
     g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
@@ -980,10 +992,11 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
 
   // down backward: dh = dZ2 W2 + s (dZ2 B2) A2, SwiGLU backward -> dZ1
   if (pair_down) {
-    const int bn = pair_out_cols(kDownBwd);
+    const int bn = pair_tile_n(I, true);
     GemmArgs g{};
     g.offsets = expert_offsets;
     g.E = E; g.R = R; g.K = H; g.N = I; g.n_tiles = (I + bn - 1) / bn; g.I = I;
+    g.tile_n = bn;
     g.b_rows = H; g.lb_rows = I; g.s = s;
     g.out = dZ1; g.ld_out = 2 * I; g.aux = Z1; g.ld_aux = 2 * I;
     g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
@@ -1012,10 +1025,11 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
   }
   // gate_up backward: dXp = dZ1 W1 + s (dZ1 B1) A1
   if (pair_gate_up) {
-    const int bn = pair_out_cols(kGateUpBwd);
+    const int bn = pair_tile_n(H, true);
     GemmArgs g{};
     g.offsets = expert_offsets;
     g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
+    g.tile_n = bn;
     g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
     g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
     g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
