@@ -505,7 +505,8 @@ moe_status_t launch_rank_down_t(const void* U, const void* F, int K, const int32
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM_BYTES) != cudaSuccess)
     return MOE_ERR_CUDA;
-  const int grid = static_cast<int>(std::min<long long>(num_sms(), R / 128 + E));
+  const int grid = static_cast<int>(
+      std::min<long long>(static_cast<long long>(num_sms()) * C::CTAS_PER_SM, R / 128 + E));
   if (grid <= 0) return MOE_OK;
   ProfScope prof(MOE_PROF_RANK_DOWN, st);
   kern<<<grid, 192, C::SMEM_BYTES, st>>>(tu, tf, a);

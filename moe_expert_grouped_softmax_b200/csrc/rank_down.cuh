@@ -21,7 +21,14 @@ struct RankDownCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BK * RK * 2;
   static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + 1023) / 1024 * 1024;
-  static constexpr int NS = 8;
+  // CTAs per SM: two CTAs of four stages keep as many bytes in flight as
+  // one of eight, and one CTA's prologue and pipeline fill overlap the
+  // other's streaming
+#ifndef MOE_RANK_CTAS
+#define MOE_RANK_CTAS 2
+#endif
+  static constexpr int CTAS_PER_SM = MOE_RANK_CTAS;
+  static constexpr int NS = 8 / CTAS_PER_SM;
   static constexpr int MISC_BYTES = 256 + 8 * 520;
   static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + MISC_BYTES;
   static constexpr int ACC_STRIDE = RK < 32 ? 32 : RK;
@@ -45,7 +52,7 @@ struct RankDownArgs {
 };
 
 template <int RK, bool KMAJ_F>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, RankDownCfg<RK, KMAJ_F>::CTAS_PER_SM)
     rank_down_kernel(const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmF, const RankDownArgs args) {
   using C = RankDownCfg<RK, KMAJ_F>;
