@@ -968,12 +968,12 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
   if ((stt = zero_rank_padding(dzb2, R, r, st)) != MOE_OK) return stt;
   if ((stt = zero_rank_padding(dzb1, R, r, st)) != MOE_OK) return stt;
   // Operand copies of the LoRA factors: the down-projection factors B2, B1
-  // zero-padded to whole MN-major atoms (64 columns for the single-CTA
-  // kernels, 32 for the CTA-pair kernels; fused into the base MMA), the
-  // up-projection factors A2, A1 transposed to K-major (both kernels).
+  // zero-padded to one 64-column MN-major atom for the single-CTA kernels
+  // (fused into the base MMA; the CTA-pair backward reads them in place in
+  // its rank-r pass), the up-projection factors A2, A1 transposed to K-major
+  // (both kernels).
   const bool pair_down = use_pairs(R, E, H, true);
   const bool pair_gate_up = use_pairs(R, E, 2 * I, true);
-  // (the CTA-pair backward reads B2, B1 in place in its rank-r pass)
   FactorPrep prep;
   if (r < 64 && !pair_down) {
     B2p = at<__nv_bfloat16>(ws, wo[3]);
