@@ -257,10 +257,10 @@ MOE_API unsigned long long moe_kernel_launches(void);
  * the next moe_lora_mlp_fwd / moe_lora_mlp_bwd call): mode > 0 runs them on
  * CTA pairs (256-row tiles on the 2-SM tensor-core instruction), mode == 0
  * on single CTAs (128-row tiles), mode < 0 (the default) chooses per GEMM:
- * pairs when the mean rows per expert R / E is at least 768 (little padding
- * on each expert's ragged last 256-row tile) and the GEMM's K is at least
- * 1024 (H for gate_up forward and down backward, I for down forward, 2I for
- * gate_up backward).  A GEMM on pairs takes its rank-r product (s Xp A1^T,
+ * pairs when the mean rows per expert R / E is at least 256 (one 256-row
+ * tile; an expert's last tile with at most 128 rows runs as a half tile)
+ * and the GEMM's K is at least 768 (H for gate_up forward and down
+ * backward, I for down forward, 2I for gate_up backward).  A GEMM on pairs takes its rank-r product (s Xp A1^T,
  * s h A2^T, s dZ2 B2 or s dZ1 B1) from a separate memory-bound pass.  All
  * compute the same result to the tolerance of bf16 rounding. */
 MOE_API void moe_set_cta_pairs(int mode);

@@ -83,6 +83,10 @@ __device__ __forceinline__ bool pair_half_tile(const int* s_off, int e, int mt) 
 #ifndef MOE_PAIR_HINTS
 #define MOE_PAIR_HINTS 1
 #endif
+// Tile order of the pair kernels (see decode_tile): m-tiles fastest.
+#ifndef MOE_PAIR_TILE_ORDER
+#define MOE_PAIR_TILE_ORDER 1
+#endif
 
 template <int MODE, int RK>
 struct PairCfg {
@@ -256,7 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
 #endif
       for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++local) {
         int e, mt, nt;
-        decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+        decode_tile<MOE_PAIR_TILE_ORDER>(tile, args.n_tiles, s_mstart, E, e, mt, nt);
         const int rows_per_cta = pair_half_tile(s_off, e, mt) ? C::BM / 2 : C::BM;
         const int row0 = s_off[e] + mt * 2 * C::BM + static_cast<int>(rank) * rows_per_cta;
         // first weight / up-factor row of this CTA's tile columns
@@ -341,7 +345,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
         const uint32_t use = (local >> 1) & 1;
         const uint32_t t_acc = tmem_base + b * C::ACC_STRIDE;
         int e, mt, nt;
-        decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+        decode_tile<MOE_PAIR_TILE_ORDER>(tile, args.n_tiles, s_mstart, E, e, mt, nt);
         const bool half = pair_half_tile(s_off, e, mt);
         const uint32_t idesc = half ? kIdescH : kIdesc;
         const uint32_t idesc_up = half ? kIdescUpH : kIdescUp;
@@ -401,7 +405,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
     int local = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++local) {
       int e, mt, nt;
-      decode_tile(tile, args.n_tiles, s_mstart, E, e, mt, nt);
+      decode_tile<MOE_PAIR_TILE_ORDER>(tile, args.n_tiles, s_mstart, E, e, mt, nt);
       const int b = local & 1;
       const uint32_t use = (local >> 1) & 1;
       const bool half = pair_half_tile(s_off, e, mt);
@@ -414,9 +418,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
       const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
       const int col0 = nt * Nt;             // first output column of the tile
       const int cend = min(args.N, col0 + Nt);
-      if constexpr (MODE == kDownBwd) {
-        if (!half) epi_prefetch_saved<BN>(args, grow, rvalid, col0, ehalf);
-      }
+      // (no L2 prefetch of the saved gate / up rows here: measured 1.5%
+      // slower in this kernel)
       if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
       tc_fence_after();
       if constexpr (kSwiGLU) {

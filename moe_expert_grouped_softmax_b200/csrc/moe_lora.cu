@@ -63,11 +63,13 @@ inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed);
 int g_stall_test = 0;                      // testing hook, see moe_test_inject_stall
 int g_cta_pairs = -1;                      // grouped GEMMs on CTA pairs: <0 auto
 // Automatic choice (measured): a GEMM runs on CTA pairs when the mean rows
-// per expert fill at least three 256-row tiles (little padding on each
-// expert's ragged last tile) and K is long enough (16 k-steps) for the
-// per-tile work around the mainloop to stay hidden.
-constexpr int kPairMinRowsPerExpert = 768;
-constexpr int kPairMinK = 1024;
+// per expert fill at least one 256-row tile (an expert's ragged last tile
+// with at most 128 rows runs as a half tile) and K has at least 12 k-steps.
+// Pairs against single CTAs, whole step: 256 rows per expert, K = 2048 to
+// 7168: -26%; 1024 rows per expert, K = 768 (down forward): -28% on that
+// GEMM.
+constexpr int kPairMinRowsPerExpert = 256;
+constexpr int kPairMinK = 768;
 bool use_pairs(int R, int E, int K, bool backward) {
   (void)backward;
   if (g_cta_pairs >= 0) return g_cta_pairs > 0;
