@@ -463,11 +463,17 @@ def main():
                                  "traffic": traffic.get(kk)}
     hb = WL.hbm_bytes(T, H, E, k)
     hb["lora_grad"] = R * (H + 2 * I + I + H) * 2 + 4 * r * R * 2 + E * r * (3 * H + 3 * I) * 2
-    # rank-r passes of the pair backward: dZ2 (K = H) and dZ1 (K = 2I), mean per launch
-    hb["rank_down"] = (R * (H + 2 * I) * 2 + E * r * (H + 2 * I) * 2 + 2 * 2 * R * r * 2) // 2
+    # rank-r passes (one per GEMM that runs on CTA pairs, which the library
+    # reports): the pass streams U [R, K] and the factor [E, K, r] and writes
+    # [R, r] twice; mean bytes per launch over the passes of one step
+    from moe_expert_grouped_softmax_b200 import ops
+    rank_k = [kr for kr in (H, I, H, 2 * I) if ops.uses_cta_pairs(R, E, kr)]
+    if rank_k:
+        hb["rank_down"] = sum(R * kr * 2 + E * r * kr * 2 + 2 * R * r * 2
+                              for kr in rank_k) // len(rank_k)
     mem = {}
     for kk in ("permute", "unpermute", "route", "lora_grad", "rank_down"):
-        if kk in kern:
+        if kk in kern and kk in hb:
             # permute / unpermute run twice per step with the same bytes
             gbs = hb[kk] / (kern[kk]["avg_ms"] / 1e3) / 1e9
             mem[kk] = {"GB_s": gbs, "frac_of_measured_hbm": gbs / pk["hbm_gbs"],

@@ -152,7 +152,9 @@ MOE_API size_t moe_workspace_bytes(int R, int E, int H, int I, int r);
  * A2 [E, r, I], B2 [E, H, r]; all bf16.  Xp [R, H], Z2 [R, H] bf16.
  * expert_offsets is the device array from moe_route_topk (read on the device;
  * no host synchronisation).  Products accumulate in fp32 on the tensor cores;
- * the rank-r intermediates are rounded to bf16 before the second product. */
+ * the rank-r intermediates are rounded to bf16 before the second product.
+ * `saved` receives the parts listed above; ws / ws_bytes are not used (NULL /
+ * 0 allowed). */
 MOE_API moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets,
                               int E, int H, int I, int r, float s,
                               const void* W1, const void* A1, const void* B1,
@@ -264,6 +266,11 @@ MOE_API unsigned long long moe_kernel_launches(void);
  * s h A2^T, s dZ2 B2 or s dZ1 B1) from a separate memory-bound pass.  All
  * compute the same result to the tolerance of bf16 rounding. */
 MOE_API void moe_set_cta_pairs(int mode);
+/* 1 when a grouped GEMM over R routed rows, E experts and reduction length
+ * K runs on CTA pairs under the current moe_set_cta_pairs setting (and then
+ * takes its rank-r product from the separate pass), else 0; for measurement
+ * (the bytes that pass moves). */
+MOE_API int moe_uses_cta_pairs(int R, int E, int K);
 
 /* Benchmark hook (not thread-safe; for measurement only).
  * moe_profile_enable(1) starts recording, for every kernel kind below, a pair

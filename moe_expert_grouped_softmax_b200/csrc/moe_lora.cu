@@ -559,6 +559,8 @@ unsigned long long moe_kernel_launches(void) {
 
 void moe_set_cta_pairs(int mode) { g_cta_pairs = mode > 0 ? 1 : (mode == 0 ? 0 : -1); }
 
+int moe_uses_cta_pairs(int R, int E, int K) { return use_pairs(R, E, K, false) ? 1 : 0; }
+
 moe_status_t moe_profile_enable(int on) {
   if (on && !g_prof_created) {
     for (int k = 0; k < MOE_PROF_KINDS; ++k)

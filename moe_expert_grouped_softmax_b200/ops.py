@@ -25,7 +25,7 @@ EXPORTS = [
     "moe_saved_bytes", "moe_saved_part_offset", "moe_workspace_bytes",
     "moe_lora_mlp_fwd", "moe_lora_mlp_bwd", "moe_lora_mlp_bwd_full", "moe_get_device_status",
     "moe_status_string", "moe_set_wait_limit_ns", "moe_test_inject_stall",
-    "moe_set_cta_pairs", "moe_kernel_launches", "moe_profile_enable",
+    "moe_set_cta_pairs", "moe_uses_cta_pairs", "moe_kernel_launches", "moe_profile_enable",
     "moe_router_fwd", "moe_router_bwd_workspace_bytes", "moe_router_bwd",
     "moe_profile_collect",
 ]
@@ -90,6 +90,8 @@ def lib():
         L.moe_set_wait_limit_ns.restype = None
         L.moe_set_cta_pairs.argtypes = [I]
         L.moe_set_cta_pairs.restype = None
+        L.moe_uses_cta_pairs.argtypes = [I, I, I]
+        L.moe_uses_cta_pairs.restype = I
         L.moe_kernel_launches.argtypes = []
         L.moe_kernel_launches.restype = ctypes.c_ulonglong
         L.moe_test_inject_stall.argtypes = [I]
@@ -144,6 +146,13 @@ def set_cta_pairs(on=True):
     """Grouped GEMMs on CTA pairs (True, 256-row tiles), single CTAs (False)
     or chosen per GEMM from the rows per expert and K (None, the default)."""
     lib().moe_set_cta_pairs(-1 if on is None else (1 if on else 0))
+
+
+def uses_cta_pairs(R, E, K):
+    """Whether a grouped GEMM over R routed rows, E experts and reduction
+    length K runs on CTA pairs under the current setting (the library's own
+    choice; host-side, no GPU needed)."""
+    return bool(lib().moe_uses_cta_pairs(R, E, K))
 
 
 def test_inject_stall(on=True):

@@ -55,6 +55,24 @@ def test_sizes(L):
     assert L.moe_route_workspace_bytes(512, 8, 2) >= 512 * 2 * 4
 
 
+def test_cta_pair_choice(L):
+    """The grouped-GEMM kernel choice is host logic: pairs from 256 rows per
+    expert and K >= 768 by default, forced either way by moe_set_cta_pairs."""
+    try:
+        assert L.moe_uses_cta_pairs(32768, 32, 2880) == 1      # gpt-oss-20b shape
+        assert L.moe_uses_cta_pairs(65536, 256, 2048) == 1     # 256 rows per expert
+        assert L.moe_uses_cta_pairs(131072, 128, 768) == 1     # K = 768
+        assert L.moe_uses_cta_pairs(65536, 256, 512) == 0      # K too short
+        assert L.moe_uses_cta_pairs(8191, 32, 2880) == 0       # < 256 rows per expert
+        L.moe_set_cta_pairs(1)
+        assert L.moe_uses_cta_pairs(100, 8, 64) == 1
+        L.moe_set_cta_pairs(0)
+        assert L.moe_uses_cta_pairs(32768, 32, 2880) == 0
+    finally:
+        L.moe_set_cta_pairs(-1)
+    assert L.moe_uses_cta_pairs(32768, 32, 2880) == 1
+
+
 def test_host_side_argument_errors(L):
     P = ctypes.c_void_p
     fake = P(256)  # never dereferenced: the call must fail before any launch
