@@ -113,6 +113,8 @@ struct PairCfg {
       RK == 16 ? kLayoutSW32 : (RK == 32 ? kLayoutSW64 : kLayoutSW128);
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_STRIDE = 256;
+  // epilogue warps as in the single-CTA kernel (measured: two per lane
+  // quarter for every mode, each draining half the columns, +0.8% per step)
   static constexpr int EPI_WARPS = gemm_epi_warps(MODE);
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   // weight rows per TMA box: gate_up fwd loads gate and up blocks of 64
@@ -124,7 +126,7 @@ struct PairCfg {
   static_assert(LB_BYTES % 1024 == 0 && XA_BYTES % 1024 == 0, "swizzle atoms");
 };
 
-// SwiGLU epilogue of one 64-column gate / up segment of a row: gate at TMEM
+// SwiGLU epilogue of one 64-column gate / up block of a row: gate at TMEM
 // column t_gate, up at t_gate + 64; output columns col .. col + 63.
 __device__ __forceinline__ void epi_swiglu_seg64(const GemmArgs& args, uint32_t t_gate,
                                                  int grow, bool rvalid, int col,
