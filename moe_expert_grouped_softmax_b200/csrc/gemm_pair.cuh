@@ -95,8 +95,6 @@ struct PairCfg {
   static constexpr int BM = 128, BK = 64;           // rows per CTA, K per stage
   static constexpr int BN = 256;                    // tile columns (MMA N)
   static constexpr int NH = BN / 2;                 // B columns per CTA
-  // output columns per tile (gate_up: 128 gate + 128 up columns)
-  static constexpr int OUT_COLS = kSwiGLU ? BN / 2 : BN;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = NH * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;

@@ -11,6 +11,13 @@
 // order inside one CTA, so the result is deterministic.  The ragged tail of
 // an expert is zeroed in shared memory before its MMA.  Experts with no rows
 // get exact zeros.
+//
+// Tiles are (expert, problem, 128-column block), experts in decreasing order
+// of their row counts (power-of-two buckets, expert index inside a bucket),
+// so that the long reductions of heavily loaded experts start first and the
+// short ones fill in behind them on the persistent CTAs.  Every CTA computes
+// the same order, and each tile is still reduced by one CTA in a fixed
+// order: the results do not depend on it.
 #pragma once
 
 #include "ptx.cuh"
@@ -20,7 +27,7 @@ namespace moe {
 struct GradProblem {
   int P;               // columns of U
   int p_tiles;         // ceil(P / 128)
-  int tile_begin;      // first global tile of this problem
+  int tile_begin;      // first tile of this problem inside an expert's tiles
   int transpose_out;   // 1: out[e][q][p]; 0: out[e][p][q]
   __nv_bfloat16* out;
 };
@@ -28,7 +35,8 @@ struct GradProblem {
 struct GradArgs {
   const int32_t* offsets;
   int E, R;
-  int total_tiles;
+  int tiles_per_expert;  // sum of the problems' p_tiles
+  int total_tiles;       // E * tiles_per_expert
   GradProblem prob[4];
   uint64_t wait_ns;
 };
@@ -39,22 +47,59 @@ struct GradCfg {
   static constexpr int V_BYTES = RK * 64 * 2;    // r rows x 64 columns
   static constexpr int STAGE_BYTES = U_BYTES + V_BYTES;
   static constexpr int NS = 8;
-  static constexpr int MISC_BYTES = 256 + 8 * 520;
+  // barriers, then s_off [E + 1], the expert order [E] and 33 bucket cursors
+  static constexpr int MISC_BYTES = 256 + 4 * (520 + 520 + 64);
   static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + MISC_BYTES;
   static constexpr int ACC_COLS = RK;
   static constexpr int TMEM_COLS = (2 * RK) < 32 ? 32 : 2 * RK;
   static_assert(SMEM_BYTES <= kSmemOptin, "grad kernel shared memory");
 };
 
-__device__ __forceinline__ void grad_decode(const GradArgs& a, int tile, int& pi,
-                                            int& e, int& pt) {
+__device__ __forceinline__ void grad_decode(const GradArgs& a, const int* s_eorder, int tile,
+                                            int& pi, int& e, int& pt) {
+  const int slot = tile / a.tiles_per_expert;
+  const int rem = tile - slot * a.tiles_per_expert;
   pi = 0;
 #pragma unroll
   for (int i = 1; i < 4; ++i)
-    if (tile >= a.prob[i].tile_begin) pi = i;
-  const int local = tile - a.prob[pi].tile_begin;
-  e = local / a.prob[pi].p_tiles;
-  pt = local - e * a.prob[pi].p_tiles;
+    if (rem >= a.prob[i].tile_begin) pi = i;
+  pt = rem - a.prob[pi].tile_begin;
+  e = s_eorder[slot];
+}
+
+// s_eorder[0..E) = the experts by decreasing row-count bucket
+// (floor(log2(rows)); empty experts last), index order inside a bucket.  One
+// warp; deterministic (bucket sizes from a histogram, positions from the
+// lanes' ranks among equal keys, chunks of 32 experts in index order).
+__device__ __forceinline__ void grad_expert_order(const int* s_off, int E, int* s_eorder,
+                                                  int* s_bcur, int lane) {
+  auto bucket = [&](int e) {  // 0 = empty, 1 + floor(log2(rows)) otherwise
+    const int n = s_off[e + 1] - s_off[e];
+    return n > 0 ? 32 - __clz(n) : 0;
+  };
+  for (int b = lane; b < 33; b += 32) s_bcur[b] = 0;
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) atomicAdd(&s_bcur[bucket(e)], 1);
+  __syncwarp();
+  if (lane == 0) {  // exclusive prefix, largest bucket first
+    int acc = 0;
+    for (int b = 32; b >= 0; --b) {
+      const int c = s_bcur[b];
+      s_bcur[b] = acc;
+      acc += c;
+    }
+  }
+  __syncwarp();
+  for (int c0 = 0; c0 < E; c0 += 32) {
+    const int e = c0 + lane;
+    const int key = e < E ? bucket(e) : 33;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (e < E) s_eorder[s_bcur[key] + rank] = e;
+    __syncwarp();
+    if (e < E && rank == 0) s_bcur[key] += __popc(peers);
+    __syncwarp();
+  }
 }
 
 template <int RK>
@@ -81,6 +126,8 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_off = reinterpret_cast<int*>(s_tmem + 4);
+  int* s_eorder = s_off + 520;
+  int* s_bcur = s_eorder + 520;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t wait_ns = args.wait_ns;
@@ -123,6 +170,8 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) set_status(5);
       for (int e = lane; e <= args.E; e += 32) s_off[e] = 0;  // all experts empty
     }
+    __syncwarp();
+    grad_expert_order(s_off, args.E, s_eorder, s_bcur, lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -137,7 +186,7 @@ __global__ void __launch_bounds__(192, 1)
       int armed = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
         int pi, e, pt;
-        grad_decode(args, tile, pi, e, pt);
+        grad_decode(args, s_eorder, tile, pi, e, pt);
         const int a = s_off[e], b = s_off[e + 1];
         const int a8 = a & ~7;  // TMA x coordinate of V must be 16-byte aligned
         const int nk = (b > a) ? ((b - a8 + 63) >> 6) : 0;
@@ -175,7 +224,7 @@ __global__ void __launch_bounds__(192, 1)
     int local = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       int pi, e, pt;
-      grad_decode(args, tile, pi, e, pt);
+      grad_decode(args, s_eorder, tile, pi, e, pt);
       const int a = s_off[e], b = s_off[e + 1];
       const int a8 = a & ~7;
       const int nk = (b > a) ? ((b - a8 + 63) >> 6) : 0;
@@ -237,7 +286,7 @@ __global__ void __launch_bounds__(192, 1)
     int local = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       int pi, e, pt;
-      grad_decode(args, tile, pi, e, pt);
+      grad_decode(args, s_eorder, tile, pi, e, pt);
       const GradProblem& pr = args.prob[pi];
       const int nk = (s_off[e + 1] > s_off[e]) ? 1 : 0;  // any rows at all
       const int bb = local & 1;

@@ -70,8 +70,7 @@ int g_cta_pairs = -1;                      // grouped GEMMs on CTA pairs: <0 aut
 // GEMM.
 constexpr int kPairMinRowsPerExpert = 256;
 constexpr int kPairMinK = 768;
-bool use_pairs(int R, int E, int K, bool backward) {
-  (void)backward;
+bool use_pairs(int R, int E, int K) {
   if (g_cta_pairs >= 0) return g_cta_pairs > 0;
   return static_cast<int64_t>(R) >= static_cast<int64_t>(kPairMinRowsPerExpert) * E &&
          K >= kPairMinK;
@@ -559,7 +558,7 @@ unsigned long long moe_kernel_launches(void) {
 
 void moe_set_cta_pairs(int mode) { g_cta_pairs = mode > 0 ? 1 : (mode == 0 ? 0 : -1); }
 
-int moe_uses_cta_pairs(int R, int E, int K) { return use_pairs(R, E, K, false) ? 1 : 0; }
+int moe_uses_cta_pairs(int R, int E, int K) { return use_pairs(R, E, K) ? 1 : 0; }
 
 moe_status_t moe_profile_enable(int on) {
   if (on && !g_prof_created) {
@@ -851,7 +850,7 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
   const uint64_t EU = static_cast<uint64_t>(E);
 
   // gate_up + SwiGLU
-  if (use_pairs(R, E, H, false)) {
+  if (use_pairs(R, E, H)) {
     // s Xp A1^T (both layouts) on its own pass, then the GEMM
     if ((stt = rank_down(r, true, Xp, A1, H, expert_offsets, E, R, s, xa1_rm, xa1, st)) !=
         MOE_OK)
@@ -883,7 +882,7 @@ moe_status_t moe_lora_mlp_fwd(const void* Xp, const int32_t* expert_offsets, int
     if ((stt = launch_gemm<kGateUpFwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
   // down
-  if (use_pairs(R, E, I, false)) {
+  if (use_pairs(R, E, I)) {
     if ((stt = rank_down(r, true, h, A2, I, expert_offsets, E, R, s, ha2_rm, ha2, st)) !=
         MOE_OK)
       return stt;
@@ -976,8 +975,8 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
   // (fused into the base MMA; the CTA-pair backward reads them in place in
   // its rank-r pass), the up-projection factors A2, A1 transposed to K-major
   // (both kernels).
-  const bool pair_down = use_pairs(R, E, H, true);
-  const bool pair_gate_up = use_pairs(R, E, 2 * I, true);
+  const bool pair_down = use_pairs(R, E, H);
+  const bool pair_gate_up = use_pairs(R, E, 2 * I);
   FactorPrep prep;
   if (r < 64 && !pair_down) {
     B2p = at<__nv_bfloat16>(ws, wo[3]);
@@ -1079,12 +1078,13 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
       if (!ok) return MOE_ERR_CUDA;
       g.prob[i].P = P[i];
       g.prob[i].p_tiles = (P[i] + 127) / 128;
-      g.prob[i].tile_begin = begin;
+      g.prob[i].tile_begin = begin;  // inside one expert's tiles
       g.prob[i].transpose_out = tr[i];
       g.prob[i].out = static_cast<__nv_bfloat16*>(out[i]);
-      begin += E * g.prob[i].p_tiles;
+      begin += g.prob[i].p_tiles;
     }
-    g.total_tiles = begin;
+    g.tiles_per_expert = begin;
+    g.total_tiles = E * begin;
     if (r == 16) stt = launch_grad_t<16>(tu, tv, g, st);
     else if (r == 32) stt = launch_grad_t<32>(tu, tv, g, st);
     else stt = launch_grad_t<64>(tu, tv, g, st);
