@@ -9,9 +9,12 @@
 // MN-major straight from the row-major activations.  The reduction over rows
 // runs in a fixed order inside one CTA (deterministic).  The rows of the next
 // expert inside an expert's last 64-row chunk are zeroed in shared memory
-// before its MMA; experts with no rows get exact zeros.
+// before its MMA; experts with no rows get exact zeros.  Tiles are (expert,
+// problem, p-tile, q-tile), experts in decreasing order of their row counts
+// (the same order in every CTA; see expert_order.cuh).
 #pragma once
 
+#include "expert_order.cuh"
 #include "gemm.cuh"
 
 namespace moe {
@@ -19,14 +22,15 @@ namespace moe {
 struct BaseGradProblem {
   int P, Q;            // columns of U (output rows) and of V (output columns)
   int p_tiles, q_tiles;
-  int tile_begin;      // first global tile of this problem
+  int tile_begin;      // first tile of this problem inside an expert's tiles
   __nv_bfloat16* out;  // [E, P, Q]
 };
 
 struct BaseGradArgs {
   const int32_t* offsets;
   int E, R;
-  int total_tiles;
+  int tiles_per_expert;  // both problems' p_tiles * q_tiles
+  int total_tiles;       // E * tiles_per_expert
   BaseGradProblem prob[2];
   uint64_t wait_ns;
 };
@@ -37,7 +41,8 @@ struct BaseGradCfg {
   static constexpr int U_BYTES = BK * 128 * 2;       // 64 rows x 128 columns
   static constexpr int V_BYTES = BK * BN * 2;        // 64 rows x BN columns
   static constexpr int STAGE_BYTES = U_BYTES + V_BYTES;
-  static constexpr int MISC_BYTES = 256 + 4 * 520;
+  // barriers, then s_off [E + 1], the expert order [E] and 33 bucket cursors
+  static constexpr int MISC_BYTES = 256 + 4 * (520 + 520 + 64);
   static constexpr int NS_FIT = (kSmemOptin - 1024 - MISC_BYTES) / STAGE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + MISC_BYTES;
@@ -47,16 +52,16 @@ struct BaseGradCfg {
   static_assert(NS >= 3, "base-gradient kernel stages");
 };
 
-__device__ __forceinline__ void base_grad_decode(const BaseGradArgs& a, int tile, int& pi,
-                                                 int& e, int& pt, int& qt) {
-  pi = tile >= a.prob[1].tile_begin ? 1 : 0;
+__device__ __forceinline__ void base_grad_decode(const BaseGradArgs& a, const int* s_eorder,
+                                                 int tile, int& pi, int& e, int& pt, int& qt) {
+  const int slot = tile / a.tiles_per_expert;
+  const int rem = tile - slot * a.tiles_per_expert;
+  pi = rem >= a.prob[1].tile_begin ? 1 : 0;
   const BaseGradProblem& p = a.prob[pi];
-  int local = tile - p.tile_begin;
-  const int per_e = p.p_tiles * p.q_tiles;
-  e = local / per_e;
-  local -= e * per_e;
+  const int local = rem - p.tile_begin;
   pt = local / p.q_tiles;       // q-tiles fastest: CTAs at work share U rows
   qt = local - pt * p.q_tiles;
+  e = s_eorder[slot];
 }
 
 template <int BN>
@@ -79,6 +84,8 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_off = reinterpret_cast<int*>(s_tmem + 4);
+  int* s_eorder = s_off + 520;
+  int* s_bcur = s_eorder + 520;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t wait_ns = args.wait_ns;
@@ -119,6 +126,8 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) set_status(5);
       for (int e = lane; e <= args.E; e += 32) s_off[e] = 0;  // all experts empty
     }
+    __syncwarp();
+    expert_load_order(s_off, args.E, s_eorder, s_bcur, lane);
   }
   tc_fence_before();
   __syncthreads();
@@ -136,7 +145,7 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int pi, e, pt, qt;
-        base_grad_decode(args, tile, pi, e, pt, qt);
+        base_grad_decode(args, s_eorder, tile, pi, e, pt, qt);
         const int a = s_off[e], b = s_off[e + 1];
         const int nk = (b - a + C::BK - 1) / C::BK;
         for (int c = 0; c < nk; ++c) {
@@ -179,7 +188,7 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++local) {
       int pi, e, pt, qt;
-      base_grad_decode(args, tile, pi, e, pt, qt);
+      base_grad_decode(args, s_eorder, tile, pi, e, pt, qt);
       const int a = s_off[e], b = s_off[e + 1];
       const int nk = (b - a + C::BK - 1) / C::BK;
       const int bb = local & 1;
@@ -236,7 +245,7 @@ __global__ void __launch_bounds__(192, 1)
     int local = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       int pi, e, pt, qt;
-      base_grad_decode(args, tile, pi, e, pt, qt);
+      base_grad_decode(args, s_eorder, tile, pi, e, pt, qt);
       const BaseGradProblem& pr = args.prob[pi];
       const bool any = s_off[e + 1] > s_off[e];
       const int bb = local & 1;

@@ -21,6 +21,7 @@
 #pragma once
 
 #include "ptx.cuh"
+#include "expert_order.cuh"
 
 namespace moe {
 
@@ -65,41 +66,6 @@ __device__ __forceinline__ void grad_decode(const GradArgs& a, const int* s_eord
     if (rem >= a.prob[i].tile_begin) pi = i;
   pt = rem - a.prob[pi].tile_begin;
   e = s_eorder[slot];
-}
-
-// s_eorder[0..E) = the experts by decreasing row-count bucket
-// (floor(log2(rows)); empty experts last), index order inside a bucket.  One
-// warp; deterministic (bucket sizes from a histogram, positions from the
-// lanes' ranks among equal keys, chunks of 32 experts in index order).
-__device__ __forceinline__ void grad_expert_order(const int* s_off, int E, int* s_eorder,
-                                                  int* s_bcur, int lane) {
-  auto bucket = [&](int e) {  // 0 = empty, 1 + floor(log2(rows)) otherwise
-    const int n = s_off[e + 1] - s_off[e];
-    return n > 0 ? 32 - __clz(n) : 0;
-  };
-  for (int b = lane; b < 33; b += 32) s_bcur[b] = 0;
-  __syncwarp();
-  for (int e = lane; e < E; e += 32) atomicAdd(&s_bcur[bucket(e)], 1);
-  __syncwarp();
-  if (lane == 0) {  // exclusive prefix, largest bucket first
-    int acc = 0;
-    for (int b = 32; b >= 0; --b) {
-      const int c = s_bcur[b];
-      s_bcur[b] = acc;
-      acc += c;
-    }
-  }
-  __syncwarp();
-  for (int c0 = 0; c0 < E; c0 += 32) {
-    const int e = c0 + lane;
-    const int key = e < E ? bucket(e) : 33;
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (e < E) s_eorder[s_bcur[key] + rank] = e;
-    __syncwarp();
-    if (e < E && rank == 0) s_bcur[key] += __popc(peers);
-    __syncwarp();
-  }
 }
 
 template <int RK>
@@ -171,7 +137,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int e = lane; e <= args.E; e += 32) s_off[e] = 0;  // all experts empty
     }
     __syncwarp();
-    grad_expert_order(s_off, args.E, s_eorder, s_bcur, lane);
+    expert_load_order(s_off, args.E, s_eorder, s_bcur, lane);
   }
   tc_fence_before();
   __syncthreads();

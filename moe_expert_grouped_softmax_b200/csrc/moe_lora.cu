@@ -415,10 +415,11 @@ moe_status_t launch_base_grad_t(const CUtensorMap* u, const CUtensorMap* v,
     BaseGradProblem& p = args.prob[i];
     p.p_tiles = (p.P + 127) / 128;
     p.q_tiles = (p.Q + BN - 1) / BN;
-    p.tile_begin = begin;
-    begin += args.E * p.p_tiles * p.q_tiles;
+    p.tile_begin = begin;  // inside one expert's tiles
+    begin += p.p_tiles * p.q_tiles;
   }
-  args.total_tiles = begin;
+  args.tiles_per_expert = begin;
+  args.total_tiles = args.E * begin;
   auto kern = base_grad_kernel<BN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM_BYTES) != cudaSuccess)
