@@ -142,8 +142,9 @@ struct GemmCfg {
 #endif
 // L2 residency hints for the mainloop loads (MOE_L2_HINTS): 0 none, 1 keep
 // weights / stream activations (default), 2 keep activations / stream
-// weights.  Measured on the gpt-oss-20b-shaped layer: order 0 with hints 1
-// is fastest; without hints the step is 5-10% slower.
+// weights.  Measured with the single-CTA kernels on the gpt-oss-20b-shaped
+// layer: order 0 with hints 1 is fastest; without hints the step is 5-10%
+// slower.
 #ifndef MOE_L2_HINTS
 #define MOE_L2_HINTS 1
 #endif

@@ -1,11 +1,11 @@
-// a3, a4, a7, a8 on CTA pairs: the grouped GEMMs with 256 x 256 tiles on the
+// a3, a4, a7, a8 on CTA pairs: the grouped GEMMs with 256-row tiles on the
 // 2-SM tensor-core instruction (tcgen05.mma.cta_group::2).
 //
-// A cluster of two CTAs on two SMs computes one 256-row x 256-column tile of
-// one expert.  Each CTA stages its own 128 rows of A and half (128 columns)
-// of the weight operand, so every SM moves a third less operand data per
-// FLOP than the single-CTA 128-row tile, through shared memory as well as
-// from L2.  The even CTA ("leader") issues the MMAs, which read both CTAs'
+// A cluster of two CTAs on two SMs computes one 256-row x Nt-column tile of
+// one expert (Nt <= 256, below).  Each CTA stages its own 128 rows of A and
+// half (Nt/2 columns) of the weight operand, so every SM moves a third less
+// operand data per FLOP than the single-CTA 128-row tile, through shared
+// memory as well as from L2.  The even CTA ("leader") issues the MMAs, which read both CTAs'
 // shared memory and write both CTAs' TMEM.
 //
 // Split LoRA: the rank-r down-products (s Xp A1^T, s h A2^T, s dZ2 B2,
@@ -115,8 +115,11 @@ struct PairCfg {
   // quarter for every mode, each draining half the columns, +0.8% per step)
   static constexpr int EPI_WARPS = gemm_epi_warps(MODE);
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  // weight rows per TMA box: gate_up fwd loads gate and up blocks of 64
-  static constexpr int W_BOX_ROWS = kSwiGLU ? 64 : NH;
+  // rows per TMA box of the K-major weight in gate_up fwd (gate and up
+  // blocks of 64; down fwd boxes hold the launch's Nt/2 rows) and of the up
+  // factor (gate_up fwd: two blocks of 64; otherwise 128, of which the MMA
+  // reads the first Nt/2)
+  static constexpr int W_BOX_ROWS = 64;
   static constexpr int LB_BOX_ROWS = kSwiGLU ? 64 : NH;
   static constexpr int MN_BOX = 64 * BK * 2;        // one 64-column MN-major atom
   static_assert(NS >= 3, "not enough shared memory for three stages");
@@ -150,8 +153,8 @@ __device__ __forceinline__ void epi_swiglu_seg64(const GemmArgs& args, uint32_t 
 }
 
 // Operand maps: tmA = A [R, K] (128-row boxes); tmW = the weight (K-major
-// [E * b_rows, K] in W_BOX_ROWS-row boxes, or MN-major [E * b_rows, N] in
-// 64 x 64 atoms); tmXA = the rank-r product [R, r] (128-row boxes);
+// [E * b_rows, K] in boxes of W_BOX_ROWS rows (gate_up fwd) or Nt/2 rows
+// (down fwd), or MN-major [E * b_rows, N] in 64 x 64 atoms); tmXA = the rank-r product [R, r] (128-row boxes);
 // tmLB = the up factor [E * lb_rows, r] (LB_BOX_ROWS-row boxes).
 template <int MODE, int RK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::THREADS, 1)
@@ -291,8 +294,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_bytes);
           tma_load_2d_pair_hint(st, &tmA, fb, kx, row0, pol_a);
           if constexpr (kBMN) {
-            // W [K, N] in place: this CTA's 128 tile columns as two 64-column
-            // atoms
+            // W [K, N] in place: this CTA's Nt/2 tile columns, loaded as two
+            // 64-column atoms
             const int krow = e * args.b_rows + kx;
             tma_load_2d_pair_hint(sb, &tmW, fb, n0, krow, pol_w);
             tma_load_2d_pair_hint(sb + C::MN_BOX, &tmW, fb, n0 + 64, krow, pol_w);
