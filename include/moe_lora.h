@@ -92,9 +92,11 @@ MOE_API moe_status_t moe_route_topk(const float* logits, int T, int E, int k,
  *    moe_route_noalloc_max_workspace_bytes() (4 MiB; e.g. T <= 65536 tokens
  *    with k <= 8 and E <= 512); larger sizes return MOE_ERR_UNSUPPORTED
  *    before anything is launched.
- *  - The first call on each device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *  - Every call looks up the array's device address with the caller's device
+ *    current (cudaGetSymbolAddress, a host-side query that allocates
+ *    nothing), so the address stays right after cudaDeviceReset and in any
+ *    context.  The first call in a process may load the library's device
+ *    code: make one call before any stream capture begins.
  *  - All calls share the one array and it keeps the last call's contents.
  *    Nothing in it needs to start at zero (each call writes every scratch
  *    byte it reads before reading it), but calls whose work overlaps on the

@@ -28,32 +28,24 @@ using namespace moe;
 // memory, so that entry point never needs a caller-provided workspace and never
 // allocates.  Every GPU that loads the library holds these bytes until the
 // process exits.  In host code `g_route_scratch` is only a host-side stand-in
-// for the symbol, never a device address: its device address is obtained with
-// cudaGetSymbolAddress on each device (see route_scratch_on_current_device).
+// for the symbol, never a device address: its device address is looked up
+// with cudaGetSymbolAddress, with the caller's device current, on every call
+// (see route_scratch_on_current_device).
 constexpr size_t kRouteScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_route_scratch_mu;
-void* g_route_scratch_dev[kMaxDevices] = {};
-
-// Device address of g_route_scratch on the current device, looked up once per
-// device (the first call on a device does the lookup, with that device
-// current) and cached.
+// Device address of g_route_scratch in the current device's context.  Looked
+// up on every call rather than cached: the lookup is a host-side query that
+// allocates nothing, and a cached address would go stale after
+// cudaDeviceReset (the module is loaded again, possibly elsewhere) or belong
+// to another context of the same device.
 moe_status_t route_scratch_on_current_device(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_route_scratch_mu);
-  if (g_route_scratch_dev[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
-      return MOE_ERR_CUDA;
-    g_route_scratch_dev[dev] = p;
-  }
-  *out = g_route_scratch_dev[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
+    return MOE_ERR_CUDA;
+  *out = p;
   return MOE_OK;
 }
 

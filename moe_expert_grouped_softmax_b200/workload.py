@@ -62,16 +62,30 @@ def block_flops(T, H, I, E, k, r, full_ft=False, train_router=False):
                 base_gemm=2 * R * (H * 2 * I + I * H) * 2)
 
 
-def gemm_flops(R, H, I, r):
-    """FLOPs of each tensor-core kernel of the block, by kernel."""
-    return dict(
-        gate_up_fwd=split_lora_proj_flops(R, H, 2 * I, r),
-        down_fwd=split_lora_proj_flops(R, I, H, r),
-        down_bwd=2 * R * (H * I + H * r + r * I),     # dh, with LoRA path
-        gate_up_bwd=2 * R * (2 * I * H + 2 * I * r + r * H),
-        lora_grads=2 * R * r * (H + 2 * I + I + H),
-        base_grad=base_grad_flops(R, H, I),
-    )
+def gemm_flops(R, H, I, r, pairs=(False, False, False, False)):
+    """FLOPs of each tensor-core kernel of the block, by kernel.
+
+    ``pairs`` says, for gate_up fwd, down fwd, down bwd and gate_up bwd,
+    whether that GEMM ran on CTA pairs: there the rank-r down-projection of
+    the GEMM (s Xp A1^T, s h A2^T, s dZ2 B2, s dZ1 B1) is computed by the
+    separate rank pass, so its FLOPs are counted under ``rank_down`` (the
+    sum over the passes that ran) and not under the GEMM."""
+    down_proj = (2 * R * H * r, 2 * R * I * r, 2 * R * H * r, 2 * R * 2 * I * r)
+    full = (split_lora_proj_flops(R, H, 2 * I, r),
+            split_lora_proj_flops(R, I, H, r),
+            2 * R * (H * I + H * r + r * I),          # dh, with LoRA path
+            2 * R * (2 * I * H + 2 * I * r + r * H))
+    names = ("gate_up_fwd", "down_fwd", "down_bwd", "gate_up_bwd")
+    out = {}
+    rank = 0
+    for n, f, d, p in zip(names, full, down_proj, pairs):
+        out[n] = f - d if p else f
+        rank += d if p else 0
+    if rank:
+        out["rank_down"] = rank
+    out["lora_grads"] = 2 * R * r * (H + 2 * I + I + H)
+    out["base_grad"] = base_grad_flops(R, H, I)
+    return out
 
 
 def hbm_bytes(T, H, E, k):

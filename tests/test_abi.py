@@ -73,29 +73,90 @@ def test_cta_pair_choice(L):
     assert L.moe_uses_cta_pairs(32768, 32, 2880) == 1
 
 
+class _Buffers:
+    """Buffers for the host-side error checks, each sized for the dimensions
+    of the call it is passed to.  With a GPU they are real device
+    allocations, so that if a host check were lost the call would launch on
+    valid memory and the test would fail on its return code, instead of a
+    kernel touching a made-up address on a shared GPU.  Without a GPU the
+    library cannot launch anything, and host memory of the same size stands
+    in."""
+
+    def __init__(self):
+        import torch
+        self.torch = torch
+        self.cuda = torch.cuda.is_available()
+        self.keep = []
+
+    def __call__(self, nbytes):
+        n = max(1, int(nbytes))
+        if self.cuda:
+            t = self.torch.zeros(n, dtype=self.torch.uint8, device="cuda")
+            self.keep.append(t)
+            return ctypes.c_void_p(t.data_ptr())
+        b = ctypes.create_string_buffer(n)
+        self.keep.append(b)
+        return ctypes.c_void_p(ctypes.addressof(b))
+
+
 def test_host_side_argument_errors(L):
-    P = ctypes.c_void_p
-    fake = P(256)  # never dereferenced: the call must fail before any launch
-    # k > E, E > 512, T*k overflow
-    assert L.moe_route_topk(fake, 4, 3, 4, fake, fake, fake, fake, fake, fake, 1 << 20, None) == 2
-    assert L.moe_route_topk(fake, 4, 513, 1, fake, fake, fake, fake, fake, fake, 1 << 20, None) == 2
-    assert L.moe_route_topk(fake, 1 << 30, 8, 4, fake, fake, fake, fake, fake, fake, 1 << 20, None) == 2
-    # null outputs / short workspace
-    assert L.moe_route_topk(fake, 4, 8, 2, None, fake, fake, fake, fake, fake, 1 << 20, None) == 1
-    assert L.moe_route_topk(fake, 4, 8, 2, fake, fake, fake, fake, fake, fake, 1, None) == 1
-    # permute: H not a multiple of 8, null, dw without Zp
-    assert L.moe_permute(fake, fake, None, 4, 12, 2, fake, None, None, None) == 2
-    assert L.moe_permute(None, fake, None, 4, 16, 2, fake, None, None, None) == 1
-    assert L.moe_permute(fake, fake, None, 4, 16, 2, fake, None, fake, None) == 1
-    assert L.moe_unpermute(fake, fake, None, 4, 16, 2, None, None) == 1
-    # GEMMs: unsupported rank / shape, missing buffers, short saved buffer
-    W = [fake] * 6
-    assert L.moe_lora_mlp_fwd(fake, fake, 8, 256, 512, 8, 2.0, *W, 64, fake, fake, 1 << 30, None, 0, None) == 2
-    assert L.moe_lora_mlp_fwd(fake, fake, 8, 200, 512, 16, 2.0, *W, 64, fake, fake, 1 << 30, None, 0, None) == 2
-    assert L.moe_lora_mlp_fwd(fake, fake, 8, 256, 512, 16, 2.0, *W, 64, None, fake, 1 << 30, None, 0, None) == 1
-    assert L.moe_lora_mlp_fwd(fake, fake, 8, 256, 512, 16, 2.0, *W, 64, fake, fake, 16, None, 0, None) == 1
-    assert L.moe_lora_mlp_bwd(fake, fake, fake, 8, 256, 512, 16, 2.0, *W, fake, 1 << 30, 64,
-                              fake, fake, fake, fake, fake, fake, 16, None) == 1
+    B = _Buffers()
+
+    def route_bufs(T, E, k, ws_bytes):
+        return (B(T * E * 4), B(T * k * 4), B(T * k * 4), B(E * 4), B((E + 1) * 4),
+                B(T * k * 4), B(ws_bytes))
+
+    ws = 1 << 20
+    # k > E, E > 512: rejected before any launch
+    lg, ix, w, c, o, d, wb = route_bufs(4, 3, 4, ws)
+    assert L.moe_route_topk(lg, 4, 3, 4, ix, w, c, o, d, wb, ws, None) == 2
+    lg, ix, w, c, o, d, wb = route_bufs(4, 513, 1, ws)
+    assert L.moe_route_topk(lg, 4, 513, 1, ix, w, c, o, d, wb, ws, None) == 2
+    # T*k overflow: no buffer can be that large, so every pointer is null
+    # (a lost overflow check would then stop at the null check, with 1)
+    assert L.moe_route_topk(None, 1 << 30, 8, 4, None, None, None, None, None, None,
+                            ws, None) == 2
+    # null output; workspace declared too short (the buffer itself is full size)
+    T, E, k = 4, 8, 2
+    need = L.moe_route_workspace_bytes(T, E, k)
+    lg, ix, w, c, o, d, wb = route_bufs(T, E, k, need)
+    assert L.moe_route_topk(lg, T, E, k, None, w, c, o, d, wb, need, None) == 1
+    assert L.moe_route_topk(lg, T, E, k, ix, w, c, o, d, wb, 1, None) == 1
+    # permute: H not a multiple of 8, null input, dw without Zp
+    T, k = 4, 2
+    assert L.moe_permute(B(T * 12 * 2), B(T * k * 4), None, T, 12, k, B(T * k * 12 * 2),
+                         None, None, None) == 2
+    assert L.moe_permute(None, B(T * k * 4), None, T, 16, k, B(T * k * 16 * 2),
+                         None, None, None) == 1
+    assert L.moe_permute(B(T * 16 * 2), B(T * k * 4), None, T, 16, k, B(T * k * 16 * 2),
+                         None, B(T * k * 4), None) == 1
+    assert L.moe_unpermute(B(T * k * 16 * 2), B(T * k * 4), None, T, 16, k, None,
+                           None) == 1
+
+    # GEMMs: unsupported rank / shape, missing output, short saved buffer and
+    # workspace (every buffer sized for the shape it is passed with)
+    def gemm_bufs(E, H, I, r, R):
+        W = [B(E * 2 * I * H * 2), B(E * r * H * 2), B(E * 2 * I * r * 2),
+             B(E * H * I * 2), B(E * r * I * 2), B(E * H * r * 2)]
+        return B(R * H * 2), B((E + 1) * 4), W
+
+    E, H, I, R = 8, 256, 512, 64
+    xp, off, W = gemm_bufs(E, H, I, 8, R)
+    assert L.moe_lora_mlp_fwd(xp, off, E, H, I, 8, 2.0, *W, R, B(R * H * 2), B(1 << 20),
+                              1 << 20, None, 0, None) == 2
+    xp, off, W = gemm_bufs(E, 200, I, 16, R)
+    assert L.moe_lora_mlp_fwd(xp, off, E, 200, I, 16, 2.0, *W, R, B(R * 200 * 2),
+                              B(1 << 20), 1 << 20, None, 0, None) == 2
+    xp, off, W = gemm_bufs(E, H, I, 16, R)
+    sb = L.moe_saved_bytes(R, H, I, 16)
+    assert L.moe_lora_mlp_fwd(xp, off, E, H, I, 16, 2.0, *W, R, None, B(sb), sb,
+                              None, 0, None) == 1
+    assert L.moe_lora_mlp_fwd(xp, off, E, H, I, 16, 2.0, *W, R, B(R * H * 2), B(sb), 16,
+                              None, 0, None) == 1
+    wsb = L.moe_workspace_bytes(R, E, H, I, 16)
+    assert L.moe_lora_mlp_bwd(B(R * H * 2), xp, off, E, H, I, 16, 2.0, *W, B(sb), sb, R,
+                              B(R * H * 2), B(E * 16 * H * 2), B(E * 2 * I * 16 * 2),
+                              B(E * 16 * I * 2), B(E * H * 16 * 2), B(wsb), 16, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

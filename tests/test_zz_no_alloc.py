@@ -72,5 +72,14 @@ def test_noalloc_route_rejects_sizes_over_its_scratch(cuda_ok):
     cap = L.moe_route_noalloc_max_workspace_bytes()
     T, E, k = 1 << 20, 64, 8  # needs far more than the fixed scratch
     assert ops.route_workspace_bytes(T, E, k) > cap
-    fake = ctypes.c_void_p(256)  # never dereferenced: rejected before any launch
-    assert f(fake, T, E, k, fake, fake, fake, fake, fake, None) == 2
+    # Real buffers of the full size for these T, E, k (about 0.4 GB), so that
+    # even if the size check were lost no kernel could reach past a caller's
+    # buffer (the scratch itself is guarded a second time by the workspace
+    # check of the routing call this entry point forwards to, which would
+    # then return 1): the call must be rejected with 2 before any launch.
+    logits = torch.zeros((T, E), dtype=torch.float32, device="cuda")
+    got = _outs(T, E, k)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert f(_p(logits), T, E, k, *[_p(t) for t in got], stream) == 2
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
