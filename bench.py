@@ -213,30 +213,53 @@ def run_ours(args, cfg):
     st = ops.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
+    # kernels the library launches per step (host-side count of one eager step)
+    l0 = ops.kernel_launches()
+    blk.step(X, logits, dY, W, Wr)
+    per_step = ops.kernel_launches() - l0
+    use_graph = args.launch == "graph"
+    if use_graph:
+        # one CUDA graph of the whole step, replayed: the same kernels with the
+        # same arguments, launched together
+        blk.capture(X, logits, dY, W, Wr)
+        torch.cuda.synchronize()
 
     K = args.steps
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     clk = Clocks(local)
     clk.start()
-    ops.profile_enable(True)
     barrier()
     torch.cuda.synchronize()
     clk.t_begin = time.time()
-    launches0 = ops.kernel_launches()
     for i in range(K):
         flush.zero_()                      # L2 flush, outside the timed span
         ev0[i].record(stream)
-        blk.step(X, logits, dY, W, Wr)
+        if use_graph:
+            blk.replay()
+        else:
+            blk.step(X, logits, dY, W, Wr)
         ev1[i].record(stream)
-    launches = ops.kernel_launches() - launches0
+    launches = per_step * K
     torch.cuda.synchronize()
     clk.t_end = time.time()
     barrier()
     clk.stop()
     timed_s = clk.t_end - clk.t_begin
+    st = ops.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timed steps")
     ms_steps = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     ms_total = float(sum(ms_steps))
+    # per-kernel durations: the same steps again, launched eagerly with a CUDA
+    # event pair around every launch on the launching stream (kept out of the
+    # headline timing above, which they would slow down)
+    ops.profile_enable(True)
+    barrier()
+    for i in range(K):
+        flush.zero_()
+        blk.step(X, logits, dY, W, Wr)
+    torch.cuda.synchronize()
     kern = {}
     for kind in ops.PROF_KINDS:   # collect before the hook is switched off
         d = ops.profile_collect(kind)
@@ -285,7 +308,10 @@ def run_ours(args, cfg):
                 comp.wait_event(ev["in_ready"][b])
                 if i >= 2:
                     comp.wait_event(ev["out_free"][b])
-                blocks[b].step(din[b][0], din[b][1], din[b][2], W, Wr)
+                if use_graph:
+                    blocks[b].replay()
+                else:
+                    blocks[b].step(din[b][0], din[b][1], din[b][2], W, Wr)
                 ev["in_free"][b].record(comp)
                 ev["done"][b].record(comp)
                 with torch.cuda.stream(s_out):
@@ -294,6 +320,11 @@ def run_ours(args, cfg):
                         h.copy_(o, non_blocking=True)
                     ev["out_free"][b].record(s_out)
 
+        if use_graph:
+            # each block's step captured on its own input buffers
+            for b in range(2):
+                blocks[b].capture(din[b][0], din[b][1], din[b][2], W, Wr)
+            torch.cuda.synchronize()
         run_e2e(max(2, args.warmup))
         torch.cuda.synchronize()
         barrier()
@@ -361,6 +392,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="gpt-oss-20b", choices=list(S.CONFIGS))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
+                    help="timed steps as replays of one captured CUDA graph of the step "
+                         "(default) or as eager launches")
     ap.add_argument("--extra-configs", default="qwen3-30b-a3b,gpt-oss-20b-long",
                     help="comma-separated configs also measured in the same run "
                          "(device-timed steps only); empty for none")
@@ -394,7 +428,9 @@ def main():
     config = {"workload": workload, "T": T, "H": H, "I": I, "E": E, "top_k": k,
               "lora_r": r, "lora_s": cfg["s"], "logits": cfg["logits"],
               "parallelism": "replicas", "l2": "256 MiB memset before each step, "
-              "outside the timed span"}
+              "outside the timed span",
+              "launch": ("one CUDA graph of the whole step, replayed" if args.launch == "graph"
+                         else "eager launches")}
     ws, rank, _ = dist_env()
 
     if args.impl == "reference":

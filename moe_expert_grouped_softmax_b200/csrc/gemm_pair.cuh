@@ -88,6 +88,31 @@ __device__ __forceinline__ bool pair_half_tile(const int* s_off, int e, int mt) 
 #define MOE_PAIR_TILE_ORDER 1
 #endif
 
+// Epilogue stores of the pair kernels: each epilogue warp stages its 32 rows
+// of an output column block (SBW bf16 columns) in a swizzled shared-memory
+// box and writes it with one TMA store, through a ring of NSTG boxes per
+// warp; boxes that would cross a tile's column range or hold rows of another
+// expert fall back to per-thread row stores.  (The per-thread stores of 32
+// different rows per instruction load the same LSU path as the pipeline's
+// barrier polls.)
+// MOE_PAIR_TMA_STORE: bit m set = mode m stores through the ring.  Measured
+// (same-box A/B): gate_up fwd and gate_up bwd about 1% faster with it; down
+// fwd no faster on the gpt-oss-20b shape and 9% slower on the Qwen3-30B-A3B
+// one (K = 768: short mainloops leave the staging no slack); down bwd 2%
+// slower.
+#ifndef MOE_PAIR_TMA_STORE
+#define MOE_PAIR_TMA_STORE 0x9
+#endif
+#ifndef MOE_PAIR_STORE_BOX
+#define MOE_PAIR_STORE_BOX 16
+#endif
+#ifndef MOE_PAIR_NSTG
+#define MOE_PAIR_NSTG 3
+#endif
+#ifndef MOE_PAIR_NSTG8
+#define MOE_PAIR_NSTG8 1
+#endif
+
 template <int MODE, int RK>
 struct PairCfg {
   static constexpr bool kSwiGLU = (MODE == kGateUpFwd);
@@ -99,11 +124,25 @@ struct PairCfg {
   static constexpr int B_BYTES = NH * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int LSPAN = RK * 2;              // bytes per K-major rank-r row
-  static constexpr int LB_BYTES = NH * LSPAN;       // this CTA's up-factor rows
+  // this CTA's up-factor block: NH rows of r (K-major, forward) or r rows of
+  // NH columns as two 64-column MN-major atoms (backward; the same bytes)
+  static constexpr int LB_BYTES = NH * LSPAN;
+  static constexpr int LB_ATOM = RK * 128;          // backward: one 64-column atom
   static constexpr int XA_BYTES = BM * LSPAN;       // this CTA's rank-r rows
   static constexpr int UP_BYTES = LB_BYTES + XA_BYTES;
   static constexpr int MISC_BYTES = 512 + 8 * 520;  // barriers, counts, tables
-  static constexpr int FIXED = 2 * UP_BYTES + MISC_BYTES;
+  // epilogue warps as in the single-CTA kernel (measured: two per lane
+  // quarter for every mode, each draining half the columns, +0.8% per step)
+  static constexpr int EPI_WARPS = gemm_epi_warps(MODE);
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  // epilogue store staging: per warp NSTG boxes of 32 rows x SBW columns
+  static constexpr bool kRing = ((MOE_PAIR_TMA_STORE >> MODE) & 1) != 0;
+  static constexpr int SBW = MOE_PAIR_STORE_BOX;
+  static constexpr int SLOT_BYTES = 32 * SBW * 2;
+  static constexpr int NSTG = EPI_WARPS == 8 ? MOE_PAIR_NSTG8 : MOE_PAIR_NSTG;
+  static constexpr int RING_BYTES = kRing ? EPI_WARPS * NSTG * SLOT_BYTES : 0;
+  static constexpr uint32_t SLOT_SWZ_SPAN = SBW * 2;  // bytes per staged row
+  static constexpr int FIXED = 2 * UP_BYTES + MISC_BYTES + RING_BYTES;
   static constexpr int NS_FIT = (kSmemOptin - 1024 - FIXED) / STAGE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + FIXED;
@@ -111,10 +150,6 @@ struct PairCfg {
       RK == 16 ? kLayoutSW32 : (RK == 32 ? kLayoutSW64 : kLayoutSW128);
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_STRIDE = 256;
-  // epilogue warps as in the single-CTA kernel (measured: two per lane
-  // quarter for every mode, each draining half the columns, +0.8% per step)
-  static constexpr int EPI_WARPS = gemm_epi_warps(MODE);
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   // rows per TMA box of the K-major weight in gate_up fwd (gate and up
   // blocks of 64; down fwd boxes hold the launch's Nt/2 rows) and of the up
   // factor (gate_up fwd: two blocks of 64; otherwise 128, of which the MMA
@@ -125,43 +160,198 @@ struct PairCfg {
   static_assert(NS >= 3, "not enough shared memory for three stages");
   static_assert(SMEM_BYTES <= kSmemOptin, "shared memory over the opt-in limit");
   static_assert(LB_BYTES % 1024 == 0 && XA_BYTES % 1024 == 0, "swizzle atoms");
+  static_assert(SBW == 16 || SBW == 32, "staged box width");
+  static_assert(NSTG >= 1 && SLOT_BYTES % 1024 == 0, "staging ring");
 };
 
+// One epilogue warp's ring of staged output boxes (32 rows x SBW bf16
+// columns each, swizzled with the box's row span).
+template <int SBW, int NSTG>
+struct StoreRing {
+  uint8_t* base;
+  int slot;
+
+  // Stores this thread's SBW values (its row of the box) at columns
+  // [x, x + SBW) of rows [y, y + 32) of the tensor behind `tm`.  Warp-wide.
+  __device__ __forceinline__ void put(const CUtensorMap* tm, const float* v, int x, int y,
+                                      uint64_t pol, int lane) {
+    constexpr uint32_t SPAN = SBW * 2;
+    uint8_t* box = base + slot * (32 * SPAN);
+    if (lane == 0) bulk_wait_group_read<NSTG - 1>();  // this slot's last store has read it
+    __syncwarp();
+#pragma unroll
+    for (int ch = 0; ch < SBW / 8; ++ch)
+      *reinterpret_cast<uint4*>(box + swz_offset(lane, ch, SPAN)) = pack8(v + 8 * ch);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tm, box, x, y, pol);
+      bulk_commit_group();
+    }
+    slot = slot + 1 == NSTG ? 0 : slot + 1;
+  }
+
+  // Every store issued by this warp has written global memory.
+  __device__ __forceinline__ void finish(int lane) {
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  }
+};
+
+// Writes this thread's W values v (output columns [col, col + W) of its
+// row) of one output: through the staging ring in SBW-column boxes when all
+// 32 rows of the warp belong to the tile's expert (rows_all) and the box
+// stays inside the tile's columns [.., hi); otherwise with per-thread row
+// stores.  Columns at or past nmax (the output's width) are never written;
+// a box that reaches past nmax is clipped by the tensor map.
+template <int W, bool kRing, int SBW, int NSTG>
+__device__ __forceinline__ void pair_out_chunk(StoreRing<SBW, NSTG>& ring, const CUtensorMap* tm,
+                                               __nv_bfloat16* rowp, const float* v, int col,
+                                               int y0, bool rows_all, bool rvalid, int hi,
+                                               int nmax, uint64_t pol, int lane) {
+  const int lim = min(hi, nmax);
+  if constexpr (W < SBW || !kRing) {
+    if (rvalid) store_row_bf16<W>(rowp + col, v, lim - col, pol);
+  } else if (rows_all) {
+#pragma unroll
+    for (int b = 0; b < W; b += SBW) {
+      const int x = col + b;
+      if (x >= lim) break;
+      if (x + SBW <= hi) ring.put(tm, v + b, x, y0, pol, lane);
+      else store_row_bf16<SBW>(rowp + x, v + b, lim - x, pol);
+    }
+  } else if (rvalid) {
+    store_row_bf16<W>(rowp + col, v, lim - col, pol);
+  }
+}
+
 // SwiGLU epilogue of one 64-column gate / up block of a row: gate at TMEM
-// column t_gate, up at t_gate + 64; output columns col .. col + 63.
-__device__ __forceinline__ void epi_swiglu_seg64(const GemmArgs& args, uint32_t t_gate,
-                                                 int grow, bool rvalid, int col,
-                                                 uint64_t pol) {
+// column t_gate, up at t_gate + 64; output columns col .. col + 63 of h
+// (tmH), of the saved gate (tmG: Z1 columns [0, I)) and of the saved up
+// (tmU: Z1 columns [I, 2I)).
+template <bool kRing, int SBW, int NSTG>
+__device__ __forceinline__ void epi_swiglu_seg64(const GemmArgs& args, StoreRing<SBW, NSTG>& ring,
+                                                 const CUtensorMap* tmH, const CUtensorMap* tmG,
+                                                 const CUtensorMap* tmU, uint32_t t_gate,
+                                                 int grow, int y0, bool rows_all, bool rvalid,
+                                                 int col, uint64_t pol, int lane) {
   __nv_bfloat16* hrow = args.out + static_cast<size_t>(grow) * args.ld_out;
   __nv_bfloat16* zrow = args.out2 + static_cast<size_t>(grow) * args.ld_out2;
-  for_chunks<64>([&](int c, auto w) {
-    constexpr int W = decltype(w)::value;
-    float g[W], u[W];
-    tmem_ld<W>(t_gate + c, g);
-    tmem_ld<W>(t_gate + 64 + c, u);
+#pragma unroll 1
+  for (int c = 0; c < 64; c += 32) {
+    float g[32], u[32], h[32];
+    tmem_ld<32>(t_gate + c, g);
+    tmem_ld<32>(t_gate + 64 + c, u);
     tmem_ld_wait();
-    if (rvalid) {
-      float h[W];
 #pragma unroll
-      for (int i = 0; i < W; ++i) h[i] = g[i] * sigmoidf_(g[i]) * u[i];
-      const int cc = col + c, nv = args.N - cc;
-      store_row_bf16<W>(hrow + cc, h, nv, pol);
-      store_row_bf16<W>(zrow + cc, g, nv, pol);
-      store_row_bf16<W>(zrow + args.I + cc, u, nv, pol);
-    }
-  });
+    for (int i = 0; i < 32; ++i) h[i] = g[i] * sigmoidf_(g[i]) * u[i];
+    const int cc = col + c, hi = col + 64;
+    pair_out_chunk<32, kRing>(ring, tmH, hrow, h, cc, y0, rows_all, rvalid, hi, args.N, pol,
+                              lane);
+    pair_out_chunk<32, kRing>(ring, tmG, zrow, g, cc, y0, rows_all, rvalid, hi, args.N, pol,
+                              lane);
+    pair_out_chunk<32, kRing>(ring, tmU, zrow + args.I, u, cc, y0, rows_all, rvalid, hi,
+                              args.N, pol, lane);
+  }
+}
+
+// Epilogue of the other modes for NC accumulator columns (this warp's share
+// of them with kSplit): tile column j of the drained range sits at TMEM
+// column t_acc + j and is output column col0 + j; nothing at or past hi
+// (the end of the tile's columns) or args.N is written.  Plain store (down
+// fwd: Z2, gate_up bwd: dXp, through tmO) or SwiGLU backward (down bwd:
+// reads the saved gate / up, writes dZ1 = [dg | du] through tmO / tmU).
+template <int MODE, int NC, bool kSplit, bool kRing, int SBW, int NSTG>
+__device__ __forceinline__ void epi_pair_drain(const GemmArgs& args, StoreRing<SBW, NSTG>& ring,
+                                               const CUtensorMap* tmO, const CUtensorMap* tmU,
+                                               uint32_t t_acc, int grow, int y0, bool rows_all,
+                                               bool rvalid, int ehalf, int col0, int hi,
+                                               uint64_t pol, int lane) {
+  const int nmax = min(args.N, hi);
+  __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
+  if constexpr (MODE == kDownBwd) {
+    const __nv_bfloat16* grow_p = args.aux + static_cast<size_t>(grow) * args.ld_aux;
+    for_my_chunks<NC, kSplit>(ehalf, [&](int c, auto w) {
+      constexpr int W = decltype(w)::value;
+      uint4 gv[W / 8], uv[W / 8];
+      // loads first (in flight during the TMEM read), 32 bytes at a time
+      // where the address allows
+      const bool a32 = ((reinterpret_cast<uintptr_t>(grow_p + col0 + c) |
+                         reinterpret_cast<uintptr_t>(grow_p + args.I + col0 + c)) & 31u) == 0;
+#pragma unroll
+      for (int q = 0; q < W / 8; q += 2) {
+        const int col = col0 + c + 8 * q;
+        gv[q] = uv[q] = make_uint4(0, 0, 0, 0);
+        if (q + 1 < W / 8) gv[q + 1] = uv[q + 1] = make_uint4(0, 0, 0, 0);
+        if (!rvalid) continue;
+        if (q + 1 < W / 8 && a32 && col + 16 <= nmax) {
+          ld_global_nc_v8(grow_p + col, gv[q], gv[q + 1]);
+          ld_global_nc_v8(grow_p + args.I + col, uv[q], uv[q + 1]);
+        } else {
+          if (col < nmax) {
+            gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
+            uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
+          }
+          if (q + 1 < W / 8 && col + 8 < nmax) {
+            gv[q + 1] = *reinterpret_cast<const uint4*>(grow_p + col + 8);
+            uv[q + 1] = *reinterpret_cast<const uint4*>(grow_p + args.I + col + 8);
+          }
+        }
+      }
+      float dh[W];
+      tmem_ld<W>(t_acc + c, dh);
+      tmem_ld_wait();
+      float dg[W], du[W];
+#pragma unroll
+      for (int q = 0; q < W / 8; ++q) {
+        const uint32_t ga[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+        const uint32_t ua[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const float gg = h2 ? bf16_hi(ga[i]) : bf16_lo(ga[i]);
+            const float uu = h2 ? bf16_hi(ua[i]) : bf16_lo(ua[i]);
+            const int j = 8 * q + 2 * i + h2;
+            const float sg = sigmoidf_(gg);
+            dg[j] = dh[j] * uu * sg * (1.f + gg * (1.f - sg));
+            du[j] = dh[j] * gg * sg;
+          }
+        }
+      }
+      const int col = col0 + c;
+      pair_out_chunk<W, kRing>(ring, tmO, orow, dg, col, y0, rows_all, rvalid, hi, args.N, pol,
+                               lane);
+      pair_out_chunk<W, kRing>(ring, tmU, orow + args.I, du, col, y0, rows_all, rvalid, hi,
+                               args.N, pol, lane);
+    });
+  } else {
+    for_my_chunks<NC, kSplit>(ehalf, [&](int c, auto w) {
+      constexpr int W = decltype(w)::value;
+      float v[W];
+      tmem_ld<W>(t_acc + c, v);
+      tmem_ld_wait();
+      pair_out_chunk<W, kRing>(ring, tmO, orow, v, col0 + c, y0, rows_all, rvalid, hi, args.N,
+                               pol, lane);
+    });
+  }
 }
 
 // Operand maps: tmA = A [R, K] (128-row boxes); tmW = the weight (K-major
 // [E * b_rows, K] in boxes of W_BOX_ROWS rows (gate_up fwd) or Nt/2 rows
 // (down fwd), or MN-major [E * b_rows, N] in 64 x 64 atoms); tmXA = the rank-r product [R, r] (128-row boxes);
-// tmLB = the up factor [E * lb_rows, r] (LB_BOX_ROWS-row boxes).
+// tmLB = the up factor: forward B [E * lb_rows, r] (LB_BOX_ROWS-row boxes);
+// backward A read in place as [E * r, N] (64-column x r-row boxes: the MMA's
+// B operand MN-major, so the factor needs no transposed copy).
 template <int MODE, int RK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::THREADS, 1)
     grouped_lora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                   const __grid_constant__ CUtensorMap tmW,
                                   const __grid_constant__ CUtensorMap tmXA,
                                   const __grid_constant__ CUtensorMap tmLB,
+                                  const __grid_constant__ CUtensorMap tmO,
+                                  const __grid_constant__ CUtensorMap tmO2,
+                                  const __grid_constant__ CUtensorMap tmO3,
                                   const GemmArgs args) {
   using C = PairCfg<MODE, RK>;
   constexpr bool kSwiGLU = C::kSwiGLU;
@@ -172,7 +362,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sStage = smem;
-  uint8_t* sLB = sStage + C::NS * C::STAGE_BYTES;
+  uint8_t* sRing = sStage + C::NS * C::STAGE_BYTES;  // epilogue store staging
+  uint8_t* sLB = sRing + C::RING_BYTES;
   uint8_t* sXA = sLB + 2 * C::LB_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sXA + 2 * C::XA_BYTES);
   uint64_t* empty = full + C::NS;
@@ -221,6 +412,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmXA);
     prefetch_tmap(&tmLB);
+  }
+  if (warp == 2 && lane == 0) {
+    prefetch_tmap(&tmO);
+    prefetch_tmap(&tmO2);
+    prefetch_tmap(&tmO3);
   }
   if (warp == 1) {
     tmem_alloc_pair(s_tmem, C::TMEM_COLS);
@@ -278,10 +474,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
           // the up factor rows of its tile columns
           const uint32_t lbb = lead(&lb_full[b]);
           uint8_t* lb = sLB + b * C::LB_BYTES;
-          const int lrow = e * args.lb_rows + n0;
-          tma_load_2d_pair(lb, &tmLB, lbb, 0, lrow);
-          if constexpr (kSwiGLU)
-            tma_load_2d_pair(lb + 64 * C::LSPAN, &tmLB, lbb, 0, lrow + args.I);
+          if constexpr (kBMN) {
+            // A[e] rows 0..r-1, this CTA's tile columns, as two atoms
+            tma_load_2d_pair(lb, &tmLB, lbb, n0, e * RK);
+            tma_load_2d_pair(lb + C::LB_ATOM, &tmLB, lbb, n0 + 64, e * RK);
+          } else {
+            const int lrow = e * args.lb_rows + n0;
+            tma_load_2d_pair(lb, &tmLB, lbb, 0, lrow);
+            if constexpr (kSwiGLU)
+              tma_load_2d_pair(lb + 64 * C::LSPAN, &tmLB, lbb, 0, lrow + args.I);
+          }
           tma_load_2d_pair(sXA + b * C::XA_BYTES, &tmXA, lbb, 0, row0);
         }
         ++n_lb;
@@ -324,8 +526,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
       // elected lane issues the tensor-core instructions.
       const uint32_t kIdesc = idesc_bf16_f32(256, Nt, false, kBMN);
       const uint32_t kIdescH = idesc_bf16_f32(128, Nt, false, kBMN);
-      const uint32_t kIdescUp = idesc_bf16_f32(256, Nt, false, false);
-      const uint32_t kIdescUpH = idesc_bf16_f32(128, Nt, false, false);
+      const uint32_t kIdescUp = idesc_bf16_f32(256, Nt, false, kBMN);
+      const uint32_t kIdescUpH = idesc_bf16_f32(128, Nt, false, kBMN);
       constexpr uint16_t kBoth = 0x3;
       const uint64_t a_desc0 = smem_desc(smem_u32(sStage), 16, 1024, kLayoutSW128);
       // MN-major: LBO = next 64-column atom, SBO = next 8 K-rows (8 x 128 B)
@@ -382,7 +584,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
 #pragma unroll
           for (int kk = 0; kk < RK / 16; ++kk)
             umma_bf16_pair(t_acc, smem_desc(xa0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
-                           smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT), idesc_up,
+                           kBMN ? smem_desc(lb0 + kk * 2048, C::LB_ATOM, 1024, kLayoutSW128)
+                                : smem_desc(lb0 + kk * 32, 16, 8 * C::LSPAN, C::LLAYOUT),
+                           idesc_up,
                            1u);
           umma_commit_pair_mc(&lb_empty[b], kBoth);
           umma_commit_pair_mc(&acc_full[b], kBoth);
@@ -405,6 +609,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
     const int ehalf = (warp - 2) >> 2;    // which share of the columns
     const uint32_t lane_base = static_cast<uint32_t>(ew * 32) << 16;
     const uint64_t pol = policy_evict_first();  // outputs stream out of L2
+    StoreRing<C::SBW, C::NSTG> ring{sRing + (warp - 2) * C::NSTG * C::SLOT_BYTES, 0};
     int local = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++local) {
       int e, mt, nt;
@@ -414,13 +619,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
       const bool half = pair_half_tile(s_off, e, mt);
       // half tile: lane quarters 0-1 hold rows 0-63 for tile columns
       // [0, 128), quarters 2-3 the same rows for [128, 256)
-      const int row_local = half ? (ew & 1) * 32 + lane : ew * 32 + lane;
-      const int grow = s_off[e] + mt * 2 * C::BM +
-                       static_cast<int>(rank) * (half ? C::BM / 2 : C::BM) + row_local;
+      const int wrow0 = half ? (ew & 1) * 32 : ew * 32;   // the warp's first row
+      const int y0 = s_off[e] + mt * 2 * C::BM +
+                     static_cast<int>(rank) * (half ? C::BM / 2 : C::BM) + wrow0;
+      const int grow = y0 + lane;
       const bool rvalid = grow < s_off[e + 1];
+      const bool rows_all = y0 + 32 <= s_off[e + 1];  // the warp's 32 rows are the expert's
       const uint32_t t_acc = tmem_base + lane_base + b * C::ACC_STRIDE;
       const int col0 = nt * Nt;             // first output column of the tile
-      const int cend = min(args.N, col0 + Nt);
       // (no L2 prefetch of the saved gate / up rows here: measured 1.5%
       // slower in this kernel)
       if (!warp_wait(&acc_full[b], use, s_abort, wait_ns)) break;
@@ -430,27 +636,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
         // 128 nt + 64 q .. +63, q = the block
         const int oc0 = nt * (BN / 2);
         if (half) {
-          epi_swiglu_seg64(args, t_acc, grow, rvalid, oc0 + (ew >> 1) * 64, pol);
+          epi_swiglu_seg64<C::kRing>(args, ring, &tmO, &tmO2, &tmO3, t_acc, grow, y0, rows_all, rvalid,
+                           oc0 + (ew >> 1) * 64, pol, lane);
         } else {
-          epi_swiglu_seg64(args, t_acc, grow, rvalid, oc0, pol);
-          epi_swiglu_seg64(args, t_acc + 128, grow, rvalid, oc0 + 64, pol);
+          epi_swiglu_seg64<C::kRing>(args, ring, &tmO, &tmO2, &tmO3, t_acc, grow, y0, rows_all, rvalid,
+                           oc0, pol, lane);
+          epi_swiglu_seg64<C::kRing>(args, ring, &tmO, &tmO2, &tmO3, t_acc + 128, grow, y0, rows_all,
+                           rvalid, oc0 + 64, pol, lane);
         }
       } else {
         // tile columns [0, Nt) = output columns col0 + c; TMEM columns past
         // Nt (or past N) hold nothing of this tile and are not stored
         if (half) {
           const int q = ew >> 1;
-          epi_drain<MODE, BN, kSplit, BN / 2>(args, t_acc, grow, rvalid, 0, ehalf,
-                                              col0 + q * NHt,
-                                              min(cend, col0 + (q + 1) * NHt));
+          epi_pair_drain<MODE, BN / 2, kSplit, C::kRing>(args, ring, &tmO, &tmO3, t_acc, grow, y0,
+                                               rows_all, rvalid, ehalf, col0 + q * NHt,
+                                               col0 + (q + 1) * NHt, pol, lane);
         } else {
-          epi_drain<MODE, BN, kSplit>(args, t_acc, grow, rvalid, 0, ehalf, col0, cend);
+          epi_pair_drain<MODE, BN, kSplit, C::kRing>(args, ring, &tmO, &tmO3, t_acc, grow, y0, rows_all,
+                                           rvalid, ehalf, col0, col0 + Nt, pol, lane);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead(&acc_empty[b]));
     }
+    if constexpr (C::kRing) ring.finish(lane);  // every staged store has left shared memory
   }
 
   // ---------------------------------------------------------------- teardown

@@ -250,8 +250,30 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* XA, const v
                        CU_TENSOR_MAP_SWIZZLE_128B);
   }
   ok = ok && tmap_2d(&txa, XA, RK, args.R, RK * 2ull, RK, C::BM, lora_swizzle(RK));
-  ok = ok && tmap_2d(&tlb, LB, RK, EU * args.lb_rows, RK * 2ull, RK, C::LB_BOX_ROWS,
-                     lora_swizzle(RK));
+  if constexpr (C::kBMN) {
+    // the up factor A [E, r, N] in place: [E * r, N], 64-column x r-row boxes
+    const uint64_t N = static_cast<uint64_t>(args.N);
+    ok = ok && tmap_2d(&tlb, LB, N, EU * RK, N * 2, 64, RK, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    ok = ok && tmap_2d(&tlb, LB, RK, EU * args.lb_rows, RK * 2ull, RK, C::LB_BOX_ROWS,
+                       lora_swizzle(RK));
+  }
+  // outputs, stored by the epilogue in boxes of 32 rows x SBW columns:
+  // gate_up fwd h [R, I], saved gate = Z1 columns [0, I) and saved up = Z1
+  // columns [I, 2I) (two views of Z1, so a box never spills from one half
+  // into the other); down bwd dZ1 = [dg | du] likewise; otherwise [R, N]
+  CUtensorMap to, to2, to3;
+  const CUtensorMapSwizzle osw =
+      C::SBW == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const uint64_t R = static_cast<uint64_t>(args.R), N = static_cast<uint64_t>(args.N);
+  ok = ok && tmap_2d(&to, args.out, N, R, args.ld_out * 2ull, C::SBW, 32, osw);
+  to2 = to3 = to;
+  if constexpr (MODE == kGateUpFwd) {
+    ok = ok && tmap_2d(&to2, args.out2, N, R, args.ld_out2 * 2ull, C::SBW, 32, osw);
+    ok = ok && tmap_2d(&to3, args.out2 + args.I, N, R, args.ld_out2 * 2ull, C::SBW, 32, osw);
+  } else if constexpr (MODE == kDownBwd) {
+    ok = ok && tmap_2d(&to3, args.out + args.I, N, R, args.ld_out * 2ull, C::SBW, 32, osw);
+  }
   if (!ok) return MOE_ERR_CUDA;
   auto kern = grouped_lora_gemm_pair_kernel<MODE, RK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -266,7 +288,7 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* XA, const v
                  : MODE == kDownBwd   ? MOE_PROF_DOWN_BWD
                                       : MOE_PROF_GATE_UP_BWD,
                  st);
-  kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tw, txa, tlb, args);
+  kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tw, txa, tlb, to, to2, to3, args);
   count_launch();
   return launch_status();
 }
@@ -699,14 +721,19 @@ moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
   const int warps = 8;
   const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
   ProfScope prof(MOE_PROF_PERMUTE, stream);
-  if (dw == nullptr)
-    permute_rows_kernel<<<grid, warps * 32, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
-        static_cast<__nv_bfloat16*>(Xp));
-  else
+  if (dw == nullptr) {
+    const int vpl = permute_vpl(H / 8);
+    auto kern = vpl == 4    ? permute_rows_kernel<4>
+                : vpl == 8  ? permute_rows_kernel<8>
+                : vpl == 12 ? permute_rows_kernel<12>
+                            : permute_rows_kernel<16>;
+    kern<<<grid, warps * 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), dest, scale, T,
+                                          H, k, static_cast<__nv_bfloat16*>(Xp));
+  } else {
     permute_kernel<<<grid, warps * 32, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
         static_cast<__nv_bfloat16*>(Xp), static_cast<const __nv_bfloat16*>(Zp), dw);
+  }
   count_launch();
   return launch_status();
 }
@@ -981,8 +1008,9 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
   }
   __nv_bfloat16* dzb2_rm = at<__nv_bfloat16>(ws, wo[7]);
   __nv_bfloat16* dzb1_rm = at<__nv_bfloat16>(ws, wo[8]);
-  prep.transpose(A2, A2t, E, r, I);
-  prep.transpose(A1, A1t, E, r, H);
+  // (the CTA-pair kernels read A2, A1 in place as MN-major operands)
+  if (!pair_down) prep.transpose(A2, A2t, E, r, I);
+  if (!pair_gate_up) prep.transpose(A1, A1t, E, r, H);
   if ((stt = prep.launch(st)) != MOE_OK) return stt;
   const CUtensorMapSwizzle lsw = lora_swizzle(r);
   const uint64_t EU = static_cast<uint64_t>(E);
@@ -1002,7 +1030,7 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     if ((stt = rank_down(r, false, dZ2, B2, H, expert_offsets, E, R, s, dzb2_rm, dzb2, st)) !=
         MOE_OK)
       return stt;
-    if ((stt = launch_pair<kDownBwd>(r, dZ2, W2, dzb2_rm, A2t, g, st)) != MOE_OK) return stt;
+    if ((stt = launch_pair<kDownBwd>(r, dZ2, W2, dzb2_rm, A2, g, st)) != MOE_OK) return stt;
   } else {
     const int bn = pick_bn(I, false, r, true);
     CUtensorMap ta, tb, tla, tlb;
@@ -1020,40 +1048,10 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     g.stall_test = g_stall_test;
     if ((stt = launch_gemm<kDownBwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
   }
-  // gate_up backward: dXp = dZ1 W1 + s (dZ1 B1) A1
-  if (pair_gate_up) {
-    const int bn = pair_tile_n(H, true);
-    GemmArgs g{};
-    g.offsets = expert_offsets;
-    g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
-    g.tile_n = bn;
-    g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
-    g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
-    g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
-    g.stall_test = g_stall_test;
-    if ((stt = rank_down(r, false, dZ1, B1, 2 * I, expert_offsets, E, R, s, dzb1_rm, dzb1, st)) !=
-        MOE_OK)
-      return stt;
-    if ((stt = launch_pair<kGateUpBwd>(r, dZ1, W1, dzb1_rm, A1t, g, st)) != MOE_OK) return stt;
-  } else {
-    const int bn = pick_bn(H, false, r, true);
-    CUtensorMap ta, tb, tla, tlb;
-    bool ok = tmap_2d(&ta, dZ1, 2 * I, R, 4ull * I, kGemmBK, 128, kKmajSwz);
-    ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tla, B1p, 64, EU * 2 * I, 128, 64, kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && tmap_2d(&tlb, A1t, r, EU * H, r * 2ull, r, bn, lsw);
-    if (!ok) return MOE_ERR_CUDA;
-    GemmArgs g{};
-    g.offsets = expert_offsets;
-    g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
-    g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
-    g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
-    g.lora_t = dzb1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
-    g.stall_test = g_stall_test;
-    if ((stt = launch_gemm<kGateUpBwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
-  }
-  // LoRA gradients
-  {
+  // LoRA gradients, after the gate_up GEMM (measured: running them before
+  // it, right after the s dZ1 B1 pass, makes neither faster)
+  auto lora_grads = [&]() -> moe_status_t {
+    moe_status_t stt;
     const int ldr = ld_rank(R);
     const void* U[4] = {Xp, dZ1, h, dZ2};
     const void* V[4] = {dzb1, xa1, dzb2, ha2};
@@ -1081,7 +1079,41 @@ moe_status_t lora_mlp_bwd_impl(const void* dZ2, const void* Xp,
     if (r == 16) stt = launch_grad_t<16>(tu, tv, g, st);
     else if (r == 32) stt = launch_grad_t<32>(tu, tv, g, st);
     else stt = launch_grad_t<64>(tu, tv, g, st);
-    if (stt != MOE_OK) return stt;
+    return stt;
+  };
+  // gate_up backward: dXp = dZ1 W1 + s (dZ1 B1) A1
+  if (pair_gate_up) {
+    const int bn = pair_tile_n(H, true);
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
+    g.tile_n = bn;
+    g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
+    g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
+    g.lora_t = nullptr; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
+    if ((stt = rank_down(r, false, dZ1, B1, 2 * I, expert_offsets, E, R, s, dzb1_rm, dzb1, st)) !=
+        MOE_OK)
+      return stt;
+    if ((stt = launch_pair<kGateUpBwd>(r, dZ1, W1, dzb1_rm, A1, g, st)) != MOE_OK) return stt;
+    if ((stt = lora_grads()) != MOE_OK) return stt;
+  } else {
+    const int bn = pick_bn(H, false, r, true);
+    CUtensorMap ta, tb, tla, tlb;
+    bool ok = tmap_2d(&ta, dZ1, 2 * I, R, 4ull * I, kGemmBK, 128, kKmajSwz);
+    ok = ok && tmap_2d(&tb, W1, H, EU * 2 * I, H * 2ull, 64, kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tla, B1p, 64, EU * 2 * I, 128, 64, kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && tmap_2d(&tlb, A1t, r, EU * H, r * 2ull, r, bn, lsw);
+    if (!ok) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.offsets = expert_offsets;
+    g.E = E; g.R = R; g.K = 2 * I; g.N = H; g.n_tiles = (H + bn - 1) / bn; g.I = I;
+    g.b_rows = 2 * I; g.lb_rows = H; g.s = s;
+    g.out = static_cast<__nv_bfloat16*>(dXp); g.ld_out = H;
+    g.lora_t = dzb1; g.ld_lora = ld_rank(R); g.wait_ns = g_wait_limit_ns;
+    g.stall_test = g_stall_test;
+    if ((stt = launch_gemm<kGateUpBwd>(bn, r, ta, tb, tla, tlb, g, st)) != MOE_OK) return stt;
+    if ((stt = lora_grads()) != MOE_OK) return stt;
   }
   // base-weight gradients (full fine-tuning)
   if (full &&

@@ -48,11 +48,10 @@ __device__ __forceinline__ float dot8(uint4 a, uint4 b) {
 
 constexpr int kCopyUnroll = 4;
 
-constexpr int kRowVec = 8;  // 16-byte vectors per lane held at once
-
 // Xp[dest[t,j]] = (scale ? scale[t,j] : 1) * X[t].  One warp per token: the
-// row is read once into registers (kRowVec vectors per lane in flight) and
-// written to all k destinations.
+// row is read once into registers (VPL 16-byte vectors per lane in flight per
+// pass, permute_vpl) and written to all k destinations.
+template <int kRowVec>
 __global__ void __launch_bounds__(256)
     permute_rows_kernel(const __nv_bfloat16* __restrict__ X,
                         const int32_t* __restrict__ dest,
@@ -96,6 +95,16 @@ __global__ void __launch_bounds__(256)
       }
     }
   }
+}
+
+// Vectors per lane per pass of permute_rows_kernel for rows of nvec 16-byte
+// vectors: enough for a whole row in one pass up to 512 vectors (H = 4096),
+// in multiples of 4 (fewest idle lane slots: H = 2880 takes 12, one pass
+// with 94% of the slots used, where 8 took two passes at 70%).
+inline int permute_vpl(int nvec) {
+  const int per_lane = (nvec + 31) / 32;
+  const int v = (per_lane + 3) / 4 * 4;
+  return v < 4 ? 4 : (v > 16 ? 16 : v);
 }
 
 // Same with the routing-weight gradient dw[t,j] = <X[t], Zp[dest[t,j]]>.

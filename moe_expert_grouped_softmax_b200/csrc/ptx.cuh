@@ -228,6 +228,37 @@ __device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const CUtensorM
       : "memory");
 }
 
+// 2-D tiled bulk tensor store shared -> global of one box, with an L2 cache
+// policy; completion is tracked in this thread's bulk async-groups.  Boxes
+// are clipped at the tensor map's extent.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int x,
+                                             int y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], "
+      "[%1], %4;" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+// Closes this thread's current bulk async-group.
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until at most N of this thread's bulk async-groups still read their
+// shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Waits until at most N of this thread's bulk async-groups are incomplete
+// (their global writes done).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Marks `bytes` of the current phase's expected transaction count as done
 // without a copy (balances copies that were expected but never issued).
 __device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {

@@ -456,3 +456,25 @@ class MoeBlock:
         ``logits`` (which may then be None)."""
         self.forward(X, logits, W, Wr)
         self.backward(dY, W, Wr)
+
+    def capture(self, X, logits, dY, W, Wr=None):
+        """Capture one ``step`` on these exact tensors into a CUDA graph;
+        ``replay`` then re-runs all of its kernels with one launch.  Inputs
+        must be updated in place (the graph holds their addresses).  The
+        library launches nothing but its own kernels and stream-ordered
+        memsets, and allocates nothing, so the captured step is the same work
+        as ``step``."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):      # one eager step off the capture
+            self.step(X, logits, dY, W, Wr)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.step(X, logits, dY, W, Wr)
+        self._graph = graph
+        return graph
+
+    def replay(self):
+        """Run the captured step on the current stream."""
+        self._graph.replay()
