@@ -171,14 +171,6 @@ __device__ __forceinline__ void decode_tile(int tile, int n_tiles,
   }
 }
 
-// Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag,
-                                          uint64_t limit_ns) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
-  return __all_sync(0xffffffffu, ok);
-}
-
 // warp_wait for a barrier that other CTAs of the cluster arrive on.
 __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort_flag,
@@ -190,22 +182,6 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity
 // Lane 0's view of a non-blocking barrier test, for the whole warp.
 __device__ __forceinline__ bool warp_uniform(bool v) {
   return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0;
-}
-
-// Bounded wait that ignores the abort flag, used before exit to let copies
-// and MMAs already in flight land.  Its limit never drops below one second,
-// whatever the configured wait limit, so that a CTA does not leave while its
-// own asynchronous work is still writing into it.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity,
-                                           uint64_t limit_ns) {
-  const uint64_t limit = limit_ns > 1000000000ull ? limit_ns : 1000000000ull;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit) {
-      set_status(4);
-      return;
-    }
-  }
 }
 
 // drain_wait for a barrier that other CTAs of the cluster arrive on with

@@ -178,7 +178,12 @@ constexpr int kCombVec = 4;  // 16-byte vectors per lane per source row
 // Y[t] = sum_j (w ? w[t,j] : 1) * Yp[dest[t,j]], fp32 in j order -> bf16.
 // With a trained router (Wr != nullptr) the router's part of dX is added
 // before the one rounding: + sum_j g[t,j] * Wr[idx[t,j]] (Wr [E, H] bf16).
-// One warp per token; kCombVec x k loads in flight per lane.
+// One warp per token.  The token's destination rows and weights are read
+// once (lane j holds slot j, broadcast by shuffle) and two source rows'
+// kCombVec vectors per lane are loaded before either is accumulated (the
+// sum stays in j order).  Measured against one row at a time with dest
+// re-read per row: Qwen3-30B-A3B shape (k = 8) 117 -> 103 us, gpt-oss-20b
+// shape unchanged.
 __global__ void __launch_bounds__(256)
     unpermute_kernel(const __nv_bfloat16* __restrict__ Yp,
                      const int32_t* __restrict__ dest,
@@ -191,35 +196,73 @@ __global__ void __launch_bounds__(256)
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const int nvec = H >> 3;
   const int R = T * k;
+  auto fma8 = [](float* a, float c, uint4 z) {
+    a[0] = fmaf(c, bf16_lo(z.x), a[0]);
+    a[1] = fmaf(c, bf16_hi(z.x), a[1]);
+    a[2] = fmaf(c, bf16_lo(z.y), a[2]);
+    a[3] = fmaf(c, bf16_hi(z.y), a[3]);
+    a[4] = fmaf(c, bf16_lo(z.z), a[4]);
+    a[5] = fmaf(c, bf16_hi(z.z), a[5]);
+    a[6] = fmaf(c, bf16_lo(z.w), a[6]);
+    a[7] = fmaf(c, bf16_hi(z.w), a[7]);
+  };
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     char* yrow = reinterpret_cast<char*>(Y + static_cast<size_t>(t) * H);
+    // slots j0 .. j0 + 31 of the token on lanes 0 .. 31 (k <= 32 in one go)
+    int my_d = -1;
+    float my_c = 1.f;
+    if (lane < k) {
+      my_d = dest[static_cast<size_t>(t) * k + lane];
+      if (w) my_c = w[static_cast<size_t>(t) * k + lane];
+      if (my_d < 0 || my_d >= R) {
+        set_status(5);
+        my_d = -1;
+      }
+    }
     for (int v0 = lane; v0 < nvec; v0 += 32 * kCombVec) {
       float acc[kCombVec][8];
 #pragma unroll
       for (int u = 0; u < kCombVec; ++u)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-      for (int j = 0; j < k; ++j) {
-        int d = dest[static_cast<size_t>(t) * k + j];
-        if (d < 0 || d >= R) {
-          if (lane == 0) set_status(5);
-          continue;
+      for (int j0 = 0; j0 < k; j0 += 32) {
+        int dj = my_d;
+        float cj = my_c;
+        if (j0 > 0) {  // slots past 32 (k > 32): reload for this group
+          dj = -1;
+          cj = 1.f;
+          if (j0 + lane < k) {
+            dj = dest[static_cast<size_t>(t) * k + j0 + lane];
+            if (w) cj = w[static_cast<size_t>(t) * k + j0 + lane];
+            if (dj < 0 || dj >= R) {
+              if (v0 == lane) set_status(5);
+              dj = -1;
+            }
+          }
         }
-        const float c = w ? w[static_cast<size_t>(t) * k + j] : 1.f;
-        const char* zrow = reinterpret_cast<const char*>(Yp + static_cast<size_t>(d) * H);
+        const int nj = min(32, k - j0);
+        for (int jj = 0; jj < nj; jj += 2) {
+          const int da = __shfl_sync(0xffffffffu, dj, jj);
+          const float ca = __shfl_sync(0xffffffffu, cj, jj);
+          const int db = __shfl_sync(0xffffffffu, dj, jj + 1 < nj ? jj + 1 : jj);
+          const float cb = __shfl_sync(0xffffffffu, cj, jj + 1 < nj ? jj + 1 : jj);
+          const bool has_b = jj + 1 < nj;
+          uint4 za[kCombVec], zb[kCombVec];
 #pragma unroll
-        for (int u = 0; u < kCombVec; ++u) {
-          const int v = v0 + 32 * u;
-          if (v < nvec) {
-            const uint4 z = ld_nc_v4(zrow + 16 * static_cast<size_t>(v));
-            acc[u][0] = fmaf(c, bf16_lo(z.x), acc[u][0]);
-            acc[u][1] = fmaf(c, bf16_hi(z.x), acc[u][1]);
-            acc[u][2] = fmaf(c, bf16_lo(z.y), acc[u][2]);
-            acc[u][3] = fmaf(c, bf16_hi(z.y), acc[u][3]);
-            acc[u][4] = fmaf(c, bf16_lo(z.z), acc[u][4]);
-            acc[u][5] = fmaf(c, bf16_hi(z.z), acc[u][5]);
-            acc[u][6] = fmaf(c, bf16_lo(z.w), acc[u][6]);
-            acc[u][7] = fmaf(c, bf16_hi(z.w), acc[u][7]);
+          for (int u = 0; u < kCombVec; ++u) {
+            const int v = v0 + 32 * u;
+            za[u] = zb[u] = make_uint4(0, 0, 0, 0);
+            if (v < nvec && da >= 0)
+              za[u] = ld_nc_v4(reinterpret_cast<const char*>(Yp + static_cast<size_t>(da) * H) +
+                               16 * static_cast<size_t>(v));
+            if (v < nvec && has_b && db >= 0)
+              zb[u] = ld_nc_v4(reinterpret_cast<const char*>(Yp + static_cast<size_t>(db) * H) +
+                               16 * static_cast<size_t>(v));
+          }
+#pragma unroll
+          for (int u = 0; u < kCombVec; ++u) {
+            if (da >= 0) fma8(acc[u], ca, za[u]);
+            if (has_b && db >= 0) fma8(acc[u], cb, zb[u]);
           }
         }
       }
@@ -235,17 +278,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u) {
             const int v = v0 + 32 * u;
-            if (v < nvec) {
-              const uint4 z = *reinterpret_cast<const uint4*>(wrow + 16 * static_cast<size_t>(v));
-              acc[u][0] = fmaf(c, bf16_lo(z.x), acc[u][0]);
-              acc[u][1] = fmaf(c, bf16_hi(z.x), acc[u][1]);
-              acc[u][2] = fmaf(c, bf16_lo(z.y), acc[u][2]);
-              acc[u][3] = fmaf(c, bf16_hi(z.y), acc[u][3]);
-              acc[u][4] = fmaf(c, bf16_lo(z.z), acc[u][4]);
-              acc[u][5] = fmaf(c, bf16_hi(z.z), acc[u][5]);
-              acc[u][6] = fmaf(c, bf16_lo(z.w), acc[u][6]);
-              acc[u][7] = fmaf(c, bf16_hi(z.w), acc[u][7]);
-            }
+            if (v < nvec)
+              fma8(acc[u], c, *reinterpret_cast<const uint4*>(wrow + 16 * static_cast<size_t>(v)));
           }
         }
       }

@@ -99,6 +99,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 }
 
 // ------------------------------------------------------- CTA-pair helpers
+// Warp-uniform bounded wait: every lane polls; the warp agrees on the result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -257,6 +265,22 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 template <int N>
 __device__ __forceinline__ void bulk_wait_group() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Bounded wait that ignores the abort flag, used before exit to let copies
+// and MMAs already in flight land.  Its limit never drops below one second,
+// whatever the configured wait limit, so that a CTA does not leave while its
+// own asynchronous work is still writing into it; records
+// MOE_ERR_DEVICE_TIMEOUT if they never land.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t limit = limit_ns > 1000000000ull ? limit_ns : 1000000000ull;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit) {
+      set_status(4);
+      return;
+    }
+  }
 }
 
 // Marks `bytes` of the current phase's expected transaction count as done
