@@ -208,6 +208,32 @@ MOE_API moe_status_t moe_lora_mlp_bwd_full(const void* dZ2, const void* Xp,
                                    void* dB2, void* dW1, void* dW2, void* ws,
                                    size_t ws_bytes, moe_stream_t stream);
 
+/* ------------------------------------------ expert parallelism (optional)
+ * The pages call multi-GPU training experimental (winningdata.io hands-on
+ * blog, section "Limitações"); they give no design.  With the E experts split
+ * over N ranks (rank p holds experts [p * E_loc, (p + 1) * E_loc)), each rank
+ * routes and permutes its own tokens over all E experts; its expert-major
+ * rows are then already ordered by destination rank, and one all-to-all
+ * (NCCL, called by the caller) sends each rank its experts' rows.  The
+ * receiving rank holds them source-major: for each source s in turn, s's
+ * rows for the E_loc local experts in expert order.  moe_ep_regroup moves
+ * rows between that order and the expert-major order over all sources that
+ * the local grouped GEMMs take (moe_lora_mlp_fwd / _bwd with E = E_loc);
+ * within each (source, expert) segment the rows keep their order.
+ *   in, out  bf16 [rows, H] device, 16-byte aligned, not overlapping.
+ *   counts   int32 [N, E_loc] device: rows source s sent for local expert e
+ *            (the all-to-all of moe_route_topk's expert_counts); rows must
+ *            equal their sum, else MOE_ERR_DEVICE_BOUNDS is recorded and
+ *            nothing is written.
+ *   dir      0: out = in reordered source-major -> expert-major (dispatch);
+ *            1: expert-major -> source-major (before the return all-to-all).
+ *   offsets  int32 [E_loc + 1] device, or NULL; dir 0 only: the local
+ *            experts' row offsets in the expert-major order ([E_loc] = rows).
+ *   N * E_loc <= 4096, H a multiple of 8.  Nothing is allocated. */
+MOE_API moe_status_t moe_ep_regroup(const void* in, const int32_t* counts, int N, int E_loc,
+                                    int rows, int H, int dir, void* out, int32_t* offsets,
+                                    moe_stream_t stream);
+
 /* ------------------------------------------ trained router (optional)
  * The pages keep the router frozen by default; these two calls make it
  * trainable.  moe_router_fwd: logits [T, E] fp32 = X [T, H] bf16 times

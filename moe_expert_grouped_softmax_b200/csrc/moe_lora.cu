@@ -21,6 +21,7 @@
 #include "base_grad.cuh"
 #include "router.cuh"
 #include "rank_down.cuh"
+#include "ep.cuh"
 
 using namespace moe;
 
@@ -826,6 +827,36 @@ moe_status_t moe_unpermute(const void* Yp, const int32_t* dest, const float* w, 
   unpermute_kernel<<<grid, warps * 32, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(Yp), dest, w, T, H, k,
       static_cast<__nv_bfloat16*>(Y));
+  count_launch();
+  return launch_status();
+}
+
+// ------------------------------------------------------ expert parallelism
+moe_status_t moe_ep_regroup(const void* in, const int32_t* counts, int N, int E_loc, int rows,
+                            int H, int dir, void* out, int32_t* offsets, moe_stream_t stream) {
+  if (N < 1 || E_loc < 1 || static_cast<long long>(N) * E_loc > kRegroupMaxSegs || rows < 0 ||
+      H <= 0 || (H % 8) || (dir != 0 && dir != 1))
+    return MOE_ERR_UNSUPPORTED;
+  if (!counts) return MOE_ERR_INVALID_ARG;
+  if (offsets != nullptr && dir != 0) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = stream;
+  if (rows > 0) {
+    if (!in || !out) return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 15u)
+      return MOE_ERR_INVALID_ARG;
+  }
+  const int nseg = N * E_loc;
+  const size_t smem = (2 * static_cast<size_t>(nseg) + 1 + 32) * 4;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(ep_regroup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int warps = kRegroupThreads / 32;
+  const int grid =
+      std::max(1, std::min((rows + warps - 1) / warps, std::max(1, num_sms()) * 8));
+  ep_regroup_kernel<<<grid, kRegroupThreads, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(in), counts, N, E_loc, rows, H, dir,
+      static_cast<__nv_bfloat16*>(out), offsets);
   count_launch();
   return launch_status();
 }

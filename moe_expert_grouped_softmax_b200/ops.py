@@ -27,7 +27,7 @@ EXPORTS = [
     "moe_status_string", "moe_set_wait_limit_ns", "moe_test_inject_stall",
     "moe_set_cta_pairs", "moe_uses_cta_pairs", "moe_kernel_launches", "moe_profile_enable",
     "moe_router_fwd", "moe_router_bwd_workspace_bytes", "moe_router_bwd",
-    "moe_profile_collect",
+    "moe_profile_collect", "moe_ep_regroup",
 ]
 
 PROF_KINDS = {"route": 0, "permute": 1, "gate_up_fwd": 2, "down_fwd": 3,
@@ -100,6 +100,8 @@ def lib():
         L.moe_profile_enable.restype = I
         L.moe_profile_collect.argtypes = [I, ctypes.POINTER(ctypes.c_float), I]
         L.moe_profile_collect.restype = I
+        L.moe_ep_regroup.argtypes = [P, P, I, I, I, I, I, P, P, P]
+        L.moe_ep_regroup.restype = I
         _lib = L
     return _lib
 
@@ -300,6 +302,25 @@ def unpermute(Yp, dest, w=None, out=None):
         out = torch.empty((T, H), dtype=torch.bfloat16, device=Yp.device)
     _check(lib().moe_unpermute(_p(Yp), _p(dest), _p(w), T, H, k, _p(out), _stream()),
            "moe_unpermute")
+    return out
+
+
+def ep_regroup(inp, counts, direction, out=None, offsets=None):
+    """Expert parallelism: rows from N source ranks for this rank's E_loc
+    experts (``counts`` [N, E_loc] int32 on the device), source-major ->
+    expert-major (``direction`` 0, optionally writing the local ``offsets``
+    [E_loc + 1]) or back (1)."""
+    rows, H = inp.shape
+    N, EL = counts.shape
+    _need(inp, torch.bfloat16, (rows, H), "rows")
+    _need(counts, torch.int32, (N, EL), "counts")
+    if out is None:
+        out = torch.empty_like(inp)
+    if offsets is not None:
+        _need(offsets, torch.int32, (EL + 1,), "offsets")
+    _check(lib().moe_ep_regroup(_p(inp), _p(counts), N, EL, rows, H, int(direction), _p(out),
+                                _p(offsets), _stream()),
+           "moe_ep_regroup")
     return out
 
 

@@ -159,6 +159,28 @@ def test_host_side_argument_errors(L):
                               B(E * 16 * I * 2), B(E * H * 16 * 2), B(wsb), 16, None) == 1
 
 
+def test_ep_regroup_host_side_argument_errors(L):
+    """Every rejection returns before a launch (no GPU needed)."""
+    B = _Buffers()
+    N, EL, rows, H = 2, 4, 10, 16
+
+    def bufs(n, el, h):
+        return B(rows * h * 2), B(n * el * 4), B(rows * h * 2), B((el + 1) * 4)
+
+    i, c, o, off = bufs(N, EL, H)
+    # unsupported: H not a multiple of 8, too many segments, bad direction
+    i12, c12, o12, _ = bufs(N, EL, 12)
+    assert L.moe_ep_regroup(i12, c12, N, EL, rows, 12, 0, o12, None, None) == 2
+    assert L.moe_ep_regroup(None, None, 65, 64, rows, H, 0, None, None, None) == 2
+    assert L.moe_ep_regroup(i, c, N, EL, rows, H, 2, o, None, None) == 2
+    assert L.moe_ep_regroup(i, c, 0, EL, rows, H, 0, o, None, None) == 2
+    # invalid: null counts, null rows with rows > 0, offsets with direction 1
+    assert L.moe_ep_regroup(i, None, N, EL, rows, H, 0, o, None, None) == 1
+    assert L.moe_ep_regroup(None, c, N, EL, rows, H, 0, o, None, None) == 1
+    assert L.moe_ep_regroup(i, c, N, EL, rows, H, 0, None, None, None) == 1
+    assert L.moe_ep_regroup(i, c, N, EL, rows, H, 1, o, off, None) == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "_LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(ops, "_lib", None)
