@@ -251,22 +251,42 @@ def run_ours(args, cfg):
         raise RuntimeError(f"device status {st} after timed steps")
     ms_steps = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     ms_total = float(sum(ms_steps))
-    # per-kernel durations: the same steps again, launched eagerly with a CUDA
-    # event pair around every launch on the launching stream (kept out of the
-    # headline timing above, which they would slow down)
-    ops.profile_enable(True)
+    # per-kernel durations: the same steps again with a CUDA event pair around
+    # every launch on the launching stream (kept out of the headline timing
+    # above, which they would slow down).  With graph launch the step is
+    # captured once more with the events as record nodes and replayed, so
+    # that no host launch gap falls inside a kernel's event pair; eager
+    # launch records them around each eager launch.
+    durations = {kind: [] for kind in ops.PROF_KINDS}
     barrier()
-    for i in range(K):
-        flush.zero_()
-        blk.step(X, logits, dY, W, Wr)
-    torch.cuda.synchronize()
+    if use_graph:
+        ops.profile_enable(True)
+        pgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(pgraph):
+            blk.step(X, logits, dY, W, Wr)
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()
+            pgraph.replay()
+            torch.cuda.synchronize()
+            for kind in ops.PROF_KINDS:
+                durations[kind] += ops.profile_collect(kind)
+        ops.profile_enable(False)
+        del pgraph
+    else:
+        ops.profile_enable(True)
+        for i in range(K):
+            flush.zero_()
+            blk.step(X, logits, dY, W, Wr)
+        torch.cuda.synchronize()
+        for kind in ops.PROF_KINDS:   # collect before the hook is switched off
+            durations[kind] = ops.profile_collect(kind)
+        ops.profile_enable(False)
     kern = {}
-    for kind in ops.PROF_KINDS:   # collect before the hook is switched off
-        d = ops.profile_collect(kind)
+    for kind, d in durations.items():
         if d:
             kern[kind] = {"launches": len(d), "avg_ms": float(np.mean(d)),
                           "total_ms": float(np.sum(d))}
-    ops.profile_enable(False)
     st = ops.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after timed steps")
@@ -430,7 +450,11 @@ def main():
               "parallelism": "replicas", "l2": "256 MiB memset before each step, "
               "outside the timed span",
               "launch": ("one CUDA graph of the whole step, replayed" if args.launch == "graph"
-                         else "eager launches")}
+                         else "eager launches"),
+              "kernel_timing": ("CUDA event pairs as record nodes of a second graph of the "
+                                "step, replayed K times after the timed steps"
+                                if args.launch == "graph" else
+                                "CUDA event pairs around each eager launch, K more steps")}
     ws, rank, _ = dist_env()
 
     if args.impl == "reference":

@@ -78,11 +78,18 @@ cudaEvent_t g_prof_ev[MOE_PROF_KINDS][kProfCap][2];
 int g_prof_n[MOE_PROF_KINDS];
 bool g_prof_created = false;
 
+// Under stream capture the records become event-record nodes of the graph
+// (re-recorded by every replay), so that a replayed step can be timed per
+// kernel without host launch gaps between the launches.
 void prof_record(int kind, int which, cudaStream_t st) {
   if (!g_prof_on || kind < 0 || kind >= MOE_PROF_KINDS) return;
   const int n = g_prof_n[kind];
   if (n >= kProfCap) return;
-  cudaEventRecord(g_prof_ev[kind][n][which], st);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) == cudaSuccess && cap == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(g_prof_ev[kind][n][which], st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(g_prof_ev[kind][n][which], st);
   if (which == 1) g_prof_n[kind] = n + 1;
 }
 
@@ -623,74 +630,11 @@ moe_status_t moe_get_device_status(moe_stream_t stream) {
 }
 
 // ------------------------------------------------------------------ route
-// Workspace: per-CTA expert histograms (the four-kernel path's chunks, or the
-// one-launch path's CTAs, whichever is more), the in-CTA ranks, and the
-// one-launch path's arrival counter.
 size_t moe_route_workspace_bytes(int T, int E, int k) {
   if (T <= 0 || E <= 0 || k <= 0) return 256;
   const size_t R = static_cast<size_t>(T) * k;
   const size_t nblk = (R + kRankChunk - 1) / kRankChunk;
-  const size_t nhist = std::max<size_t>(nblk, kRFMaxCtas);
-  return align256(nhist * E * 4) + align256(R * 4) + 256;
-}
-
-#ifndef MOE_ROUTE_FUSED
-#define MOE_ROUTE_FUSED 0
-#endif
-
-// The one-launch router (route_fused_kernel) as a cooperative launch, so
-// that all its CTAs are resident for its one grid-wide wait.  *done stays
-// false where the device cannot hold the grid at once or has no cooperative
-// launch; the caller then runs the four kernels.
-static moe_status_t launch_route_fused(const float* logits, int T, int E, int k,
-                                       int32_t* topk_idx, float* topk_w, int32_t* counts,
-                                       int32_t* offsets, int32_t* dest, int32_t* blk_hist,
-                                       int32_t* local_rank, unsigned int* arrived,
-                                       cudaStream_t st, bool* done) {
-  *done = false;
-  int dev = 0, coop = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  const int sms = num_sms();
-  if (!coop || sms < 1) return MOE_OK;
-  int G = std::min(T, std::min(sms, kRFMaxCtas));
-  const int tpc = (T + G - 1) / G;
-  G = (T + tpc - 1) / tpc;
-  const size_t smem = route_fused_smem(E, k);
-  const int epl = (E + 31) / 32;
-  void (*kern)(const float*, int, int, int, int, int32_t*, float*, int32_t*, int32_t*,
-               int32_t*, int32_t*, int32_t*, unsigned int*, uint64_t) =
-      epl <= 1 ? route_fused_kernel<1>
-      : epl <= 2 ? route_fused_kernel<2>
-      : epl <= 4 ? route_fused_kernel<4>
-      : epl <= 8 ? route_fused_kernel<8>
-                 : route_fused_kernel<16>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kRFThreads, smem) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (static_cast<long long>(occ) * sms < G) return MOE_OK;
-  if (cudaMemsetAsync(arrived, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(G);
-  cfg.blockDim = dim3(kRFThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, logits, T, E, k, tpc, topk_idx, topk_w, counts, offsets,
-                         dest, blk_hist, local_rank, arrived, g_wait_limit_ns) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  count_launch();
-  *done = true;
-  return launch_status();
+  return align256(nblk * E * 4) + align256(R * 4);
 }
 
 moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* topk_idx,
@@ -711,19 +655,8 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
   ProfScope prof(MOE_PROF_ROUTE, st);
   const int R = T * k;
   const int nblk = (R + kRankChunk - 1) / kRankChunk;
-  const size_t hist_bytes =
-      align256(static_cast<size_t>(std::max(nblk, kRFMaxCtas)) * E * 4);
   int32_t* blk_hist = static_cast<int32_t*>(ws);
-  int32_t* local_rank = at<int32_t>(ws, hist_bytes);
-  if (MOE_ROUTE_FUSED && (reinterpret_cast<uintptr_t>(ws) & 15u) == 0) {
-    unsigned int* arrived =
-        at<unsigned int>(ws, hist_bytes + align256(static_cast<size_t>(R) * 4));
-    bool done = false;
-    const moe_status_t s0 = launch_route_fused(logits, T, E, k, topk_idx, topk_w, expert_counts,
-                                               expert_offsets, dest, blk_hist, local_rank,
-                                               arrived, st, &done);
-    if (s0 != MOE_OK || done) return s0;
-  }
+  int32_t* local_rank = at<int32_t>(ws, align256(static_cast<size_t>(nblk) * E * 4));
   // 1. top-k + weights, one token per warp
   const size_t smem1 = static_cast<size_t>(kRouteWarps) * k * 4;
   const int epl = (E + 31) / 32;
@@ -824,9 +757,10 @@ moe_status_t moe_unpermute(const void* Yp, const int32_t* dest, const float* w, 
   const int warps = 8;
   const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
   ProfScope prof(MOE_PROF_UNPERMUTE, stream);
-  unpermute_kernel<<<grid, warps * 32, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(Yp), dest, w, T, H, k,
-      static_cast<__nv_bfloat16*>(Y));
+  auto kern = combine_vec(H / 8) == 4 ? unpermute_kernel<4, 3> : unpermute_kernel<2, 4>;
+  kern<<<grid, warps * 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(Yp), dest, w, T, H, k,
+                                        static_cast<__nv_bfloat16*>(Y), nullptr, nullptr,
+                                        nullptr, 0);
   count_launch();
   return launch_status();
 }
@@ -916,7 +850,8 @@ moe_status_t moe_router_bwd(const float* w, const float* dw, const int32_t* topk
   if ((s = launch_status()) != MOE_OK) return s;
   const int warps = 8;
   const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
-  unpermute_kernel<<<grid, warps * 32, 0, st>>>(
+  auto kern = combine_vec(H / 8) == 4 ? unpermute_kernel<4, 3> : unpermute_kernel<2, 4>;
+  kern<<<grid, warps * 32, 0, st>>>(
       static_cast<const __nv_bfloat16*>(dXp), dest, nullptr, T, H, k,
       static_cast<__nv_bfloat16*>(dX), static_cast<const __nv_bfloat16*>(Wr), topk_idx, g, E);
   count_launch();

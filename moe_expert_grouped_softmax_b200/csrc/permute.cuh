@@ -48,11 +48,18 @@ __device__ __forceinline__ float dot8(uint4 a, uint4 b) {
 
 constexpr int kCopyUnroll = 4;
 
+// The gather's register budget allows 3 resident CTAs of 256 threads per SM
+// (measured against 2, the allocation without a minimum: Qwen3-30B-A3B
+// shape 108 -> 106 us per launch, gpt-oss-20b shape unchanged; 4 spills).
+#ifndef MOE_PERMUTE_MINB
+#define MOE_PERMUTE_MINB 3
+#endif
+
 // Xp[dest[t,j]] = (scale ? scale[t,j] : 1) * X[t].  One warp per token: the
 // row is read once into registers (VPL 16-byte vectors per lane in flight per
 // pass, permute_vpl) and written to all k destinations.
 template <int kRowVec>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, MOE_PERMUTE_MINB)
     permute_rows_kernel(const __nv_bfloat16* __restrict__ X,
                         const int32_t* __restrict__ dest,
                         const float* __restrict__ scale, int T, int H, int k,
@@ -173,8 +180,6 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-constexpr int kCombVec = 4;  // 16-byte vectors per lane per source row
-
 // Y[t] = sum_j (w ? w[t,j] : 1) * Yp[dest[t,j]], fp32 in j order -> bf16.
 // With a trained router (Wr != nullptr) the router's part of dX is added
 // before the one rounding: + sum_j g[t,j] * Wr[idx[t,j]] (Wr [E, H] bf16).
@@ -183,8 +188,10 @@ constexpr int kCombVec = 4;  // 16-byte vectors per lane per source row
 // kCombVec vectors per lane are loaded before either is accumulated (the
 // sum stays in j order).  Measured against one row at a time with dest
 // re-read per row: Qwen3-30B-A3B shape (k = 8) 117 -> 103 us, gpt-oss-20b
-// shape unchanged.
-__global__ void __launch_bounds__(256)
+// shape unchanged.  kCombVec 16-byte vectors per lane and source row per
+// pass, kMinB resident CTAs per SM (see combine_vec).
+template <int kCombVec, int kMinB>
+__global__ void __launch_bounds__(256, kMinB)
     unpermute_kernel(const __nv_bfloat16* __restrict__ Yp,
                      const int32_t* __restrict__ dest,
                      const float* __restrict__ w, int T, int H, int k,
@@ -355,5 +362,12 @@ __global__ void __launch_bounds__(256) factor_prep_kernel(const FactorJobs jobs)
     }
   }
 }
+
+// Vectors per lane per pass of the combine for rows of nvec 16-byte vectors:
+// 4 (3 CTAs per SM) when the row is whole 128-vector passes, else 2 (4 CTAs
+// per SM: more rows in flight for the ragged last pass).  Measured, per
+// launch: H = 2880, 51 us with (4, 2 CTAs) -> 45 us with (2, 4); H = 2048,
+// 103 -> 98 us with (4, 3).
+inline int combine_vec(int nvec) { return nvec % 128 == 0 ? 4 : 2; }
 
 }  // namespace moe

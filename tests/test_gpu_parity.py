@@ -65,27 +65,6 @@ def test_route_ties(cuda_ok):
     assert np.abs(w.cpu().double().numpy() - rw).max() <= W_ABS
 
 
-@pytest.mark.parametrize("T,E,k", [(1000, 32, 4), (777, 128, 8), (129, 512, 16)])
-def test_route_both_paths_bit_exact(cuda_ok, T, E, k):
-    """The one-launch router takes a 16-byte-aligned workspace; a workspace 4
-    bytes off that alignment runs the four-kernel path.  Both match the
-    oracle bit for bit."""
-    g = torch.Generator().manual_seed(T + E)
-    L = torch.randn(T, E, generator=g)
-    ridx, _ = O.route_topk(L.numpy(), k)
-    rc, ro, rd = O.permutation(ridx, E)
-    nbytes = ops.route_workspace_bytes(T, E, k)
-    buf = torch.empty(nbytes + 16, dtype=torch.uint8, device=DEV)
-    for off in (0, 4):
-        ws = buf[off:off + nbytes]
-        idx, w, counts, offsets, dest = ops.route_topk(L.to(DEV), k, ws=ws)
-        np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
-        np.testing.assert_array_equal(counts.cpu().numpy(), rc)
-        np.testing.assert_array_equal(offsets.cpu().numpy(), ro)
-        np.testing.assert_array_equal(dest.cpu().numpy(), rd)
-    assert ops.device_status() == 0
-
-
 def test_route_deterministic(cuda_ok):
     L = torch.randn(5000, 64).to(DEV)
     a = [t.clone() for t in ops.route_topk(L, 6)]
