@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe_lora.so")
 SOURCES = ["moe_lora.cu"]
 DEPS = ["ptx.cuh", "route.cuh", "permute.cuh", "gemm.cuh", "gemm_pair.cuh", "lora_grad.cuh",
-        "base_grad.cuh", "router.cuh", "rank_down.cuh",
+        "base_grad.cuh", "base_grad_pair.cuh", "router.cuh", "rank_down.cuh",
         "expert_order.cuh", "ep.cuh"]
 
 NVCC_FLAGS = [

@@ -19,6 +19,7 @@
 #include "gemm_pair.cuh"
 #include "lora_grad.cuh"
 #include "base_grad.cuh"
+#include "base_grad_pair.cuh"
 #include "router.cuh"
 #include "rank_down.cuh"
 #include "ep.cuh"
@@ -454,8 +455,41 @@ moe_status_t launch_base_grad_t(const CUtensorMap* u, const CUtensorMap* v,
   return launch_status();
 }
 
-// dW1 = per-expert dZ1^T Xp, dW2 = dZ2^T h (one launch for both).  The tile
-// width is the one of {256, 192} with the smaller estimated cost
+// The same two problems as 256 x 256 (or 256 x 128) tiles on CTA pairs
+// (measured against the single-CTA kernel: gpt-oss-20b shape 1770 -> 1510 us,
+// Qwen3-30B-A3B shape 1315 -> 1232 us per launch).
+#ifndef MOE_BASE_GRAD_PAIR
+#define MOE_BASE_GRAD_PAIR 1
+#endif
+
+moe_status_t launch_base_grad_pair(const CUtensorMap* u, const CUtensorMap* v,
+                                   BaseGradArgs args, cudaStream_t st) {
+  using C = BaseGradPairCfg;
+  int begin = 0;
+  for (int i = 0; i < 2; ++i) {
+    BaseGradProblem& p = args.prob[i];
+    p.p_tiles = (p.P + 255) / 256;
+    p.q_tiles = (p.Q + 255) / 256;
+    p.tile_begin = begin;
+    begin += p.p_tiles * p.q_tiles;
+  }
+  args.tiles_per_expert = begin;
+  args.total_tiles = args.E * begin;
+  if (cudaFuncSetAttribute(base_grad_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_BYTES) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int pairs = std::min(num_sms() / 2, args.total_tiles);
+  if (pairs <= 0) return MOE_OK;
+  ProfScope prof(MOE_PROF_BASE_GRAD, st);
+  base_grad_pair_kernel<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(u[0], u[1], v[0], v[1],
+                                                                      args);
+  count_launch();
+  return launch_status();
+}
+
+// dW1 = per-expert dZ1^T Xp, dW2 = dZ2^T h (one launch for both).  On CTA
+// pairs where the backward GEMMs run on pairs; otherwise single CTAs with
+// the tile width of {256, 192} with the smaller estimated cost
 // tiles * (BN + 32) over both problems.
 moe_status_t base_grads(const void* dZ1, const void* Xp, const void* dZ2, const void* h,
                         const int32_t* offsets, int E, int H, int I, int R, void* dW1,
@@ -476,6 +510,7 @@ moe_status_t base_grads(const void* dZ1, const void* Xp, const void* dZ2, const 
   g.wait_ns = g_wait_limit_ns;
   g.prob[0].P = P[0]; g.prob[0].Q = Q[0]; g.prob[0].out = static_cast<__nv_bfloat16*>(dW1);
   g.prob[1].P = P[1]; g.prob[1].Q = Q[1]; g.prob[1].out = static_cast<__nv_bfloat16*>(dW2);
+  if (MOE_BASE_GRAD_PAIR && use_pairs(R, E, 2 * I)) return launch_base_grad_pair(tu, tv, g, st);
   double cost[2] = {0, 0};
   const int bns[2] = {256, 192};
   for (int c = 0; c < 2; ++c)
@@ -715,6 +750,17 @@ moe_status_t moe_route_topk_noalloc(const float* logits, int T, int E, int k,
 size_t moe_route_noalloc_max_workspace_bytes(void) { return kRouteScratchBytes; }
 
 // ---------------------------------------------------------- permute / combine
+// The combine (unpermute_kernel), its vector width and register budget
+// chosen from the row length.
+void launch_combine(const __nv_bfloat16* Yp, const int32_t* dest, const float* w, int T, int H,
+                    int k, __nv_bfloat16* Y, const __nv_bfloat16* Wr, const int32_t* idx,
+                    const float* g, int E, cudaStream_t st) {
+  const int warps = 8;
+  const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
+  auto kern = combine_vec(H / 8) == 4 ? unpermute_kernel<4, 3> : unpermute_kernel<2, 4>;
+  kern<<<grid, warps * 32, 0, st>>>(Yp, dest, w, T, H, k, Y, Wr, idx, g, E);
+}
+
 moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale, int T,
                          int H, int k, void* Xp, const void* Zp, float* dw,
                          moe_stream_t stream) {
@@ -727,17 +773,23 @@ moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
        reinterpret_cast<uintptr_t>(Zp)) & 15u)
     return MOE_ERR_INVALID_ARG;
   const int warps = 8;
-  const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
+  const int sms = std::max(1, num_sms());
   ProfScope prof(MOE_PROF_PERMUTE, stream);
   if (dw == nullptr) {
-    const int vpl = permute_vpl(H / 8);
+    const int nvec = H / 8;
+    const int parts = row_parts(T, nvec, sms * MOE_PERMUTE_MINB * warps);
+    const int vpl = permute_vpl((nvec + parts - 1) / parts);
     auto kern = vpl == 4    ? permute_rows_kernel<4>
+                : vpl == 6  ? permute_rows_kernel<6>
                 : vpl == 8  ? permute_rows_kernel<8>
                 : vpl == 12 ? permute_rows_kernel<12>
                             : permute_rows_kernel<16>;
+    const long long units = static_cast<long long>(T) * parts;
+    const int grid = static_cast<int>(std::min<long long>((units + warps - 1) / warps, sms * 8));
     kern<<<grid, warps * 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), dest, scale, T,
-                                          H, k, static_cast<__nv_bfloat16*>(Xp));
+                                          H, k, static_cast<__nv_bfloat16*>(Xp), parts);
   } else {
+    const int grid = std::min((T + warps - 1) / warps, sms * 8);
     permute_kernel<<<grid, warps * 32, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
         static_cast<__nv_bfloat16*>(Xp), static_cast<const __nv_bfloat16*>(Zp), dw);
@@ -754,13 +806,9 @@ moe_status_t moe_unpermute(const void* Yp, const int32_t* dest, const float* w, 
   if (!Yp || !dest || !Y) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(Yp) | reinterpret_cast<uintptr_t>(Y)) & 15u)
     return MOE_ERR_INVALID_ARG;
-  const int warps = 8;
-  const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
   ProfScope prof(MOE_PROF_UNPERMUTE, stream);
-  auto kern = combine_vec(H / 8) == 4 ? unpermute_kernel<4, 3> : unpermute_kernel<2, 4>;
-  kern<<<grid, warps * 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(Yp), dest, w, T, H, k,
-                                        static_cast<__nv_bfloat16*>(Y), nullptr, nullptr,
-                                        nullptr, 0);
+  launch_combine(static_cast<const __nv_bfloat16*>(Yp), dest, w, T, H, k,
+                 static_cast<__nv_bfloat16*>(Y), nullptr, nullptr, nullptr, 0, stream);
   count_launch();
   return launch_status();
 }
@@ -848,12 +896,9 @@ moe_status_t moe_router_bwd(const float* w, const float* dw, const int32_t* topk
       static_cast<const __nv_bfloat16*>(Xp), g_row, expert_offsets, E, H, R, dWr);
   count_launch();
   if ((s = launch_status()) != MOE_OK) return s;
-  const int warps = 8;
-  const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
-  auto kern = combine_vec(H / 8) == 4 ? unpermute_kernel<4, 3> : unpermute_kernel<2, 4>;
-  kern<<<grid, warps * 32, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(dXp), dest, nullptr, T, H, k,
-      static_cast<__nv_bfloat16*>(dX), static_cast<const __nv_bfloat16*>(Wr), topk_idx, g, E);
+  launch_combine(static_cast<const __nv_bfloat16*>(dXp), dest, nullptr, T, H, k,
+                 static_cast<__nv_bfloat16*>(dX), static_cast<const __nv_bfloat16*>(Wr),
+                 topk_idx, g, E, st);
   count_launch();
   return launch_status();
 }

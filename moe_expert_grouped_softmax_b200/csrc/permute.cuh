@@ -55,32 +55,40 @@ constexpr int kCopyUnroll = 4;
 #define MOE_PERMUTE_MINB 3
 #endif
 
-// Xp[dest[t,j]] = (scale ? scale[t,j] : 1) * X[t].  One warp per token: the
-// row is read once into registers (VPL 16-byte vectors per lane in flight per
-// pass, permute_vpl) and written to all k destinations.
+// Xp[dest[t,j]] = (scale ? scale[t,j] : 1) * X[t].  The unit of work is a
+// part of a row (one of `parts` consecutive vector ranges of the row; the
+// host picks parts so that every warp gets several units, which evens out
+// the last round of a launch); one warp per unit, grid-stride: the part is
+// read once into registers (VPL 16-byte vectors per lane in flight per pass,
+// permute_vpl) and written to all k destinations.
 template <int kRowVec>
 __global__ void __launch_bounds__(256, MOE_PERMUTE_MINB)
     permute_rows_kernel(const __nv_bfloat16* __restrict__ X,
                         const int32_t* __restrict__ dest,
                         const float* __restrict__ scale, int T, int H, int k,
-                        __nv_bfloat16* __restrict__ Xp) {
+                        __nv_bfloat16* __restrict__ Xp, int parts) {
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const int nvec = H >> 3;
+  const int nvp = (nvec + parts - 1) / parts;
   const int R = T * k;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+  const long long units = static_cast<long long>(T) * parts;
+  for (long long q = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < units; q += warps) {
+    const int t = static_cast<int>(q / parts);
+    const int part = static_cast<int>(q - static_cast<long long>(t) * parts);
+    const int v_lo = part * nvp, v_hi = min(nvec, v_lo + nvp);
     const char* xrow = reinterpret_cast<const char*>(X + static_cast<size_t>(t) * H);
-    for (int v0 = lane; v0 < nvec; v0 += 32 * kRowVec) {
+    for (int v0 = v_lo + lane; v0 < v_hi; v0 += 32 * kRowVec) {
       uint4 x[kRowVec];
 #pragma unroll
       for (int u = 0; u < kRowVec; ++u) {
         const int v = v0 + 32 * u;
-        if (v < nvec) x[u] = ld_nc_v4(xrow + 16 * static_cast<size_t>(v));
+        if (v < v_hi) x[u] = ld_nc_v4(xrow + 16 * static_cast<size_t>(v));
       }
       for (int j = 0; j < k; ++j) {
         const int d = dest[static_cast<size_t>(t) * k + j];
         if (d < 0 || d >= R) {
-          if (lane == 0 && v0 == lane) set_status(5);
+          if (lane == 0 && v0 == v_lo) set_status(5);
           continue;
         }
         char* orow = reinterpret_cast<char*>(Xp + static_cast<size_t>(d) * H);
@@ -88,7 +96,7 @@ __global__ void __launch_bounds__(256, MOE_PERMUTE_MINB)
 #pragma unroll
         for (int u = 0; u < kRowVec; ++u) {
           const int v = v0 + 32 * u;
-          if (v < nvec) {
+          if (v < v_hi) {
             uint4 y = x[u];
             if (scale) {
               y.x = scale2(y.x, c);
@@ -104,14 +112,29 @@ __global__ void __launch_bounds__(256, MOE_PERMUTE_MINB)
   }
 }
 
-// Vectors per lane per pass of permute_rows_kernel for rows of nvec 16-byte
-// vectors: enough for a whole row in one pass up to 512 vectors (H = 4096),
-// in multiples of 4 (fewest idle lane slots: H = 2880 takes 12, one pass
-// with 94% of the slots used, where 8 took two passes at 70%).
-inline int permute_vpl(int nvec) {
-  const int per_lane = (nvec + 31) / 32;
-  const int v = (per_lane + 3) / 4 * 4;
-  return v < 4 ? 4 : (v > 16 ? 16 : v);
+// Vectors per lane per pass of permute_rows_kernel for row parts of nvp
+// 16-byte vectors: enough for a whole part in one pass up to 512 vectors
+// (H = 4096), one of 4, 6, 8, 12, 16 (fewest idle lane slots: 360 vectors,
+// H = 2880, take 12, one pass with 94% of the slots used, where 8 took two
+// passes at 70%; half of that row takes 6).
+inline int permute_vpl(int nvp) {
+  const int per_lane = (nvp + 31) / 32;
+  return per_lane <= 4 ? 4 : per_lane <= 6 ? 6 : per_lane <= 8 ? 8 : per_lane <= 12 ? 12 : 16;
+}
+
+#ifndef MOE_ROW_PARTS_MAX
+#define MOE_ROW_PARTS_MAX 2
+#endif
+// Parts per row for the gather: enough that each of the `warps` resident
+// warps gets about four units (T tokens in all), at most MOE_ROW_PARTS_MAX,
+// and no part under 128 vectors (measured, gpt-oss-20b shape: 2 parts, 52 ->
+// 48 us per launch; the last round of whole rows left SMs idle).
+inline int row_parts(int T, int nvec, int warps) {
+  int p = 1;
+  while (p < MOE_ROW_PARTS_MAX && static_cast<long long>(T) * p < 4ll * warps &&
+         nvec / (p + 1) >= 128)
+    ++p;
+  return p;
 }
 
 // Same with the routing-weight gradient dw[t,j] = <X[t], Zp[dest[t,j]]>.
@@ -183,10 +206,11 @@ __global__ void __launch_bounds__(256)
 // Y[t] = sum_j (w ? w[t,j] : 1) * Yp[dest[t,j]], fp32 in j order -> bf16.
 // With a trained router (Wr != nullptr) the router's part of dX is added
 // before the one rounding: + sum_j g[t,j] * Wr[idx[t,j]] (Wr [E, H] bf16).
-// One warp per token.  The token's destination rows and weights are read
-// once (lane j holds slot j, broadcast by shuffle) and two source rows'
-// kCombVec vectors per lane are loaded before either is accumulated (the
-// sum stays in j order).  Measured against one row at a time with dest
+// One warp per token (splitting rows into parts as the gather does
+// measured no faster here).  The token's destination rows and weights are
+// read once (lane j holds slot j, broadcast by shuffle) and two source rows'
+// kCombVec vectors per lane are loaded before either is accumulated (the sum
+// stays in j order).  Measured against one row at a time with dest
 // re-read per row: Qwen3-30B-A3B shape (k = 8) 117 -> 103 us, gpt-oss-20b
 // shape unchanged.  kCombVec 16-byte vectors per lane and source row per
 // pass, kMinB resident CTAs per SM (see combine_vec).
@@ -213,6 +237,7 @@ __global__ void __launch_bounds__(256, kMinB)
     a[6] = fmaf(c, bf16_lo(z.w), a[6]);
     a[7] = fmaf(c, bf16_hi(z.w), a[7]);
   };
+  const int v_lo = 0, v_hi = nvec;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     char* yrow = reinterpret_cast<char*>(Y + static_cast<size_t>(t) * H);
     // slots j0 .. j0 + 31 of the token on lanes 0 .. 31 (k <= 32 in one go)
@@ -226,7 +251,10 @@ __global__ void __launch_bounds__(256, kMinB)
         my_d = -1;
       }
     }
-    for (int v0 = lane; v0 < nvec; v0 += 32 * kCombVec) {
+    // the pass loop's trip count is the same on every lane (the shuffles
+    // below need the whole warp); vectors past v_hi are masked
+    for (int base = v_lo; base < v_hi; base += 32 * kCombVec) {
+      const int v0 = base + lane;
       float acc[kCombVec][8];
 #pragma unroll
       for (int u = 0; u < kCombVec; ++u)
@@ -242,7 +270,7 @@ __global__ void __launch_bounds__(256, kMinB)
             dj = dest[static_cast<size_t>(t) * k + j0 + lane];
             if (w) cj = w[static_cast<size_t>(t) * k + j0 + lane];
             if (dj < 0 || dj >= R) {
-              if (v0 == lane) set_status(5);
+              if (base == v_lo) set_status(5);
               dj = -1;
             }
           }
@@ -259,10 +287,10 @@ __global__ void __launch_bounds__(256, kMinB)
           for (int u = 0; u < kCombVec; ++u) {
             const int v = v0 + 32 * u;
             za[u] = zb[u] = make_uint4(0, 0, 0, 0);
-            if (v < nvec && da >= 0)
+            if (v < v_hi && da >= 0)
               za[u] = ld_nc_v4(reinterpret_cast<const char*>(Yp + static_cast<size_t>(da) * H) +
                                16 * static_cast<size_t>(v));
-            if (v < nvec && has_b && db >= 0)
+            if (v < v_hi && has_b && db >= 0)
               zb[u] = ld_nc_v4(reinterpret_cast<const char*>(Yp + static_cast<size_t>(db) * H) +
                                16 * static_cast<size_t>(v));
           }
@@ -285,7 +313,7 @@ __global__ void __launch_bounds__(256, kMinB)
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u) {
             const int v = v0 + 32 * u;
-            if (v < nvec)
+            if (v < v_hi)
               fma8(acc[u], c, *reinterpret_cast<const uint4*>(wrow + 16 * static_cast<size_t>(v)));
           }
         }
@@ -293,7 +321,7 @@ __global__ void __launch_bounds__(256, kMinB)
 #pragma unroll
       for (int u = 0; u < kCombVec; ++u) {
         const int v = v0 + 32 * u;
-        if (v < nvec) {
+        if (v < v_hi) {
           uint4 o;
           o.x = pack_bf16x2(acc[u][0], acc[u][1]);
           o.y = pack_bf16x2(acc[u][2], acc[u][3]);

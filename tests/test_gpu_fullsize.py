@@ -38,9 +38,17 @@ def run(request, cuda_ok):
     W = [inp[n].to(dev) for n in NAMES]
     full_ft = request.param in FULL_FT
     blk = ops.MoeBlock(T, H, I, E, k, r, s, device=dev, full_ft=full_ft)
-    blk.step(inp["X"].to(dev), inp["logits"].to(dev), inp["dY"].to(dev), W)
+    Xd, dYd = inp["X"].to(dev), inp["dY"].to(dev)
+    blk.step(Xd, inp["logits"].to(dev), dYd, W)
     torch.cuda.synchronize()
     status = ops.device_status()
+    # the gather and the weighted dY gather are exact copies / one rounding:
+    # every routed row, compared on the device
+    dflat = blk.dest.long().flatten()
+    xp_exact = torch.equal(blk.Xp[dflat], Xd.repeat_interleave(k, dim=0))
+    dz2_ref = (dYd.float().repeat_interleave(k, dim=0) * blk.w.flatten()[:, None]).to(torch.bfloat16)
+    dz2_exact = torch.equal(blk.dZ2[dflat], dz2_ref)
+    del dflat, dz2_ref, Xd, dYd
     names = ["idx", "w", "counts", "offsets", "dest", "Y", "dX", "Z2",
              "dA1", "dB1", "dA2", "dB2"] + (["dW1", "dW2"] if full_ft else [])
     got = {n: getattr(blk, n).cpu() for n in names}
@@ -50,11 +58,19 @@ def run(request, cuda_ok):
     ridx, rw = O.route_topk(inp["logits"].numpy(), k)
     rc, ro, rd = O.permutation(ridx, E)
     yield dict(cfg=cfg, inp=inp, got=got, status=status, ridx=ridx, rw=rw, rc=rc,
-               ro=ro, rd=rd)
+               ro=ro, rd=rd, xp_exact=xp_exact, dz2_exact=dz2_exact)
 
 
 def test_status(run):
     assert run["status"] == 0
+
+
+def test_gathers_exact_full(run):
+    """Xp[dest[t, j]] == X[t] and dZ2[dest[t, j]] == bf16(w[t, j] dY[t]) for
+    every routed row of the full-size step (the launch configuration the
+    benchmark times, row parts included)."""
+    assert run["xp_exact"]
+    assert run["dz2_exact"]
 
 
 def test_routing_full(run):

@@ -109,6 +109,33 @@ def test_permute_and_combine(cuda_ok):
     assert ops.device_status() == 0
 
 
+@pytest.mark.parametrize("H", [2048, 2880, 4104])
+def test_permute_and_combine_row_parts(cuda_ok, H):
+    """Few tokens and long rows: the gather splits each row into parts (one
+    warp per part); results are those of whole rows.  H = 4104 (513 vectors)
+    gives the combine a last pass that only some lanes' vectors reach, while
+    its shuffles still need the whole warp."""
+    T, E, k = 333, 16, 4
+    g = torch.Generator().manual_seed(H)
+    X = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    L = torch.randn(T, E, generator=g)
+    Z = torch.randn(T * k, H, generator=g).to(torch.bfloat16)
+    dY = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    idx, w, counts, offsets, dest = ops.route_topk(L.to(DEV), k)
+    rdest = dest.cpu().numpy()
+    rw = w.cpu().double().numpy()
+    Xp = ops.permute(X.to(DEV), dest)
+    np.testing.assert_array_equal(f32(Xp), O.permute(f32(X), rdest).astype(np.float32))
+    Sg = ops.permute(dY.to(DEV), dest, scale=w)
+    ref = (dY.float().repeat_interleave(k, 0) * w.cpu().flatten()[:, None]).to(torch.bfloat16)
+    assert torch.equal(Sg.cpu()[torch.as_tensor(rdest.reshape(-1), dtype=torch.long)], ref)
+    assert_bf16_close(ops.unpermute(Z.to(DEV), dest, w), O.unpermute(f32(Z), rdest, rw),
+                      "combine")
+    assert_bf16_close(ops.unpermute(Z.to(DEV), dest, None), O.unpermute(f32(Z), rdest, None),
+                      "combine w=1")
+    assert ops.device_status() == 0
+
+
 # ------------------------------------------------------------------ expert MLP + block
 BLOCK_CASES = {
     "tiny": S.make_config("tiny"),
