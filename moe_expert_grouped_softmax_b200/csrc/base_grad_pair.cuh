@@ -265,7 +265,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BaseGradPairCfg::THR
       });
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead(&acc_empty[bb]));
+      // the accumulator's TMEM reads have completed (tcgen05.wait::ld); the
+      // release needs no ordering of the output stores
+      if (lane == 0) MOE_ACC_RELEASE(lead(&acc_empty[bb]));
     }
   }
 

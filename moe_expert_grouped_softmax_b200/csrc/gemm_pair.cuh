@@ -666,7 +666,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead(&acc_empty[b]));
+      // the accumulator's TMEM reads have completed (tcgen05.wait::ld); the
+      // release needs no ordering of the output stores
+      if (lane == 0) MOE_ACC_RELEASE(lead(&acc_empty[b]));
     }
     if constexpr (C::kRing) ring.finish(lane);  // every staged store has left shared memory
   }

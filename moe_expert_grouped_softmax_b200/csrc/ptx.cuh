@@ -127,6 +127,25 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Arrive (relaxed, cluster scope) on an mbarrier given by its cluster
+// address: for hand-offs whose only ordering need is already met by a
+// completed wait (e.g. a TMEM accumulator released after tcgen05.wait::ld),
+// so that the arrive does not wait for this thread's earlier global stores.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   cluster_addr)
+               : "memory");
+}
+
+#ifndef MOE_ACC_RELAXED
+#define MOE_ACC_RELAXED 1
+#endif
+#if MOE_ACC_RELAXED
+#define MOE_ACC_RELEASE mbar_arrive_cluster_relaxed
+#else
+#define MOE_ACC_RELEASE mbar_arrive_cluster
+#endif
+
 // True on one lane of the (converged) warp: the tensor-core issue of a role
 // that the whole warp runs, so that its loop state stays warp-uniform.
 __device__ __forceinline__ bool elect_one() {
