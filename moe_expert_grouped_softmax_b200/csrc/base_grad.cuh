@@ -71,6 +71,7 @@ __global__ void __launch_bounds__(192, 1)
                      const __grid_constant__ CUtensorMap tmV0,
                      const __grid_constant__ CUtensorMap tmV1,
                      const __grid_constant__ BaseGradArgs args) {
+  griddep_sync();  // before any global memory access
   using C = BaseGradCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(

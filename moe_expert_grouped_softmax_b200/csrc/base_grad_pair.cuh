@@ -105,6 +105,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BaseGradPairCfg::THR
     tmem_alloc_pair(s_tmem, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  // everything above touches only shared memory, TMEM and the kernel's
+  // parameters; the preceding kernel's outputs are read from here on
+  griddep_sync();
   if (warp == 2) {
     bool bad = false;
     for (int e = lane; e <= args.E; e += 32) {

@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(kRegroupThreads)
     ep_regroup_kernel(const __nv_bfloat16* __restrict__ in, const int32_t* __restrict__ counts,
                       int N, int EL, int rows, int H, int dir,
                       __nv_bfloat16* __restrict__ out, int32_t* __restrict__ offsets) {
+  griddep_sync();  // before any global memory access
   extern __shared__ int sm_rg[];
   const int nseg = N * EL;
   int* s_src = sm_rg;              // [nseg + 1]: segment (s, e) start, source-major

@@ -469,6 +469,7 @@ __global__ void __launch_bounds__(gemm_threads(MODE), 1)
                              const __grid_constant__ CUtensorMap tmLA,
                              const __grid_constant__ CUtensorMap tmLB,
                              const GemmArgs args) {
+  griddep_sync();  // before any global memory access
   using C = GemmCfg<MODE, BN, RK>;
   constexpr bool kSwiGLU = (MODE == kGateUpFwd);
   constexpr bool kBMN = C::kBMN;

@@ -429,6 +429,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
     tmem_alloc_pair(s_tmem, C::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  // everything above touches only shared memory, TMEM and the kernel's
+  // parameters; the preceding kernel's outputs are read from here on
+  griddep_sync();
   if (warp == 2) build_tile_table(args.offsets, E, args.R, s_off, s_mstart, lane, 8);
   tc_fence_before();
   cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated

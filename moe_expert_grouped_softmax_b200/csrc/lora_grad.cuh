@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(192, 1)
                      const __grid_constant__ CUtensorMap tmV2,
                      const __grid_constant__ CUtensorMap tmV3,
                      const GradArgs args) {
+  griddep_sync();  // before any global memory access
   using C = GradCfg<RK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <utility>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -68,6 +69,30 @@ bool use_pairs(int R, int E, int K) {
   if (g_cta_pairs >= 0) return g_cta_pairs > 0;
   return static_cast<int64_t>(R) >= static_cast<int64_t>(kPairMinRowsPerExpert) * E &&
          K >= kPairMinK;
+}
+
+// Launches a kernel on `st`; with MOE_PDL the launch allows programmatic
+// dependent launch (the kernel's griddep_sync waits for the preceding kernel
+// of the stream before touching global memory, and lets the next one launch
+// while this one's CTAs finish).  Errors are left for launch_status().
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+              Args&&... args) {
+#if MOE_PDL
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+#else
+  kern<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
+#endif
 }
 
 // ------------------------------------------------ optional per-kernel timing
@@ -212,7 +237,7 @@ moe_status_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b,
   ProfScope prof(MODE == kGateUpFwd ? MOE_PROF_GATE_UP_FWD
                  : MODE == kDownFwd ? MOE_PROF_DOWN_FWD
                  : MODE == kDownBwd ? MOE_PROF_DOWN_BWD : MOE_PROF_GATE_UP_BWD, st);
-  kern<<<grid, gemm_threads(MODE), C::SMEM_BYTES, st>>>(a, b, la, lb, args);
+  launch_k(kern, grid, gemm_threads(MODE), C::SMEM_BYTES, st, a, b, la, lb, args);
   count_launch();
   return launch_status();
 }
@@ -297,7 +322,7 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* XA, const v
                  : MODE == kDownBwd   ? MOE_PROF_DOWN_BWD
                                       : MOE_PROF_GATE_UP_BWD,
                  st);
-  kern<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tw, txa, tlb, to, to2, to3, args);
+  launch_k(kern, 2 * pairs, C::THREADS, C::SMEM_BYTES, st, ta, tw, txa, tlb, to, to2, to3, args);
   count_launch();
   return launch_status();
 }
@@ -334,7 +359,7 @@ moe_status_t launch_grad_t(const CUtensorMap* u, const CUtensorMap* v,
   const int grid = std::min(num_sms(), args.total_tiles);
   if (grid <= 0) return MOE_OK;
   ProfScope prof(MOE_PROF_LORA_GRAD, st);
-  kern<<<grid, 192, C::SMEM_BYTES, st>>>(u[0], u[1], u[2], u[3], v[0], v[1], v[2],
+  launch_k(kern, grid, 192, C::SMEM_BYTES, st, u[0], u[1], u[2], u[3], v[0], v[1], v[2],
                                          v[3], args);
   count_launch();
   return launch_status();
@@ -423,7 +448,7 @@ struct FactorPrep {
   moe_status_t launch(cudaStream_t st) {
     if (total == 0) return MOE_OK;
     ProfScope prof(MOE_PROF_TRANSPOSE, st);
-    factor_prep_kernel<<<total, 256, 0, st>>>(jobs);
+    launch_k(factor_prep_kernel, total, 256, 0, st, jobs);
     count_launch();
     return launch_status();
   }
@@ -450,7 +475,7 @@ moe_status_t launch_base_grad_t(const CUtensorMap* u, const CUtensorMap* v,
   const int grid = std::min(num_sms(), args.total_tiles);
   if (grid <= 0) return MOE_OK;
   ProfScope prof(MOE_PROF_BASE_GRAD, st);
-  kern<<<grid, 192, C::SMEM_BYTES, st>>>(u[0], u[1], v[0], v[1], args);
+  launch_k(kern, grid, 192, C::SMEM_BYTES, st, u[0], u[1], v[0], v[1], args);
   count_launch();
   return launch_status();
 }
@@ -481,7 +506,7 @@ moe_status_t launch_base_grad_pair(const CUtensorMap* u, const CUtensorMap* v,
   const int pairs = std::min(num_sms() / 2, args.total_tiles);
   if (pairs <= 0) return MOE_OK;
   ProfScope prof(MOE_PROF_BASE_GRAD, st);
-  base_grad_pair_kernel<<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(u[0], u[1], v[0], v[1],
+  launch_k(base_grad_pair_kernel, 2 * pairs, C::THREADS, C::SMEM_BYTES, st, u[0], u[1], v[0], v[1],
                                                                       args);
   count_launch();
   return launch_status();
@@ -535,7 +560,7 @@ moe_status_t launch_router_logits_t(const void* X, const void* Wr, int T, int H,
     return MOE_ERR_CUDA;
   dim3 grid((T + 127) / 128, (E + BN - 1) / BN);
   ProfScope prof(MOE_PROF_ROUTER_FWD, st);
-  kern<<<grid, 192, C::SMEM_BYTES, st>>>(tx, tw, T, H, E, logits, g_wait_limit_ns);
+  launch_k(kern, grid, 192, C::SMEM_BYTES, st, tx, tw, T, H, E, logits, g_wait_limit_ns);
   count_launch();
   return launch_status();
 }
@@ -568,7 +593,7 @@ moe_status_t launch_rank_down_t(const void* U, const void* F, int K, const int32
       std::min<long long>(static_cast<long long>(num_sms()) * C::CTAS_PER_SM, R / 128 + E));
   if (grid <= 0) return MOE_OK;
   ProfScope prof(MOE_PROF_RANK_DOWN, st);
-  kern<<<grid, 192, C::SMEM_BYTES, st>>>(tu, tf, a);
+  launch_k(kern, grid, 192, C::SMEM_BYTES, st, tu, tf, a);
   count_launch();
   return launch_status();
 }
@@ -701,7 +726,7 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem1)) != cudaSuccess)
       return MOE_ERR_CUDA;
-    kern<<<grid1, kRouteWarps * 32, smem1, st>>>(logits, T, E, k, topk_idx, topk_w);
+    launch_k(kern, grid1, kRouteWarps * 32, smem1, st, logits, T, E, k, topk_idx, topk_w);
     count_launch();
     return launch_status();
   };
@@ -713,20 +738,20 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
   else s = launch(route_topk_kernel<16>);
   if (s != MOE_OK) return s;
   // 2. stable in-chunk ranks + chunk histograms
-  route_rank_kernel<<<nblk, kRankWarps * 32, static_cast<size_t>(kRankWarps) * E * 4, st>>>(
+  launch_k(route_rank_kernel, nblk, kRankWarps * 32, static_cast<size_t>(kRankWarps) * E * 4, st, 
       topk_idx, R, E, blk_hist, local_rank);
   count_launch();
   if ((s = launch_status()) != MOE_OK) return s;
   // 3. expert totals, offsets and per-chunk base rows (one CTA)
   const int P = std::max(1, 1024 / E);
   const size_t smem2 = (static_cast<size_t>(P) * E + E + 1) * 4;
-  route_scan_kernel<<<1, 1024, smem2, st>>>(blk_hist, nblk, E, R, expert_counts,
+  launch_k(route_scan_kernel, 1, 1024, smem2, st, blk_hist, nblk, E, R, expert_counts,
                                             expert_offsets);
   count_launch();
   if ((s = launch_status()) != MOE_OK) return s;
   // 4. destination rows
   const int grid = std::min((R + 255) / 256, std::max(1, num_sms()) * 8);
-  route_dest_kernel<<<grid, 256, 0, st>>>(topk_idx, blk_hist, local_rank, R, E, dest);
+  launch_k(route_dest_kernel, grid, 256, 0, st, topk_idx, blk_hist, local_rank, R, E, dest);
   count_launch();
   return launch_status();
 }
@@ -758,7 +783,7 @@ void launch_combine(const __nv_bfloat16* Yp, const int32_t* dest, const float* w
   const int warps = 8;
   const int grid = std::min((T + warps - 1) / warps, std::max(1, num_sms()) * 8);
   auto kern = combine_vec(H / 8) == 4 ? unpermute_kernel<4, 3> : unpermute_kernel<2, 4>;
-  kern<<<grid, warps * 32, 0, st>>>(Yp, dest, w, T, H, k, Y, Wr, idx, g, E);
+  launch_k(kern, grid, warps * 32, 0, st, Yp, dest, w, T, H, k, Y, Wr, idx, g, E);
 }
 
 moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale, int T,
@@ -786,11 +811,11 @@ moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
                             : permute_rows_kernel<16>;
     const long long units = static_cast<long long>(T) * parts;
     const int grid = static_cast<int>(std::min<long long>((units + warps - 1) / warps, sms * 8));
-    kern<<<grid, warps * 32, 0, stream>>>(static_cast<const __nv_bfloat16*>(X), dest, scale, T,
+    launch_k(kern, grid, warps * 32, 0, stream, static_cast<const __nv_bfloat16*>(X), dest, scale, T,
                                           H, k, static_cast<__nv_bfloat16*>(Xp), parts);
   } else {
     const int grid = std::min((T + warps - 1) / warps, sms * 8);
-    permute_kernel<<<grid, warps * 32, 0, stream>>>(
+    launch_k(permute_kernel, grid, warps * 32, 0, stream, 
         static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
         static_cast<__nv_bfloat16*>(Xp), static_cast<const __nv_bfloat16*>(Zp), dw);
   }
@@ -836,7 +861,7 @@ moe_status_t moe_ep_regroup(const void* in, const int32_t* counts, int N, int E_
   const int warps = kRegroupThreads / 32;
   const int grid =
       std::max(1, std::min((rows + warps - 1) / warps, std::max(1, num_sms()) * 8));
-  ep_regroup_kernel<<<grid, kRegroupThreads, smem, st>>>(
+  launch_k(ep_regroup_kernel, grid, kRegroupThreads, smem, st, 
       static_cast<const __nv_bfloat16*>(in), counts, N, E_loc, rows, H, dir,
       static_cast<__nv_bfloat16*>(out), offsets);
   count_launch();
@@ -888,11 +913,11 @@ moe_status_t moe_router_bwd(const float* w, const float* dw, const int32_t* topk
   float* g_row = at<float>(ws, align256(static_cast<size_t>(R) * 4));
   ProfScope prof(MOE_PROF_ROUTER_BWD, st);
   const int grid0 = std::min((T + 255) / 256, std::max(1, num_sms()) * 4);
-  router_dlogit_kernel<<<grid0, 256, 0, st>>>(w, dw, dest, T, k, g, g_row);
+  launch_k(router_dlogit_kernel, grid0, 256, 0, st, w, dw, dest, T, k, g, g_row);
   count_launch();
   moe_status_t s;
   if ((s = launch_status()) != MOE_OK) return s;
-  router_wgrad_kernel<<<dim3(E, (H + kRouterWCols - 1) / kRouterWCols), 256, 0, st>>>(
+  launch_k(router_wgrad_kernel, dim3(E, (H + kRouterWCols - 1) / kRouterWCols), 256, 0, st, 
       static_cast<const __nv_bfloat16*>(Xp), g_row, expert_offsets, E, H, R, dWr);
   count_launch();
   if ((s = launch_status()) != MOE_OK) return s;

@@ -6,6 +6,14 @@
 
 #include "ptx.cuh"
 
+// L2 cache hints: evict-first on the gather's stores / the combine's loads.
+#ifndef MOE_GATHER_STORE_HINT
+#define MOE_GATHER_STORE_HINT 0
+#endif
+#ifndef MOE_COMBINE_LOAD_HINT
+#define MOE_COMBINE_LOAD_HINT 0
+#endif
+
 namespace moe {
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -15,6 +23,20 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
                : "l"(p));
   return v;
 }
+
+// 16-byte read-only load with an L2 cache policy.
+__device__ __forceinline__ uint4 ld_nc_v4_hint(const void* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+#if MOE_COMBINE_LOAD_HINT
+#define COMB_LD(p) ld_nc_v4_hint(p, pol_ld)
+#else
+#define COMB_LD(p) ld_nc_v4(p)
+#endif
 
 __device__ __forceinline__ uint4 ld_v4(const void* p) {
   uint4 v;
@@ -67,12 +89,16 @@ __global__ void __launch_bounds__(256, MOE_PERMUTE_MINB)
                         const int32_t* __restrict__ dest,
                         const float* __restrict__ scale, int T, int H, int k,
                         __nv_bfloat16* __restrict__ Xp, int parts) {
+  griddep_sync();  // before any global memory access
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const int nvec = H >> 3;
   const int nvp = (nvec + parts - 1) / parts;
   const int R = T * k;
   const long long units = static_cast<long long>(T) * parts;
+#if MOE_GATHER_STORE_HINT
+  const uint64_t pol = policy_evict_first();
+#endif
   for (long long q = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < units; q += warps) {
     const int t = static_cast<int>(q / parts);
     const int part = static_cast<int>(q - static_cast<long long>(t) * parts);
@@ -104,7 +130,11 @@ __global__ void __launch_bounds__(256, MOE_PERMUTE_MINB)
               y.z = scale2(y.z, c);
               y.w = scale2(y.w, c);
             }
+#if MOE_GATHER_STORE_HINT
+            st_global_v4_hint(orow + 16 * static_cast<size_t>(v), y, pol);
+#else
             st_v4(orow + 16 * static_cast<size_t>(v), y);
+#endif
           }
         }
       }
@@ -146,6 +176,7 @@ __global__ void __launch_bounds__(256)
                    __nv_bfloat16* __restrict__ Xp,
                    const __nv_bfloat16* __restrict__ Zp,
                    float* __restrict__ dw) {
+  griddep_sync();  // before any global memory access
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const int nvec = H >> 3;
@@ -223,6 +254,7 @@ __global__ void __launch_bounds__(256, kMinB)
                      const __nv_bfloat16* __restrict__ Wr = nullptr,
                      const int32_t* __restrict__ idx = nullptr,
                      const float* __restrict__ g = nullptr, int E = 0) {
+  griddep_sync();  // before any global memory access
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const int nvec = H >> 3;
@@ -238,6 +270,9 @@ __global__ void __launch_bounds__(256, kMinB)
     a[7] = fmaf(c, bf16_hi(z.w), a[7]);
   };
   const int v_lo = 0, v_hi = nvec;
+#if MOE_COMBINE_LOAD_HINT
+  const uint64_t pol_ld = policy_evict_first();
+#endif
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     char* yrow = reinterpret_cast<char*>(Y + static_cast<size_t>(t) * H);
     // slots j0 .. j0 + 31 of the token on lanes 0 .. 31 (k <= 32 in one go)
@@ -288,11 +323,11 @@ __global__ void __launch_bounds__(256, kMinB)
             const int v = v0 + 32 * u;
             za[u] = zb[u] = make_uint4(0, 0, 0, 0);
             if (v < v_hi && da >= 0)
-              za[u] = ld_nc_v4(reinterpret_cast<const char*>(Yp + static_cast<size_t>(da) * H) +
-                               16 * static_cast<size_t>(v));
+              za[u] = COMB_LD(reinterpret_cast<const char*>(Yp + static_cast<size_t>(da) * H) +
+                              16 * static_cast<size_t>(v));
             if (v < v_hi && has_b && db >= 0)
-              zb[u] = ld_nc_v4(reinterpret_cast<const char*>(Yp + static_cast<size_t>(db) * H) +
-                               16 * static_cast<size_t>(v));
+              zb[u] = COMB_LD(reinterpret_cast<const char*>(Yp + static_cast<size_t>(db) * H) +
+                              16 * static_cast<size_t>(v));
           }
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u) {
@@ -354,6 +389,7 @@ struct FactorJobs {
 };
 
 __global__ void __launch_bounds__(256) factor_prep_kernel(const FactorJobs jobs) {
+  griddep_sync();  // before any global memory access
   int b = blockIdx.x, ji = 0;
   while (ji < jobs.n && b >= jobs.job[ji].blocks) {
     b -= jobs.job[ji].blocks;

@@ -18,6 +18,22 @@ __device__ __forceinline__ void set_status(int code) {
   atomicCAS(&g_status, 0, code);
 }
 
+// Programmatic dependent launch.  Built with MOE_PDL, every kernel is
+// launched with programmatic stream serialisation and calls this before its
+// first access to global memory: it waits until the preceding kernel of the
+// stream has completed and its writes are visible, then lets the next kernel
+// of the stream launch (its CTAs take SMs as this kernel's CTAs leave and
+// wait here in turn).  Without the launch attribute it returns at once.
+#ifndef MOE_PDL
+#define MOE_PDL 0
+#endif
+__device__ __forceinline__ void griddep_sync() {
+#if MOE_PDL
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

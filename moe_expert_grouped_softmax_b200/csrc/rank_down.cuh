@@ -55,6 +55,7 @@ template <int RK, bool KMAJ_F>
 __global__ void __launch_bounds__(192, RankDownCfg<RK, KMAJ_F>::CTAS_PER_SM)
     rank_down_kernel(const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmF, const RankDownArgs args) {
+  griddep_sync();  // before any global memory access
   using C = RankDownCfg<RK, KMAJ_F>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(

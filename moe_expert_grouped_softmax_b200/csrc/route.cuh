@@ -28,6 +28,7 @@ template <int EPL>
 __global__ void __launch_bounds__(kRouteWarps * 32)
     route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                       int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  griddep_sync();  // before any global memory access
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   extern __shared__ float s_val_all[];
   float* my_val = s_val_all + warp * k;
@@ -92,6 +93,7 @@ __global__ void __launch_bounds__(kRankWarps * 32)
     route_rank_kernel(const int32_t* __restrict__ idx, int R, int E,
                       int32_t* __restrict__ blk_hist,
                       int32_t* __restrict__ local_rank) {
+  griddep_sync();  // before any global memory access
   extern __shared__ int s_cnt[];  // [kRankWarps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kRankWarps * E; i += blockDim.x) s_cnt[i] = 0;
@@ -142,6 +144,7 @@ __global__ void __launch_bounds__(1024)
     route_scan_kernel(int32_t* __restrict__ blk_hist, int nblk, int E, int R,
                       int32_t* __restrict__ counts,
                       int32_t* __restrict__ offsets) {
+  griddep_sync();  // before any global memory access
   extern __shared__ int smem_i[];
   const int P = max(1, static_cast<int>(blockDim.x) / E);
   int* s_part = smem_i;              // [P][E]
@@ -204,6 +207,7 @@ __global__ void route_dest_kernel(const int32_t* __restrict__ idx,
                                   const int32_t* __restrict__ blk_base,
                                   const int32_t* __restrict__ local_rank,
                                   int R, int E, int32_t* __restrict__ dest) {
+  griddep_sync();  // before any global memory access
   for (int f = blockIdx.x * blockDim.x + threadIdx.x; f < R;
        f += gridDim.x * blockDim.x) {
     const int b = f / kRankChunk;

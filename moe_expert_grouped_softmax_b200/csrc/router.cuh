@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(192, 1)
     router_logits_kernel(const __grid_constant__ CUtensorMap tmX,
                          const __grid_constant__ CUtensorMap tmW, int T, int H, int E,
                          float* __restrict__ logits, uint64_t wait_ns) {
+  griddep_sync();  // before any global memory access
   using C = RouterCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -164,6 +165,7 @@ __global__ void __launch_bounds__(192, 1)
 __global__ void router_dlogit_kernel(const float* __restrict__ w, const float* __restrict__ dw,
                                      const int32_t* __restrict__ dest, int T, int k,
                                      float* __restrict__ g, float* __restrict__ g_row) {
+  griddep_sync();  // before any global memory access
   const int R = T * k;
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
     const size_t b = static_cast<size_t>(t) * k;
@@ -193,6 +195,7 @@ __global__ void __launch_bounds__(256)
     router_wgrad_kernel(const __nv_bfloat16* __restrict__ Xp, const float* __restrict__ g_row,
                         const int32_t* __restrict__ offsets, int E, int H, int R,
                         float* __restrict__ dWr) {
+  griddep_sync();  // before any global memory access
   __shared__ float part[8][kRouterWCols];
   const int e = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
