@@ -314,36 +314,50 @@ def run_ours(args, cfg):
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
         comp = torch.cuda.current_stream()
         ev = {n: [torch.cuda.Event() for _ in range(2)]
-              for n in ("in_ready", "in_free", "done", "out_free")}
+              for n in ("fwd_in", "bwd_in", "fwd_done", "in_free", "done", "out_free")}
 
         def run_e2e(nsteps):
+            # per block b (two, alternating steps): X and logits upload -> forward;
+            # dY upload (overlapping the forward) -> backward; Y download
+            # (overlapping the backward), then dX and the gradients
             for i in range(nsteps):
                 b = i & 1
                 with torch.cuda.stream(s_in):
                     if i >= 2:
                         s_in.wait_event(ev["in_free"][b])
-                    for d, h in zip(din[b], hin[b]):
-                        d.copy_(h, non_blocking=True)
-                    ev["in_ready"][b].record(s_in)
-                comp.wait_event(ev["in_ready"][b])
+                    din[b][0].copy_(hin[b][0], non_blocking=True)
+                    din[b][1].copy_(hin[b][1], non_blocking=True)
+                    ev["fwd_in"][b].record(s_in)
+                    din[b][2].copy_(hin[b][2], non_blocking=True)
+                    ev["bwd_in"][b].record(s_in)
+                comp.wait_event(ev["fwd_in"][b])
                 if i >= 2:
                     comp.wait_event(ev["out_free"][b])
                 if use_graph:
-                    blocks[b].replay()
+                    blocks[b].replay_forward()
                 else:
-                    blocks[b].step(din[b][0], din[b][1], din[b][2], W, Wr)
+                    blocks[b].forward(din[b][0], din[b][1], W, Wr)
+                ev["fwd_done"][b].record(comp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev["fwd_done"][b])
+                    hout[b][0].copy_(outs(blocks[b])[0], non_blocking=True)
+                comp.wait_event(ev["bwd_in"][b])
+                if use_graph:
+                    blocks[b].replay_backward()
+                else:
+                    blocks[b].backward(din[b][2], W, Wr)
                 ev["in_free"][b].record(comp)
                 ev["done"][b].record(comp)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(ev["done"][b])
-                    for o, h in zip(outs(blocks[b]), hout[b]):
+                    for o, h in zip(outs(blocks[b])[1:], hout[b][1:]):
                         h.copy_(o, non_blocking=True)
                     ev["out_free"][b].record(s_out)
 
         if use_graph:
-            # each block's step captured on its own input buffers
+            # each block's forward and backward captured on its own input buffers
             for b in range(2):
-                blocks[b].capture(din[b][0], din[b][1], din[b][2], W, Wr)
+                blocks[b].capture_parts(din[b][0], din[b][1], din[b][2], W, Wr)
             torch.cuda.synchronize()
         run_e2e(max(2, args.warmup))
         torch.cuda.synchronize()
@@ -365,7 +379,8 @@ def run_ours(args, cfg):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / K,
                "note": "pinned host buffers; copies on two streams overlap the "
-                       "neighbouring steps' compute (double-buffered)"
+                       "neighbouring steps' compute (double-buffered; dY's upload "
+                       "overlaps the forward, Y's download the backward)"
                        + ("; dW1, dW2 stay on the device (an optimizer step would "
                           "consume them there)" if args.full_ft else "")}
         st = ops.device_status()

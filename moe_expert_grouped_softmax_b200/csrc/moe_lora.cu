@@ -775,6 +775,9 @@ moe_status_t moe_route_topk_noalloc(const float* logits, int T, int E, int k,
 size_t moe_route_noalloc_max_workspace_bytes(void) { return kRouteScratchBytes; }
 
 // ---------------------------------------------------------- permute / combine
+#ifndef MOE_DW_ROWS
+#define MOE_DW_ROWS 1
+#endif
 // The combine (unpermute_kernel), its vector width and register budget
 // chosen from the row length.
 void launch_combine(const __nv_bfloat16* Yp, const int32_t* dest, const float* w, int T, int H,
@@ -813,6 +816,18 @@ moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
     const int grid = static_cast<int>(std::min<long long>((units + warps - 1) / warps, sms * 8));
     launch_k(kern, grid, warps * 32, 0, stream, static_cast<const __nv_bfloat16*>(X), dest, scale, T,
                                           H, k, static_cast<__nv_bfloat16*>(Xp), parts);
+  } else if (MOE_DW_ROWS && k <= 32 && H / 8 <= 32 * 16) {
+    // routing-weight gradient with the whole row in registers
+    const int vpl = permute_vpl(H / 8);
+    auto kern = vpl == 4    ? permute_dw_rows_kernel<4>
+                : vpl == 6  ? permute_dw_rows_kernel<6>
+                : vpl == 8  ? permute_dw_rows_kernel<8>
+                : vpl == 12 ? permute_dw_rows_kernel<12>
+                            : permute_dw_rows_kernel<16>;
+    const int grid = std::min((T + warps - 1) / warps, sms * 8);
+    launch_k(kern, grid, warps * 32, 0, stream, static_cast<const __nv_bfloat16*>(X), dest,
+             scale, T, H, k, static_cast<__nv_bfloat16*>(Xp),
+             static_cast<const __nv_bfloat16*>(Zp), dw);
   } else {
     const int grid = std::min((T + warps - 1) / warps, sms * 8);
     launch_k(permute_kernel, grid, warps * 32, 0, stream, 

@@ -6,14 +6,6 @@
 
 #include "ptx.cuh"
 
-// L2 cache hints: evict-first on the gather's stores / the combine's loads.
-#ifndef MOE_GATHER_STORE_HINT
-#define MOE_GATHER_STORE_HINT 0
-#endif
-#ifndef MOE_COMBINE_LOAD_HINT
-#define MOE_COMBINE_LOAD_HINT 0
-#endif
-
 namespace moe {
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
@@ -23,20 +15,6 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
                : "l"(p));
   return v;
 }
-
-// 16-byte read-only load with an L2 cache policy.
-__device__ __forceinline__ uint4 ld_nc_v4_hint(const void* p, uint64_t pol) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p), "l"(pol));
-  return v;
-}
-#if MOE_COMBINE_LOAD_HINT
-#define COMB_LD(p) ld_nc_v4_hint(p, pol_ld)
-#else
-#define COMB_LD(p) ld_nc_v4(p)
-#endif
 
 __device__ __forceinline__ uint4 ld_v4(const void* p) {
   uint4 v;
@@ -96,9 +74,6 @@ __global__ void __launch_bounds__(256, MOE_PERMUTE_MINB)
   const int nvp = (nvec + parts - 1) / parts;
   const int R = T * k;
   const long long units = static_cast<long long>(T) * parts;
-#if MOE_GATHER_STORE_HINT
-  const uint64_t pol = policy_evict_first();
-#endif
   for (long long q = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < units; q += warps) {
     const int t = static_cast<int>(q / parts);
     const int part = static_cast<int>(q - static_cast<long long>(t) * parts);
@@ -130,11 +105,7 @@ __global__ void __launch_bounds__(256, MOE_PERMUTE_MINB)
               y.z = scale2(y.z, c);
               y.w = scale2(y.w, c);
             }
-#if MOE_GATHER_STORE_HINT
-            st_global_v4_hint(orow + 16 * static_cast<size_t>(v), y, pol);
-#else
             st_v4(orow + 16 * static_cast<size_t>(v), y);
-#endif
           }
         }
       }
@@ -165,6 +136,77 @@ inline int row_parts(int T, int nvec, int warps) {
          nvec / (p + 1) >= 128)
     ++p;
   return p;
+}
+
+// The same sums as permute_kernel (below) for rows of at most 32 * kRowVec
+// vectors: the row is read once into registers (kRowVec vectors per lane),
+// then for each slot j its Zp row is loaded (all of the lane's vectors in
+// flight together), dotted with the row in the lane's vector order, the
+// scaled row stored, and the lane sums reduced across the warp in the same
+// order as permute_kernel (so dw is the same bits).  k <= 32: lane j holds
+// slot j's destination and weight.
+template <int kRowVec>
+__global__ void __launch_bounds__(256, 2)
+    permute_dw_rows_kernel(const __nv_bfloat16* __restrict__ X,
+                           const int32_t* __restrict__ dest,
+                           const float* __restrict__ scale, int T, int H, int k,
+                           __nv_bfloat16* __restrict__ Xp,
+                           const __nv_bfloat16* __restrict__ Zp,
+                           float* __restrict__ dw) {
+  griddep_sync();  // before any global memory access
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int nvec = H >> 3;
+  const int R = T * k;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+    const char* xrow = reinterpret_cast<const char*>(X + static_cast<size_t>(t) * H);
+    int my_d = -1;
+    float my_c = 1.f;
+    if (lane < k) {
+      my_d = dest[static_cast<size_t>(t) * k + lane];
+      if (scale) my_c = scale[static_cast<size_t>(t) * k + lane];
+      if (my_d < 0 || my_d >= R) {
+        set_status(5);
+        my_d = -1;
+      }
+    }
+    uint4 x[kRowVec];
+#pragma unroll
+    for (int u = 0; u < kRowVec; ++u) {
+      const int v = lane + 32 * u;
+      if (v < nvec) x[u] = ld_v4(xrow + 16 * static_cast<size_t>(v));
+    }
+    for (int j = 0; j < k; ++j) {
+      const int d = __shfl_sync(0xffffffffu, my_d, j);
+      const float c = __shfl_sync(0xffffffffu, my_c, j);
+      if (d < 0) continue;  // recorded above; the same on every lane
+      char* orow = reinterpret_cast<char*>(Xp + static_cast<size_t>(d) * H);
+      const char* zrow = reinterpret_cast<const char*>(Zp + static_cast<size_t>(d) * H);
+      uint4 z[kRowVec];
+#pragma unroll
+      for (int u = 0; u < kRowVec; ++u) {
+        const int v = lane + 32 * u;
+        if (v < nvec) z[u] = ld_nc_v4(zrow + 16 * static_cast<size_t>(v));
+      }
+      float acc = 0.f;
+#pragma unroll
+      for (int u = 0; u < kRowVec; ++u) {
+        const int v = lane + 32 * u;
+        if (v < nvec) {
+          acc += dot8(x[u], z[u]);
+          uint4 y = x[u];
+          y.x = scale2(y.x, c);
+          y.y = scale2(y.y, c);
+          y.z = scale2(y.z, c);
+          y.w = scale2(y.w, c);
+          st_v4(orow + 16 * static_cast<size_t>(v), y);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) dw[static_cast<size_t>(t) * k + j] = acc;
+    }
+  }
 }
 
 // Same with the routing-weight gradient dw[t,j] = <X[t], Zp[dest[t,j]]>.
@@ -270,9 +312,6 @@ __global__ void __launch_bounds__(256, kMinB)
     a[7] = fmaf(c, bf16_hi(z.w), a[7]);
   };
   const int v_lo = 0, v_hi = nvec;
-#if MOE_COMBINE_LOAD_HINT
-  const uint64_t pol_ld = policy_evict_first();
-#endif
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
     char* yrow = reinterpret_cast<char*>(Y + static_cast<size_t>(t) * H);
     // slots j0 .. j0 + 31 of the token on lanes 0 .. 31 (k <= 32 in one go)
@@ -323,10 +362,10 @@ __global__ void __launch_bounds__(256, kMinB)
             const int v = v0 + 32 * u;
             za[u] = zb[u] = make_uint4(0, 0, 0, 0);
             if (v < v_hi && da >= 0)
-              za[u] = COMB_LD(reinterpret_cast<const char*>(Yp + static_cast<size_t>(da) * H) +
+              za[u] = ld_nc_v4(reinterpret_cast<const char*>(Yp + static_cast<size_t>(da) * H) +
                               16 * static_cast<size_t>(v));
             if (v < v_hi && has_b && db >= 0)
-              zb[u] = COMB_LD(reinterpret_cast<const char*>(Yp + static_cast<size_t>(db) * H) +
+              zb[u] = ld_nc_v4(reinterpret_cast<const char*>(Yp + static_cast<size_t>(db) * H) +
                               16 * static_cast<size_t>(v));
           }
 #pragma unroll

@@ -499,3 +499,27 @@ class MoeBlock:
     def replay(self):
         """Run the captured step on the current stream."""
         self._graph.replay()
+
+    def capture_parts(self, X, logits, dY, W, Wr=None):
+        """Capture the forward and the backward of one step on these exact
+        tensors into two CUDA graphs (``replay_forward``, ``replay_backward``),
+        so that a caller can overlap dY's upload with the forward and Y's
+        download with the backward."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):      # one eager step off the capture
+            self.step(X, logits, dY, W, Wr)
+        torch.cuda.current_stream().wait_stream(side)
+        gf, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gf):
+            self.forward(X, logits, W, Wr)
+        with torch.cuda.graph(gb):
+            self.backward(dY, W, Wr)
+        self._graph_fwd, self._graph_bwd = gf, gb
+        return gf, gb
+
+    def replay_forward(self):
+        self._graph_fwd.replay()
+
+    def replay_backward(self):
+        self._graph_bwd.replay()

@@ -54,3 +54,25 @@ def test_graph_replay_matches_eager_step(cuda_ok, pairs):
     assert_bf16_close(graphed.Y, Y, "Y (replay on new inputs)")
     assert_bf16_close(graphed.dX, grads["dX"], "dX (replay on new inputs)")
     assert_bf16_close(graphed.dA1, grads["dA1"], "dA1 (replay on new inputs)")
+
+
+def test_forward_and_backward_graphs_match_eager_step(cuda_ok):
+    """capture_parts: the forward and the backward as two graphs, replayed in
+    turn, give the eager step's bytes."""
+    cfg = S.make_config("tiny")
+    inp = S.make_inputs(cfg)
+    g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    W = [g[n] for n in NAMES]
+    args = (cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"], cfg["r"], cfg["s"])
+    eager = ops.MoeBlock(*args)
+    eager.step(g["X"], g["logits"], g["dY"], W)
+    parts = ops.MoeBlock(*args)
+    parts.capture_parts(g["X"].clone(), g["logits"].clone(), g["dY"].clone(), W)
+    for n in OUTS:
+        getattr(parts, n).fill_(0)
+    parts.replay_forward()
+    parts.replay_backward()
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    for n in OUTS:
+        assert torch.equal(getattr(parts, n), getattr(eager, n)), n
