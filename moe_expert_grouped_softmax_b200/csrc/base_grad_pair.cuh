@@ -23,6 +23,10 @@
 
 namespace moe {
 
+#ifndef MOE_BGP_EPI_WARPS
+#define MOE_BGP_EPI_WARPS 4
+#endif
+
 struct BaseGradPairCfg {
   static constexpr int BK = 64;                      // rows (K) per stage
   static constexpr int U_BYTES = BK * 128 * 2;       // this CTA's 128 p columns
@@ -34,7 +38,10 @@ struct BaseGradPairCfg {
   static constexpr int NS_FIT = (kSmemOptin - 1024 - MISC_BYTES) / STAGE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int SMEM_BYTES = 1024 + NS * STAGE_BYTES + MISC_BYTES;
-  static constexpr int THREADS = 192;  // producer, MMA (leader), 4 epilogue warps
+  // producer, MMA (leader), epilogue warps: one per TMEM lane quarter (4), or
+  // two per quarter draining half the columns each (8)
+  static constexpr int EPI_WARPS = MOE_BGP_EPI_WARPS;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int ACC_STRIDE = 256;
   static constexpr int TMEM_COLS = 512;
   static_assert(NS >= 3, "base-gradient pair kernel stages");
@@ -86,7 +93,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BaseGradPairCfg::THR
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 2 * 4);  // both CTAs' epilogue warps
+      mbar_init(&acc_empty[i], 2 * C::EPI_WARPS);  // both CTAs' epilogue warps
     }
     mbar_init(final_bar, 1);
     mbar_init(peer_done, 1);
@@ -236,6 +243,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BaseGradPairCfg::THR
   } else {
     // ------------------------------------------------------------ epilogue
     const int ew = warp & 3;  // TMEM lane quarter this warp may access
+    const int ehalf = C::EPI_WARPS == 8 ? (warp - 2) >> 2 : 0;  // its share of the columns
     const uint32_t lane_base = static_cast<uint32_t>(ew * 32) << 16;
     const uint64_t pol = policy_evict_first();  // gradients stream out of L2
     int local = 0;
@@ -253,9 +261,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BaseGradPairCfg::THR
       const int q0 = qt * 256;
       __nv_bfloat16* orow = pr.out + (static_cast<size_t>(e) * pr.P + p) * pr.Q + q0;
       const uint32_t t_acc = tmem_base + lane_base + bb * C::ACC_STRIDE;
+      const int c_lo = C::EPI_WARPS == 8 ? ehalf * (nt >> 1) : 0;
+      const int c_hi = C::EPI_WARPS == 8 ? c_lo + (nt >> 1) : nt;
       for_chunks<256>([&](int c, auto w) {
         constexpr int W = decltype(w)::value;
-        if (c >= nt) return;
+        if (c < c_lo || c >= c_hi) return;
         float v[W];
         if (any) {
           tmem_ld<W>(t_acc + c, v);
