@@ -356,7 +356,7 @@ moe_status_t launch_grad_t(const CUtensorMap* u, const CUtensorMap* v,
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::SMEM_BYTES) != cudaSuccess)
     return MOE_ERR_CUDA;
-  const int grid = std::min(num_sms(), args.total_tiles);
+  const int grid = std::min(num_sms() * C::CTAS_PER_SM, args.total_tiles);
   if (grid <= 0) return MOE_OK;
   ProfScope prof(MOE_PROF_LORA_GRAD, st);
   launch_k(kern, grid, 192, C::SMEM_BYTES, st, u[0], u[1], u[2], u[3], v[0], v[1], v[2],
