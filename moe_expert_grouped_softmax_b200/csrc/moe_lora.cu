@@ -322,7 +322,8 @@ moe_status_t launch_pair_t(const void* A, const void* W, const void* XA, const v
                  : MODE == kDownBwd   ? MOE_PROF_DOWN_BWD
                                       : MOE_PROF_GATE_UP_BWD,
                  st);
-  launch_k(kern, 2 * pairs, C::THREADS, C::SMEM_BYTES, st, ta, tw, txa, tlb, to, to2, to3, args);
+  launch_k(kern, 2 * pairs, C::THREADS, C::SMEM_BYTES, st, ta, tw, txa, tlb, to, to2, to3,
+           args);
   count_launch();
   return launch_status();
 }
@@ -359,8 +360,8 @@ moe_status_t launch_grad_t(const CUtensorMap* u, const CUtensorMap* v,
   const int grid = std::min(num_sms() * C::CTAS_PER_SM, args.total_tiles);
   if (grid <= 0) return MOE_OK;
   ProfScope prof(MOE_PROF_LORA_GRAD, st);
-  launch_k(kern, grid, 192, C::SMEM_BYTES, st, u[0], u[1], u[2], u[3], v[0], v[1], v[2],
-                                         v[3], args);
+  launch_k(kern, grid, 192, C::SMEM_BYTES, st, u[0], u[1], u[2], u[3], v[0], v[1], v[2], v[3],
+           args);
   count_launch();
   return launch_status();
 }
@@ -506,8 +507,8 @@ moe_status_t launch_base_grad_pair(const CUtensorMap* u, const CUtensorMap* v,
   const int pairs = std::min(num_sms() / 2, args.total_tiles);
   if (pairs <= 0) return MOE_OK;
   ProfScope prof(MOE_PROF_BASE_GRAD, st);
-  launch_k(base_grad_pair_kernel, 2 * pairs, C::THREADS, C::SMEM_BYTES, st, u[0], u[1], v[0], v[1],
-                                                                      args);
+  launch_k(base_grad_pair_kernel, 2 * pairs, C::THREADS, C::SMEM_BYTES, st, u[0], u[1], v[0],
+           v[1], args);
   count_launch();
   return launch_status();
 }
@@ -738,15 +739,15 @@ moe_status_t moe_route_topk(const float* logits, int T, int E, int k, int32_t* t
   else s = launch(route_topk_kernel<16>);
   if (s != MOE_OK) return s;
   // 2. stable in-chunk ranks + chunk histograms
-  launch_k(route_rank_kernel, nblk, kRankWarps * 32, static_cast<size_t>(kRankWarps) * E * 4, st, 
-      topk_idx, R, E, blk_hist, local_rank);
+  launch_k(route_rank_kernel, nblk, kRankWarps * 32, static_cast<size_t>(kRankWarps) * E * 4,
+           st, topk_idx, R, E, blk_hist, local_rank);
   count_launch();
   if ((s = launch_status()) != MOE_OK) return s;
   // 3. expert totals, offsets and per-chunk base rows (one CTA)
   const int P = std::max(1, 1024 / E);
   const size_t smem2 = (static_cast<size_t>(P) * E + E + 1) * 4;
   launch_k(route_scan_kernel, 1, 1024, smem2, st, blk_hist, nblk, E, R, expert_counts,
-                                            expert_offsets);
+           expert_offsets);
   count_launch();
   if ((s = launch_status()) != MOE_OK) return s;
   // 4. destination rows
@@ -814,8 +815,8 @@ moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
                             : permute_rows_kernel<16>;
     const long long units = static_cast<long long>(T) * parts;
     const int grid = static_cast<int>(std::min<long long>((units + warps - 1) / warps, sms * 8));
-    launch_k(kern, grid, warps * 32, 0, stream, static_cast<const __nv_bfloat16*>(X), dest, scale, T,
-                                          H, k, static_cast<__nv_bfloat16*>(Xp), parts);
+    launch_k(kern, grid, warps * 32, 0, stream, static_cast<const __nv_bfloat16*>(X), dest,
+             scale, T, H, k, static_cast<__nv_bfloat16*>(Xp), parts);
   } else if (MOE_DW_ROWS && k <= 32 && H / 8 <= 32 * 16) {
     // routing-weight gradient with the whole row in registers
     const int vpl = permute_vpl(H / 8);
@@ -830,7 +831,7 @@ moe_status_t moe_permute(const void* X, const int32_t* dest, const float* scale,
              static_cast<const __nv_bfloat16*>(Zp), dw);
   } else {
     const int grid = std::min((T + warps - 1) / warps, sms * 8);
-    launch_k(permute_kernel, grid, warps * 32, 0, stream, 
+    launch_k(permute_kernel, grid, warps * 32, 0, stream,
         static_cast<const __nv_bfloat16*>(X), dest, scale, T, H, k,
         static_cast<__nv_bfloat16*>(Xp), static_cast<const __nv_bfloat16*>(Zp), dw);
   }
@@ -876,7 +877,7 @@ moe_status_t moe_ep_regroup(const void* in, const int32_t* counts, int N, int E_
   const int warps = kRegroupThreads / 32;
   const int grid =
       std::max(1, std::min((rows + warps - 1) / warps, std::max(1, num_sms()) * 8));
-  launch_k(ep_regroup_kernel, grid, kRegroupThreads, smem, st, 
+  launch_k(ep_regroup_kernel, grid, kRegroupThreads, smem, st,
       static_cast<const __nv_bfloat16*>(in), counts, N, E_loc, rows, H, dir,
       static_cast<__nv_bfloat16*>(out), offsets);
   count_launch();
@@ -932,7 +933,7 @@ moe_status_t moe_router_bwd(const float* w, const float* dw, const int32_t* topk
   count_launch();
   moe_status_t s;
   if ((s = launch_status()) != MOE_OK) return s;
-  launch_k(router_wgrad_kernel, dim3(E, (H + kRouterWCols - 1) / kRouterWCols), 256, 0, st, 
+  launch_k(router_wgrad_kernel, dim3(E, (H + kRouterWCols - 1) / kRouterWCols), 256, 0, st,
       static_cast<const __nv_bfloat16*>(Xp), g_row, expert_offsets, E, H, R, dWr);
   count_launch();
   if ((s = launch_status()) != MOE_OK) return s;

@@ -126,14 +126,21 @@ inline int permute_vpl(int nvp) {
 #ifndef MOE_ROW_PARTS_MAX
 #define MOE_ROW_PARTS_MAX 2
 #endif
+#ifndef MOE_ROW_PART_MIN
+#define MOE_ROW_PART_MIN 128
+#endif
+#ifndef MOE_ROW_UNITS_PER_WARP
+#define MOE_ROW_UNITS_PER_WARP 4
+#endif
 // Parts per row for the gather: enough that each of the `warps` resident
 // warps gets about four units (T tokens in all), at most MOE_ROW_PARTS_MAX,
 // and no part under 128 vectors (measured, gpt-oss-20b shape: 2 parts, 52 ->
 // 48 us per launch; the last round of whole rows left SMs idle).
 inline int row_parts(int T, int nvec, int warps) {
   int p = 1;
-  while (p < MOE_ROW_PARTS_MAX && static_cast<long long>(T) * p < 4ll * warps &&
-         nvec / (p + 1) >= 128)
+  while (p < MOE_ROW_PARTS_MAX &&
+         static_cast<long long>(T) * p < static_cast<long long>(MOE_ROW_UNITS_PER_WARP) * warps &&
+         nvec / (p + 1) >= MOE_ROW_PART_MIN)
     ++p;
   return p;
 }
