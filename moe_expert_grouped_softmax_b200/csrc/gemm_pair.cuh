@@ -117,6 +117,15 @@ __device__ __forceinline__ bool pair_half_tile(const int* s_off, int e, int mt) 
 // quarter with half the columns each: 1.5% faster on the gpt-oss-20b shape,
 // 2.5% on the Qwen3-30B-A3B one; loading the saved gate / up rows one
 // 32-column chunk ahead of their use was 25-45% slower, with either count).
+// Down-backward epilogue: the dZ1 stores of whole 32 x 32 chunks go through
+// a 2 KB shared staging tile per warp, so that each store instruction
+// covers 16 rows x 64 bytes instead of 32 rows x 32 bytes (measured: down
+// bwd 4-5% faster on the Qwen3-30B-A3B shape, 2-3% on gpt-oss-20b; staging
+// the saved gate / up loads the same way gained nothing more, and 64-column
+// chunks stored as 16 rows x 128 bytes were 10% slower).
+#ifndef MOE_DBWD_STAGED
+#define MOE_DBWD_STAGED 1
+#endif
 #ifndef MOE_PAIR_DOWN_BWD_WARPS
 #define MOE_PAIR_DOWN_BWD_WARPS 4
 #endif
@@ -147,7 +156,11 @@ struct PairCfg {
   static constexpr int SBW = MOE_PAIR_STORE_BOX;
   static constexpr int SLOT_BYTES = 32 * SBW * 2;
   static constexpr int NSTG = EPI_WARPS == 8 ? MOE_PAIR_NSTG8 : MOE_PAIR_NSTG;
-  static constexpr int RING_BYTES = kRing ? EPI_WARPS * NSTG * SLOT_BYTES : 0;
+  // down bwd: one 32-row x 64-byte staging tile per epilogue warp
+  static constexpr bool kStg = MODE == kDownBwd && MOE_DBWD_STAGED != 0;
+  static constexpr int STG_TILE = 32 * 64;
+  static constexpr int RING_BYTES =
+      kRing ? EPI_WARPS * NSTG * SLOT_BYTES : (kStg ? EPI_WARPS * STG_TILE : 0);
   static constexpr uint32_t SLOT_SWZ_SPAN = SBW * 2;  // bytes per staged row
   static constexpr int FIXED = 2 * UP_BYTES + MISC_BYTES + RING_BYTES;
   static constexpr int NS_FIT = (kSmemOptin - 1024 - FIXED) / STAGE_BYTES;
@@ -262,57 +275,107 @@ __device__ __forceinline__ void epi_swiglu_seg64(const GemmArgs& args, StoreRing
   }
 }
 
+// The saved gate and up values of W columns [col, col + W) of one row of
+// Z1 (gate at grow_p[col], up at grow_p[I + col]); zeros past nmax and for a
+// row outside the expert.  32-byte loads where the addresses allow.
+template <int W>
+struct SavedGU {
+  uint4 g[W / 8], u[W / 8];
+};
+
+template <int W>
+__device__ __forceinline__ void load_saved_gu(SavedGU<W>& sv, const __nv_bfloat16* grow_p, int I,
+                                              int col0, int nmax, bool rvalid) {
+  const bool a32 = ((reinterpret_cast<uintptr_t>(grow_p + col0) |
+                     reinterpret_cast<uintptr_t>(grow_p + I + col0)) & 31u) == 0;
+#pragma unroll
+  for (int q = 0; q < W / 8; q += 2) {
+    const int col = col0 + 8 * q;
+    sv.g[q] = sv.u[q] = make_uint4(0, 0, 0, 0);
+    if (q + 1 < W / 8) sv.g[q + 1] = sv.u[q + 1] = make_uint4(0, 0, 0, 0);
+    if (!rvalid) continue;
+    if (q + 1 < W / 8 && a32 && col + 16 <= nmax) {
+      ld_global_nc_v8(grow_p + col, sv.g[q], sv.g[q + 1]);
+      ld_global_nc_v8(grow_p + I + col, sv.u[q], sv.u[q + 1]);
+    } else {
+      if (col < nmax) {
+        sv.g[q] = *reinterpret_cast<const uint4*>(grow_p + col);
+        sv.u[q] = *reinterpret_cast<const uint4*>(grow_p + I + col);
+      }
+      if (q + 1 < W / 8 && col + 8 < nmax) {
+        sv.g[q + 1] = *reinterpret_cast<const uint4*>(grow_p + col + 8);
+        sv.u[q + 1] = *reinterpret_cast<const uint4*>(grow_p + I + col + 8);
+      }
+    }
+  }
+}
+
+// Byte offset of 16-byte unit u (columns 8u .. 8u + 7) of row r in a
+// 32-row x 64-byte staging tile; the unit index is XORed with bits 1-2 of
+// the row, so that a warp's 16-byte accesses, one row per lane or two lanes
+// per row, fall in distinct banks within each 8-lane phase.
+__device__ __forceinline__ uint32_t stg_off(int r, int u) {
+  return static_cast<uint32_t>(r * 64 + ((u ^ ((r >> 1) & 3)) << 4));
+}
+
+// Stores 32 bf16 columns [col, col + 32) of the warp's 32 rows y0 .. y0 + 31
+// (this thread's row, v, rounded as the per-row stores round it) through the
+// warp's staging tile: lane l then writes 32 bytes (half l % 2) of rows l / 2
+// and l / 2 + 16, so that each store instruction covers 16 rows x 64 bytes
+// instead of 32 rows x 32 bytes.  All 32 rows and columns must be in range
+// and every row piece 32-byte aligned.  Warp-wide.
+template <class Args>
+__device__ __forceinline__ void store_rows_staged32(const Args& args, uint8_t* stg, const float* v,
+                                                    int y0, size_t col, uint64_t pol, int lane) {
+  __syncwarp();  // the tile's previous reads are done
+#pragma unroll
+  for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(stg + stg_off(lane, q)) = pack8(v + 8 * q);
+  __syncwarp();
+  const int rr = lane >> 1, hh = lane & 1;
+  const uint4 a0 = *reinterpret_cast<const uint4*>(stg + stg_off(rr, 2 * hh));
+  const uint4 a1 = *reinterpret_cast<const uint4*>(stg + stg_off(rr, 2 * hh + 1));
+  const uint4 b0 = *reinterpret_cast<const uint4*>(stg + stg_off(rr + 16, 2 * hh));
+  const uint4 b1 = *reinterpret_cast<const uint4*>(stg + stg_off(rr + 16, 2 * hh + 1));
+  const size_t ra = static_cast<size_t>(y0 + rr);
+  st_global_v8_hint(args.out + ra * args.ld_out + col + 16 * hh, a0, a1, pol);
+  st_global_v8_hint(args.out + (ra + 16) * args.ld_out + col + 16 * hh, b0, b1, pol);
+}
+
 // Epilogue of the other modes for NC accumulator columns (this warp's share
 // of them with kSplit): tile column j of the drained range sits at TMEM
 // column t_acc + j and is output column col0 + j; nothing at or past hi
 // (the end of the tile's columns) or args.N is written.  Plain store (down
 // fwd: Z2, gate_up bwd: dXp, through tmO) or SwiGLU backward (down bwd:
 // reads the saved gate / up, writes dZ1 = [dg | du] through tmO / tmU).
-template <int MODE, int NC, bool kSplit, bool kRing, int SBW, int NSTG>
+template <int MODE, int NC, bool kSplit, bool kRing, bool C_STG, int SBW, int NSTG>
 __device__ __forceinline__ void epi_pair_drain(const GemmArgs& args, StoreRing<SBW, NSTG>& ring,
-                                               const CUtensorMap* tmO, const CUtensorMap* tmU,
-                                               uint32_t t_acc, int grow, int y0, bool rows_all,
-                                               bool rvalid, int ehalf, int col0, int hi,
-                                               uint64_t pol, int lane) {
+                                               uint8_t* stg, const CUtensorMap* tmO,
+                                               const CUtensorMap* tmU, uint32_t t_acc, int grow,
+                                               int y0, bool rows_all, bool rvalid, int ehalf,
+                                               int col0, int hi, uint64_t pol, int lane) {
   const int nmax = min(args.N, hi);
   __nv_bfloat16* orow = args.out + static_cast<size_t>(grow) * args.ld_out;
   if constexpr (MODE == kDownBwd) {
     const __nv_bfloat16* grow_p = args.aux + static_cast<size_t>(grow) * args.ld_aux;
+    // staged stores need 32-byte aligned row pieces of dZ1
+    bool stg_ok = false;
+    if constexpr (C_STG) {
+      const __nv_bfloat16* o0 = args.out + static_cast<size_t>(y0) * args.ld_out + col0;
+      stg_ok = (reinterpret_cast<uintptr_t>(o0) & 31u) == 0 && ((args.ld_out | args.I) & 15) == 0;
+    }
     for_my_chunks<NC, kSplit>(ehalf, [&](int c, auto w) {
       constexpr int W = decltype(w)::value;
-      uint4 gv[W / 8], uv[W / 8];
-      // loads first (in flight during the TMEM read), 32 bytes at a time
-      // where the address allows
-      const bool a32 = ((reinterpret_cast<uintptr_t>(grow_p + col0 + c) |
-                         reinterpret_cast<uintptr_t>(grow_p + args.I + col0 + c)) & 31u) == 0;
-#pragma unroll
-      for (int q = 0; q < W / 8; q += 2) {
-        const int col = col0 + c + 8 * q;
-        gv[q] = uv[q] = make_uint4(0, 0, 0, 0);
-        if (q + 1 < W / 8) gv[q + 1] = uv[q + 1] = make_uint4(0, 0, 0, 0);
-        if (!rvalid) continue;
-        if (q + 1 < W / 8 && a32 && col + 16 <= nmax) {
-          ld_global_nc_v8(grow_p + col, gv[q], gv[q + 1]);
-          ld_global_nc_v8(grow_p + args.I + col, uv[q], uv[q + 1]);
-        } else {
-          if (col < nmax) {
-            gv[q] = *reinterpret_cast<const uint4*>(grow_p + col);
-            uv[q] = *reinterpret_cast<const uint4*>(grow_p + args.I + col);
-          }
-          if (q + 1 < W / 8 && col + 8 < nmax) {
-            gv[q + 1] = *reinterpret_cast<const uint4*>(grow_p + col + 8);
-            uv[q + 1] = *reinterpret_cast<const uint4*>(grow_p + args.I + col + 8);
-          }
-        }
-      }
+      const int col = col0 + c;
+      SavedGU<W> sv;  // loads first (in flight during the TMEM read)
+      load_saved_gu<W>(sv, grow_p, args.I, col, nmax, rvalid);
       float dh[W];
       tmem_ld<W>(t_acc + c, dh);
       tmem_ld_wait();
       float dg[W], du[W];
 #pragma unroll
       for (int q = 0; q < W / 8; ++q) {
-        const uint32_t ga[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
-        const uint32_t ua[4] = {uv[q].x, uv[q].y, uv[q].z, uv[q].w};
+        const uint32_t ga[4] = {sv.g[q].x, sv.g[q].y, sv.g[q].z, sv.g[q].w};
+        const uint32_t ua[4] = {sv.u[q].x, sv.u[q].y, sv.u[q].z, sv.u[q].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
 #pragma unroll
@@ -326,7 +389,14 @@ __device__ __forceinline__ void epi_pair_drain(const GemmArgs& args, StoreRing<S
           }
         }
       }
-      const int col = col0 + c;
+      if constexpr (C_STG && W == 32) {
+        // a whole chunk of the warp's 32 rows, all inside the expert
+        if (rows_all && col + 32 <= nmax && stg_ok) {
+          store_rows_staged32(args, stg, dg, y0, col, pol, lane);
+          store_rows_staged32(args, stg, du, y0, static_cast<size_t>(col) + args.I, pol, lane);
+          return;
+        }
+      }
       pair_out_chunk<W, kRing>(ring, tmO, orow, dg, col, y0, rows_all, rvalid, hi, args.N, pol,
                                lane);
       pair_out_chunk<W, kRing>(ring, tmU, orow + args.I, du, col, y0, rows_all, rvalid, hi,
@@ -620,6 +690,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
     const uint32_t lane_base = static_cast<uint32_t>(ew * 32) << 16;
     const uint64_t pol = policy_evict_first();  // outputs stream out of L2
     StoreRing<C::SBW, C::NSTG> ring{sRing + (warp - 2) * C::NSTG * C::SLOT_BYTES, 0};
+    uint8_t* stg = sRing + (warp - 2) * C::STG_TILE;  // down bwd staging (kStg)
     int local = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++local) {
       int e, mt, nt;
@@ -659,12 +730,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<MODE, RK>::T
         // Nt (or past N) hold nothing of this tile and are not stored
         if (half) {
           const int q = ew >> 1;
-          epi_pair_drain<MODE, BN / 2, kSplit, C::kRing>(args, ring, &tmO, &tmO3, t_acc, grow, y0,
-                                               rows_all, rvalid, ehalf, col0 + q * NHt,
-                                               col0 + (q + 1) * NHt, pol, lane);
+          epi_pair_drain<MODE, BN / 2, kSplit, C::kRing, C::kStg>(
+              args, ring, stg, &tmO, &tmO3, t_acc, grow, y0, rows_all, rvalid, ehalf,
+              col0 + q * NHt, col0 + (q + 1) * NHt, pol, lane);
         } else {
-          epi_pair_drain<MODE, BN, kSplit, C::kRing>(args, ring, &tmO, &tmO3, t_acc, grow, y0, rows_all,
-                                           rvalid, ehalf, col0, col0 + Nt, pol, lane);
+          epi_pair_drain<MODE, BN, kSplit, C::kRing, C::kStg>(args, ring, stg, &tmO, &tmO3, t_acc,
+                                                            grow, y0, rows_all, rvalid, ehalf,
+                                                            col0, col0 + Nt, pol, lane);
         }
       }
       tc_fence_before();
